@@ -1,0 +1,215 @@
+/*
+ * mhc.h - C ABI of the B200 (sm_100a) mHC decode boundary library, libmhc.so.
+ *
+ * The boundary sits between two decoder sublayers of a DeepSeek-V4-style decode
+ * step. It reduces the previous sublayer's output into the hc_mult residual
+ * streams (mHC post), collapses and RMS-normalises the streams into the next
+ * sublayer's input (mHC pre), optionally as MXFP8, and computes the next mHC
+ * coefficients. Sources, by page title and section:
+ *   [boundary]   vllm ...specialized_decode.boundary.boundary:
+ *                Boundaries.first / sublayer / post_only / _pre / _reduce,
+ *                BoundaryState, empty_quantized_layer_input
+ *   [all_reduce] vllm ...specialized_decode.boundary.all_reduce:
+ *                BoundaryAllReduce.__call__ / finalize
+ *   [decode]     vllm ...specialized_decode.runtime.decode:
+ *                SpecializedDecode.run (the layer loop), _head
+ *
+ * Notation: R = rows (decode tokens), H = hidden, n = hc_mult, K = n*H,
+ * C = 2n + n^2 (coefficient logits), P = partial buffers, k = top_k.
+ *
+ * Conventions shared by every entry point
+ *   - bf16 tensors are passed as mhc_bf16 (the raw 16-bit pattern), fp32 as
+ *     float, all row-major and contiguous unless a stride is given.
+ *   - Every pointer is a DEVICE pointer owned by the caller. The library never
+ *     allocates, frees or keeps a pointer after the call returns.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and
+ *     do not synchronise the host. Host-side argument checks happen before any
+ *     launch; a call that returns an error launched nothing.
+ *   - Errors are returned, never raised or aborted on. Errors found by a kernel
+ *     (a wait that ran out, a gather index out of range) are recorded in the
+ *     workspace and read with mhc_get_device_status.
+ *   - Shapes: 1 <= R <= 128, H a multiple of 64 with H/64 no larger than the
+ *     number of co-resident blocks of the GPU (148 on B200, so H <= 9472),
+ *     n in {1, 2, 4}, 1 <= P <= 16, 1 <= k <= 16.
+ *   - Alignment: bf16 tensors and fn 16-byte aligned, MXFP8 data 8-byte aligned,
+ *     fp32 vectors 4-byte aligned; partial_stride a multiple of 8 elements.
+ *   - residual_out may be the same buffer as residual (in place) but must not
+ *     partially overlap it. No other output may overlap any input.
+ */
+#ifndef MHC_H
+#define MHC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MHC_API __attribute__((visibility("default")))
+#else
+#define MHC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mhc_bf16;         /* bfloat16 bit pattern */
+typedef struct CUstream_st* mhc_stream; /* the same type as cudaStream_t */
+
+typedef enum {
+  MHC_OK = 0,
+  MHC_ERR_INVALID_ARG = 1,       /* NULL where required, bad alignment, eps < 0 ... */
+  MHC_ERR_UNSUPPORTED_SHAPE = 2, /* rows/hidden/hc_mult/P/top_k outside the limits */
+  MHC_ERR_WORKSPACE = 3,         /* workspace NULL, misaligned or too small */
+  MHC_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, query) */
+  MHC_ERR_DEVICE_TIMEOUT = 5,    /* device: a cross-block wait gave up */
+  MHC_ERR_DEVICE_INDEX = 6       /* device: expanded_idx_to_permuted_idx past the end */
+} mhc_status;
+
+/* Weights and scalars of the next-coefficient step, as the stock mHC pre takes
+ * them ([boundary] Boundaries.sublayer passes fn, scale, base, rms_norm_eps,
+ * hc_eps, hc_eps, hc_post_alpha, hc_sinkhorn_iters).
+ *   fn    [n*H, C] fp32; row k = j*H + h is stream j, column h of a row's streams.
+ *         Columns: [pre 0..n-1 | post n..2n-1 | comb 2n..], comb column
+ *         2n + j*n + i is comb[j][i] (stream j into stream i).
+ *   scale [3] fp32, one per group pre / post / comb.
+ *   base  [C] fp32.
+ * Per row r, with v the row's streams flattened to K values:
+ *   inv  = 1/sqrt(mean(v^2) + rms_eps);  l_c = scale[group c] * inv * (v . fn[:,c]) + base[c]
+ *   pre  = sigmoid(l_pre) + pre_eps;     post = post_alpha * sigmoid(l_post)
+ *   comb = Sinkhorn(l_comb, sinkhorn_iters, sinkhorn_eps):
+ *          M = exp(L - max L); repeat: rows /= (row sum + eps), then columns /= (column sum + eps).
+ * Constraints: eps values >= 0, 0 <= sinkhorn_iters <= 1000. */
+typedef struct {
+  const float* fn;
+  const float* scale;
+  const float* base;
+  float rms_eps;
+  float pre_eps;
+  float sinkhorn_eps;
+  float post_alpha;
+  int sinkhorn_iters;
+} mhc_coeff_args;
+
+/* MXFP8 layer input ([boundary] empty_quantized_layer_input: E4M3 data [R, H] and
+ * a uint8 scale buffer in FlashInfer's swizzled 128x4 layout).
+ *   data  [R, H] E4M3 bytes (OCP "fn" variant), RNE, saturating to +-448.
+ *   scale E8M0 bytes, one per 32 consecutive elements of a row, e = the smallest
+ *         integer with amax <= 448 * 2^e (clamped to [-127, 127]), byte e + 127.
+ *         swizzled_128x4 != 0: mhc_mxfp8_scale_bytes(R, H, 1) bytes; the [R, H/32]
+ *         scale matrix padded to 128-row x 4-column tiles of 512 bytes, tiles in
+ *         row-major order, (r, c) inside a tile at (r%32)*16 + (r/32)*4 + c;
+ *         padding bytes are written as 0.
+ *         swizzled_128x4 == 0: linear [R, H/32].
+ *   A block holding NaN or Inf is out of contract: scale 0xFF, data 0x7F. */
+typedef struct {
+  uint8_t* data;
+  uint8_t* scale;
+  int swizzled_128x4;
+} mhc_mxfp8_out;
+
+/* Bytes of workspace the boundary entry points need for (rows, hidden, hc_mult).
+ * A workspace sized for R rows serves every call with rows <= R and the same
+ * hidden and hc_mult. It must be 256-byte aligned, zeroed once before first use
+ * (mhc_workspace_init) and used by one stream at a time: calls sharing a
+ * workspace must not overlap on the GPU. Returns 0 for unsupported shapes. */
+MHC_API size_t mhc_workspace_bytes(int rows, int hidden, int hc_mult);
+
+/* Bytes of the MXFP8 scale buffer: roundup(R,128) * roundup(H/32, 4) when
+ * swizzled, R * H/32 when linear. Returns 0 for H not a multiple of 32. */
+MHC_API size_t mhc_mxfp8_scale_bytes(int rows, int hidden, int swizzled_128x4);
+
+/* Zero the workspace on `stream` (cudaMemsetAsync). Needed once before first use
+ * and again after a call reported MHC_ERR_DEVICE_TIMEOUT. */
+MHC_API mhc_status mhc_workspace_init(void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* Full boundary after a sublayer with TP-partial output ([all_reduce]
+ * BoundaryAllReduce.__call__, [boundary] Boundaries.sublayer / _reduce):
+ *   x[r,h]        = sum_p partials[p*partial_stride + r*H + h]      (fp32)
+ *   new[r,i,h]    = bf16( sum_j comb[r,j,i]*residual[r,j,h] + post[r,i]*x[r,h] )
+ *   residual_out  = new                                              [R, n, H]
+ * and when pre != NULL (pre is the pre-mix carried from the previous boundary,
+ * [boundary] BoundaryState.pre):
+ *   c[r,h]        = sum_j pre[r,j]*new[r,j,h]
+ *   layer_input   = bf16( c * rsqrt(mean_h c^2 + norm_eps) * norm_weight[h] )  [R, H]
+ *   mxfp8 (optional, may be NULL) = MXFP8 of layer_input
+ *   coeffs (optional, may be NULL) -> post_out [R,n], comb_out [R,n,n], pre_out [R,n]
+ *     computed from the new streams (see mhc_coeff_args).
+ * pre == NULL is the residual-only variant ([boundary] Boundaries._reduce with no
+ * pre and no norm): then norm_weight, layer_input, mxfp8 and coeffs must be NULL.
+ * Inputs post [R,n], comb [R,n,n], pre [R,n] are fp32; norm_weight [H] bf16.
+ * workspace: see mhc_workspace_bytes. */
+MHC_API mhc_status mhc_boundary_post_pre(
+    const mhc_bf16* partials, int num_partials, int64_t partial_stride,
+    const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
+    const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+    mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    float* post_out, float* comb_out, float* pre_out,
+    int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* Boundary after a MoE sublayer whose output was left unfinalized ([all_reduce]
+ * BoundaryAllReduce.finalize, [boundary] Boundaries._reduce):
+ *   x[r,h] = shared_output[r,h] + sum_t expert_weights[r*top_k+t] *
+ *            gemm2_permuted[e2p[r*top_k+t]*H + h]
+ * with e2p = expanded_idx_to_permuted_idx [R*top_k] int32: an entry < 0 adds
+ * nothing; an entry >= num_permuted adds nothing and records
+ * MHC_ERR_DEVICE_INDEX. gemm2_permuted [num_permuted, H] bf16, expert_weights
+ * [R, top_k] fp32, shared_output [R, H] bf16. Everything after x is as in
+ * mhc_boundary_post_pre, including the residual-only variant (pre == NULL). */
+MHC_API mhc_status mhc_boundary_moe_finalize(
+    const mhc_bf16* gemm2_permuted, int num_permuted, const float* expert_weights,
+    const int32_t* expanded_idx_to_permuted_idx, int top_k, const mhc_bf16* shared_output,
+    const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
+    const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+    mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    float* post_out, float* comb_out, float* pre_out,
+    int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* Residual-only boundary ([boundary] Boundaries.post_only: all-reduce then mHC
+ * post, streams only): residual_out = bf16(comb-mix of residual + post * sum of
+ * partials). Needs no workspace. */
+MHC_API mhc_status mhc_boundary_residual_only(
+    const mhc_bf16* partials, int num_partials, int64_t partial_stride,
+    const mhc_bf16* residual, const float* post, const float* comb,
+    mhc_bf16* residual_out, int rows, int hidden, int hc_mult, mhc_stream stream);
+
+/* The stock mHC pre without a reduction ([boundary] Boundaries._pre), two forms:
+ *   residual != NULL, x == NULL: coefficients of the given streams [R, n, H]; with
+ *     layer_input != NULL also the layer input from pre_mix [R, n] (required then).
+ *   x != NULL, residual == NULL: the first layer ([boundary] Boundaries.first). The
+ *     embedding x [R, H] is broadcast to the n streams; the identity pre-mix
+ *     selects stream 0, so layer_input = bf16(x * rsqrt(mean x^2 + norm_eps) * w).
+ *     pre_mix must be NULL. residual_out (may be NULL) receives the broadcast
+ *     streams [R, n, H]. The coefficients are those of the broadcast streams with
+ *     fn [n*H, C] (the first layer's hc_attn_fn_broadcast).
+ * post_out, comb_out and pre_out are always written. */
+MHC_API mhc_status mhc_coeffs(
+    const mhc_bf16* residual, const mhc_coeff_args* coeffs, const float* pre_mix,
+    const mhc_bf16* x, mhc_bf16* residual_out,
+    const mhc_bf16* norm_weight, float norm_eps, mhc_bf16* layer_input,
+    float* post_out, float* comb_out, float* pre_out,
+    int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* MXFP8 of a bf16 [R, H] matrix (x, row-major, 16-byte aligned), same encoding
+ * and scale layouts as mhc_mxfp8_out. 1 <= R <= 65535, H a multiple of 32. */
+MHC_API mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden,
+                               const mhc_mxfp8_out* out, mhc_stream stream);
+
+/* Wait for `stream`, then read and clear the error a kernel recorded in
+ * `workspace` (MHC_OK when none). The only entry point that synchronises. */
+MHC_API mhc_status mhc_get_device_status(void* workspace, mhc_stream stream);
+
+/* Static, human-readable name of a status code. */
+MHC_API const char* mhc_status_string(mhc_status status);
+
+/* Test hook for the bounded waits: `budget_ns` > 0 sets the time a block waits
+ * at a cross-block barrier before giving up (default 1e9 ns); `extra_arrivals`
+ * makes the barrier expect that many blocks beyond the grid, so that it can
+ * never complete and every wait runs out. Affects launches made after the call
+ * by this process. Returns the previous budget. */
+MHC_API int64_t mhc_debug_set_wait(int64_t budget_ns, int extra_arrivals);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MHC_H */

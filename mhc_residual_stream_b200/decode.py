@@ -1,0 +1,177 @@
+"""The boundaries of one decode step's layer loop, on the CUDA library.
+
+Mirrors the layer loop of vllm ...specialized_decode.runtime.decode,
+SpecializedDecode.run, with the sublayers (attention, MoE) replaced by seeded
+synthetic outputs: per layer the attention entry (the first layer's broadcast,
+else the finalize of the previous MoE output with an MXFP8 layer input), the
+attention's TP-partial output, the FFN entry (the partial sum, bf16 layer
+input) and the MoE's unfinalized output; after the last layer the
+residual-only finalize that feeds the final collapse. The streams and the
+post / comb / pre mixes chain from boundary to boundary as in BoundaryState.
+
+Every boundary has its own seeded fn, scale, base and norm_weight, so the
+weights a step reads exceed the L2 cache and come from HBM.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import torch
+
+from . import mhc as M
+from . import synthetic as S
+
+
+@dataclass
+class BoundaryWeights:
+    coeffs: M.Coeffs
+    norm_weight: torch.Tensor
+
+
+@dataclass
+class Pending:
+    kind: str  # "partials" or "moe"
+    partials: Optional[torch.Tensor] = None
+    gemm2_permuted: Optional[torch.Tensor] = None
+    expert_weights: Optional[torch.Tensor] = None
+    e2p: Optional[torch.Tensor] = None
+    shared_output: Optional[torch.Tensor] = None
+
+
+@dataclass
+class Step:
+    """One boundary of the schedule."""
+    kind: str            # "first", "attn", "ffn", "final"
+    layer: int
+    weights: Optional[BoundaryWeights]
+    pending: Optional[Pending]
+    mxfp8: bool
+    src: int = 0         # state slot read
+    dst: int = 0         # state slot written
+
+
+@dataclass
+class DecodeLoop:
+    rows: int
+    hidden: int = 7168
+    hc_mult: int = 4
+    layers: int = 61
+    partials: int = 8
+    top_k: int = 8
+    seed: int = 5000
+    device: str = "cuda"
+    steps: List[Step] = field(default_factory=list)
+
+    def __post_init__(self):
+        R, H, n, dev = self.rows, self.hidden, self.hc_mult, self.device
+        s0 = self.seed
+        first = S.draw_first_layer(R, H, n=n, seed=s0)
+        self.x = first["x"].to(dev)
+        # state slots: streams and mixes, ping-pong between boundaries
+        self.res = [torch.empty(R, n, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.post = [torch.empty(R, n, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.comb = [torch.empty(R, n, n, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.pre = [torch.empty(R, n, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.layer_input = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+        self.q_data = torch.empty(R, H, dtype=torch.uint8, device=dev)
+        self.q_scale = torch.empty(M.mhc_mxfp8_scale_bytes(R, H, True), dtype=torch.uint8, device=dev)
+        self.workspace = M.new_workspace(R, H, n, dev)
+
+        def weights(seed):
+            g = S.gen(seed)
+            cw = S.draw_coeff_weights(g, H, n, 0.01, affine=True)
+            nw = (1.0 + torch.randn(H, generator=g) * 0.1).to(torch.bfloat16)
+            return BoundaryWeights(M.Coeffs.from_weights(cw, dev), nw.to(dev))
+
+        def attn_pending(seed):
+            g = S.gen(seed)
+            p = (torch.randn(self.partials, R, H, generator=g) * 0.05).to(torch.bfloat16)
+            return Pending("partials", partials=p.to(dev))
+
+        def moe_pending(seed):
+            d = S.draw_moe(R, H, n=n, top_k=self.top_k, seed=seed)
+            return Pending("moe", gemm2_permuted=d["gemm2_permuted"].to(dev),
+                           expert_weights=d["expert_weights"].to(dev),
+                           e2p=d["expanded_idx_to_permuted_idx"].to(dev),
+                           shared_output=d["shared_output"].to(dev))
+
+        steps = []
+        slot = 0
+        prev_moe = None
+        for layer in range(self.layers):
+            base = s0 + 10 * (layer + 1)
+            if layer == 0:
+                steps.append(Step("first", 0, weights(base + 1), None, False, src=0, dst=0))
+            else:
+                steps.append(Step("attn", layer, weights(base + 1), prev_moe, True, src=slot, dst=1 - slot))
+                slot = 1 - slot
+            attn_out = attn_pending(base + 2)
+            steps.append(Step("ffn", layer, weights(base + 3), attn_out, False, src=slot, dst=1 - slot))
+            slot = 1 - slot
+            prev_moe = moe_pending(base + 4)
+        steps.append(Step("final", self.layers, None, prev_moe, False, src=slot, dst=1 - slot))
+        self.steps = steps
+        self.final_slot = 1 - slot
+
+    # ------------------------------------------------------------------ running
+
+    def run_step(self, st: Step, stream=None):
+        ws = self.workspace
+        if st.kind == "first":
+            M.mhc_coeffs(st.weights.coeffs, self.post[st.dst], self.comb[st.dst], self.pre[st.dst], x=self.x,
+                         residual_out=self.res[st.dst], norm_weight=st.weights.norm_weight, norm_eps=1e-6,
+                         layer_input=self.layer_input, workspace=ws, stream=stream)
+            return
+        a, b = st.src, st.dst
+        final = st.kind == "final"
+        w = st.weights
+        q = (self.q_data, self.q_scale, True) if st.mxfp8 else None
+        if st.pending.kind == "partials":
+            M.mhc_boundary_post_pre(st.pending.partials, self.res[a], self.post[a], self.comb[a], self.pre[a],
+                                    w.norm_weight, 1e-6, w.coeffs, self.res[b], layer_input=self.layer_input,
+                                    mxfp8=q, post_out=self.post[b], comb_out=self.comb[b], pre_out=self.pre[b],
+                                    workspace=ws, stream=stream)
+        else:
+            pd = st.pending
+            M.mhc_boundary_moe_finalize(
+                pd.gemm2_permuted, pd.expert_weights, pd.e2p, pd.shared_output, self.res[a], self.post[a],
+                self.comb[a], None if final else self.pre[a], None if final else w.norm_weight, 1e-6,
+                None if final else w.coeffs, self.res[b], layer_input=None if final else self.layer_input,
+                mxfp8=q, post_out=None if final else self.post[b], comb_out=None if final else self.comb[b],
+                pre_out=None if final else self.pre[b], workspace=ws, stream=stream)
+
+    def run(self, stream=None):
+        """Enqueue every boundary of the step on `stream` (no host synchronisation)."""
+        for st in self.steps:
+            self.run_step(st, stream)
+
+    def streams(self) -> torch.Tensor:
+        """The residual streams after the final residual-only boundary."""
+        return self.res[self.final_slot]
+
+    def algorithmic_bytes(self) -> int:
+        """Bytes each boundary must move (inputs read once, outputs written once), summed."""
+        R, H, n = self.rows, self.hidden, self.hc_mult
+        C = 2 * n + n * n
+        total = 0
+        for st in self.steps:
+            b = 0
+            fn_b = n * H * C * 4 + (3 + C) * 4
+            mix_in = R * (2 * n + n * n) * 4
+            coeff_out = R * (2 * n + n * n) * 4
+            if st.kind == "first":
+                b = R * H * 2 + R * n * H * 2 + R * H * 2 + fn_b + H * 2 + coeff_out
+            else:
+                if st.pending.kind == "partials":
+                    b += self.partials * R * H * 2
+                else:
+                    b += (R * self.top_k + R) * H * 2 + R * self.top_k * 8
+                b += 2 * R * n * H * 2 + mix_in
+                if st.kind != "final":
+                    b += R * H * 2 + H * 2 + fn_b + coeff_out
+                    if st.mxfp8:
+                        b += R * H + M.mhc_mxfp8_scale_bytes(R, H, True)
+            total += b
+        return total
