@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Benchmark of the mHC decode boundary on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-sweep]
+
+A step is one decode attention-side boundary at rows=32, H=7168, hc_mult=4 with
+8 bf16 TP-partials, an MXFP8 layer input (swizzled 128x4 scales) and the next
+coefficients (20 Sinkhorn iterations): the partial sum, post-mix, collapse +
+RMSNorm + MXFP8 and coefficient steps of the boundary in one launch. Inputs are
+seeded synthetic tensors of that shape, resident in HBM; enough distinct buffer
+sets (inputs, weights and outputs; 27 sets, ~0.29 GB, at rows 32) to exceed
+twice the 126 MB L2 are
+rotated so that every step reads HBM, not L2. Steps are replayed from CUDA
+graphs and timed with CUDA events on the launching stream; the metric is
+microseconds per boundary (lower is better) and the achieved HBM GB/s of the
+algorithmic bytes (each input read once, each output written once).
+
+Also reported on the same JSON line: the rows sweep 1..128 of the same boundary,
+one decode step of the layer loop (61 layers: 123 chained boundaries), the
+end-to-end time through the C ABI with host buffers (copies included), the CPU
+oracle on the machine's host cores, and the SM clocks sampled during the timed region.
+
+With --gpus N > 1 (one process per GPU under torchrun) every rank runs its own
+replica of the workload (the boundary has no exchange step on one GPU's decode
+batch); the value is the aggregate time per boundary, max over ranks.
+
+--impl reference times the CPU oracle (the float64 restatement of the method)
+as the reference arm, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+ROWS, HIDDEN, HC, PARTIALS = 32, 7168, 4, 8
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "µs/boundary and achieved HBM GB/s (% of B200 peak) at rows 1–128, H=7168, n=4"
+
+
+def boundary_bytes(R, H=HIDDEN, n=HC, P=PARTIALS, mxfp8=True, coeff=True, scale_bytes=None):
+    """Algorithmic bytes of one partial-sum boundary: each input read once, each output written once."""
+    C = 2 * n + n * n
+    b = P * R * H * 2            # partials
+    b += R * n * H * 2 * 2       # residual in + out
+    b += R * (2 * n + n * n) * 4  # post, comb, pre
+    b += H * 2 + R * H * 2       # norm_weight, layer_input
+    if coeff:
+        b += n * H * C * 4 + (3 + C) * 4 + R * (2 * n + n * n) * 4  # fn, scale, base; coefficients out
+    if mxfp8:
+        b += R * H + (scale_bytes if scale_bytes is not None else ((R + 127) // 128 * 128) * ((H // 32 + 3) // 4 * 4))
+    return b
+
+
+def sets_for(R):
+    """Distinct buffer sets so that one pass over them moves more than twice the L2 size."""
+    return max(4, -(-int(2.2 * L2_BYTES) // boundary_bytes(R)))
+
+
+def load_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic():
+    """DRAM bytes per launch of the boundary kernel from the committed ncu summary,
+    or None when the kernel sources changed since it was taken."""
+    from mhc_residual_stream_b200 import build
+    p = os.path.join(ROOT, "profiles", "boundary_kernel_traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        if t.get("source_sha256") == build.source_digest():
+            return t.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.ident = None
+
+    def start(self):
+        if self.ident is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- our arm
+
+class BoundarySet:
+    """Device buffers of one boundary of the benchmark workload."""
+
+    def __init__(self, R, seed, device, mxfp8=True):
+        from mhc_residual_stream_b200 import mhc as M
+        from mhc_residual_stream_b200 import synthetic as S
+        d = S.draw_boundary(R, HIDDEN, n=HC, partials=PARTIALS, seed=seed)
+        self.host = d
+        self.partials = d["partials"].to(device)
+        self.residual = d["residual"].to(device)
+        self.post = d["post"].to(device)
+        self.comb = d["comb"].to(device)
+        self.pre = d["pre"].to(device)
+        self.norm_weight = d["norm_weight"].to(device)
+        self.coeffs = M.Coeffs.from_weights(d["coeff"], device)
+        self.residual_out = torch.empty_like(self.residual)
+        self.layer_input = torch.empty(R, HIDDEN, dtype=torch.bfloat16, device=device)
+        self.q_data = torch.empty(R, HIDDEN, dtype=torch.uint8, device=device) if mxfp8 else None
+        self.q_scale = (torch.empty(M.mhc_mxfp8_scale_bytes(R, HIDDEN, True), dtype=torch.uint8, device=device)
+                        if mxfp8 else None)
+        self.post_out = torch.empty_like(self.post)
+        self.comb_out = torch.empty_like(self.comb)
+        self.pre_out = torch.empty_like(self.pre)
+
+    def launch(self, ws, stream=None):
+        from mhc_residual_stream_b200 import mhc as M
+        M.mhc_boundary_post_pre(self.partials, self.residual, self.post, self.comb, self.pre, self.norm_weight,
+                                1e-6, self.coeffs, self.residual_out, layer_input=self.layer_input,
+                                mxfp8=None if self.q_data is None else (self.q_data, self.q_scale, True),
+                                post_out=self.post_out, comb_out=self.comb_out, pre_out=self.pre_out,
+                                workspace=ws, stream=stream)
+
+
+def capture(fn, n):
+    """A CUDA graph of n calls of fn(i)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(0)  # a launch outside the capture on the capture's stream (initialisation)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    return g
+
+
+def timed_graph_steps(sets, ws, steps, warmup, graph_len=240):
+    """Run `warmup` then time `steps` boundaries (rotating over `sets`) from CUDA graphs;
+    returns elapsed ms of the timed region on the launching stream."""
+    nset = len(sets)
+    main = capture(lambda i: sets[i % nset].launch(ws), graph_len)
+    tail_len = steps % graph_len
+    tail = capture(lambda i: sets[i % nset].launch(ws), tail_len) if tail_len else None
+    wgraph = capture(lambda i: sets[i % nset].launch(ws), max(1, min(warmup, graph_len)))
+    for _ in range(max(1, (warmup + graph_len - 1) // graph_len)):
+        wgraph.replay()
+    torch.cuda.synchronize()
+    return main, tail
+
+
+def run_timed(main, tail, steps, graph_len, sampler=None):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    torch.cuda._sleep(2_000_000)  # keep the GPU busy while the replays are queued behind the start event
+    start.record()
+    for _ in range(steps // graph_len):
+        main.replay()
+    if tail is not None:
+        tail.replay()
+    end.record()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.stop()
+    return start.elapsed_time(end)
+
+
+def e2e_time(bset, ws, steps, device):
+    """Per boundary through the C ABI with host buffers: pinned H2D copies of the step's inputs,
+    the launch, and the D2H read of every output, all inside the timed region."""
+    h_in = {k: getattr(bset, k).cpu().pin_memory() for k in ("partials", "residual", "post", "comb", "pre")}
+    outs = ("residual_out", "layer_input", "q_data", "q_scale", "post_out", "comb_out", "pre_out")
+    h_out = {k: torch.empty(getattr(bset, k).shape, dtype=getattr(bset, k).dtype).pin_memory() for k in outs}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    def one():
+        for k, t in h_in.items():
+            getattr(bset, k).copy_(t, non_blocking=True)
+        bset.launch(ws)
+        for k, t in h_out.items():
+            t.copy_(getattr(bset, k), non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        one()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) * 1000.0 / steps, h2d, d2h
+
+
+def cpu_baseline(budget_s=12.0):
+    """The oracle (float64, as it stands) on the benchmark boundary, on this host's cores."""
+    import threadpoolctl
+    import oracle as O
+    from mhc_residual_stream_b200 import synthetic as S
+    d = S.draw_boundary(ROWS, HIDDEN, n=HC, partials=PARTIALS, seed=2032)
+    f = {k: d[k].double().numpy() for k in ("partials", "residual", "post", "comb", "pre", "norm_weight")}
+    cw = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in d["coeff"].as_dict().items()}
+    info = threadpoolctl.threadpool_info()
+    cores = max([i.get("num_threads", 1) for i in info] + [1])
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while True:
+        t0 = time.perf_counter()
+        O.boundary(partials=f["partials"], residual=f["residual"], post=f["post"], comb=f["comb"], pre=f["pre"],
+                   norm_weight=f["norm_weight"], norm_eps=1e-6, coeff=cw, mxfp8=True, swizzled=True)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() > t_end or len(times) >= 200:
+            break
+    us = statistics.median(times) * 1e6
+    return {"value": round(us, 1), "unit": "µs/boundary", "cores": cores, "kind": "oracle",
+            "sample": f"{len(times)} full boundaries (rows 32, H 7168, n 4, P 8, MXFP8, coefficients), median; "
+                      f"numpy float64, BLAS threads {cores}"}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    """Largest value over the ranks (every rank gets it); device-timed numbers use this."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_us_per_boundary(ms_max, steps, world):
+    """Whole-job time per boundary: the slowest rank's elapsed time over all ranks' boundaries."""
+    return ms_max * 1000.0 / (steps * world)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def ours(args):
+    from mhc_residual_stream_b200 import build
+    from mhc_residual_stream_b200 import mhc as M
+    world, rank, local = dist_setup(args)
+    build.build()
+    M.lib()
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    peak, peak_kind = load_peak()
+
+    nsets = sets_for(ROWS)
+    sets = [BoundarySet(ROWS, 900000 + 97 * i + 1000 * rank, device) for i in range(nsets)]
+    ws = M.new_workspace(ROWS, HIDDEN, HC, device)
+    set_bytes = sum(t.numel() * t.element_size() for s in sets[:1] for t in
+                    (s.partials, s.residual, s.coeffs.fn, s.residual_out, s.layer_input, s.q_data))
+    assert set_bytes * nsets > 2 * L2_BYTES
+    graph_len = 240
+    main, tail = timed_graph_steps(sets, ws, args.steps, args.warmup, graph_len)
+    sampler = ClockSampler(device) if rank == 0 else None
+    barrier(world)
+    ms = run_timed(main, tail, args.steps, graph_len, sampler)
+    ms = max_over_ranks(ms, world)
+    st = M.mhc_get_device_status(ws)
+    if st != M.OK:
+        raise RuntimeError(f"device status {M.STATUS_NAMES[st]}")
+    us_per = aggregate_us_per_boundary(ms, args.steps, world)
+    us_kernel = ms * 1000.0 / args.steps                 # per launch on one GPU
+    bpb = boundary_bytes(ROWS)
+    achieved = bpb / (us_kernel * 1e-6) / 1e9
+
+    result = {
+        "metric": METRIC, "value": round(us_per, 4), "unit": "µs/boundary", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 7),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; decode attention-side boundary inputs, no trained weights)",
+        "config": {"workload": "decode attention-side boundary: rows 32, H 7168, hc_mult 4, 8 bf16 partials, "
+                               "MXFP8 layer input (swizzled 128x4), coefficients with 20 Sinkhorn iterations",
+                   "rows": ROWS, "hidden": HIDDEN, "hc_mult": HC, "partials": PARTIALS,
+                   "l2": f"inputs larger than L2: {nsets} rotating buffer sets, {set_bytes * nsets / 1e6:.0f} MB",
+                   "timing": "CUDA graphs of 240 boundaries, CUDA events on the launching stream",
+                   "parallelism": f"replicas x{world}"},
+        "gb_per_s": round(achieved * world, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": load_traffic(),
+                     "algorithmic_bytes": bpb, "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "kernel": "boundary_kernel<4, partials>"},
+        "gpu_launches": args.steps,
+    }
+    if sampler is not None:
+        result["clocks"] = sampler.summary()
+
+    if not args.no_sweep:
+        sweep = {}
+        for R in (1, 2, 4, 8, 16, 32, 64, 128):
+            ss = [BoundarySet(R, 800000 + 131 * i + R, device) for i in range(sets_for(R))]
+            wsr = M.new_workspace(R, HIDDEN, HC, device)
+            n = min(args.steps, 24000) // graph_len * graph_len or graph_len
+            m, t = timed_graph_steps(ss, wsr, n, 2 * graph_len, graph_len)
+            msr = run_timed(m, t, n, graph_len)
+            us = msr * 1000.0 / n
+            gbs = boundary_bytes(R) / (us * 1e-6) / 1e9
+            sweep[str(R)] = {"us": round(us, 3), "gb_per_s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                             "algorithmic_bytes": boundary_bytes(R), "sets": len(ss)}
+            del ss, m, t
+        result["rows_sweep"] = sweep
+        # one decode step: the 123 chained boundaries of the 61-layer loop at rows 32
+        from mhc_residual_stream_b200.decode import DecodeLoop
+        loop = DecodeLoop(rows=ROWS, device=str(device))
+        g = capture(lambda i: loop.run(), 1)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = 20
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(2_000_000)
+        start.record()
+        for _ in range(reps):
+            g.replay()
+        end.record()
+        torch.cuda.synchronize()
+        us_step = start.elapsed_time(end) * 1000.0 / reps
+        lb = loop.algorithmic_bytes()
+        result["decode_step"] = {"boundaries": len(loop.steps), "us": round(us_step, 2),
+                                 "us_per_boundary": round(us_step / len(loop.steps), 3),
+                                 "gb_per_s": round(lb / (us_step * 1e-6) / 1e9, 1), "algorithmic_bytes": lb}
+        if M.mhc_get_device_status(loop.workspace) != M.OK:
+            raise RuntimeError("decode loop device status")
+
+    e2e_us, h2d, d2h = e2e_time(sets[0], ws, min(200, max(10, args.steps // 100)), device)
+    e2e_us = max_over_ranks(e2e_us, world) / world
+    result["e2e"] = {"value": round(e2e_us, 2), "unit": "µs/boundary", "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h}
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline()
+    barrier(world)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def reference(args):
+    """The reference arm: the CPU oracle, on rank 0 only, on this machine's host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import threadpoolctl
+    import oracle as O
+    from mhc_residual_stream_b200 import synthetic as S
+    d = S.draw_boundary(ROWS, HIDDEN, n=HC, partials=PARTIALS, seed=2032)
+    f = {k: d[k].double().numpy() for k in ("partials", "residual", "post", "comb", "pre", "norm_weight")}
+    cw = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in d["coeff"].as_dict().items()}
+
+    def step():
+        O.boundary(partials=f["partials"], residual=f["residual"], post=f["post"], comb=f["comb"], pre=f["pre"],
+                   norm_weight=f["norm_weight"], norm_eps=1e-6, coeff=cw, mxfp8=True, swizzled=True)
+
+    for _ in range(min(args.warmup, 3)):
+        step()
+    budget = 90.0
+    t0 = time.perf_counter()
+    done = 0
+    while done < args.steps:
+        step()
+        done += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    el = time.perf_counter() - t0
+    us = el * 1e6 / done
+    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    sample = (f"{done} of {args.steps} requested boundaries timed (bounded at {budget:.0f} s); "
+              "full rows-32 boundary each")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "µs/boundary",
+        "n_gpus": world, "steps": done, "warmup": min(args.warmup, 3), "ms_per_step": round(us / 1000, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "decode attention-side boundary: rows 32, H 7168, hc_mult 4, 8 bf16 partials, "
+                               "MXFP8 layer input (swizzled 128x4), coefficients with 20 Sinkhorn iterations",
+                   "rows": ROWS, "hidden": HIDDEN, "hc_mult": HC, "partials": PARTIALS},
+        "cpu_baseline": {"value": round(us, 1), "unit": "µs/boundary", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(us, 1), "unit": "µs/boundary", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=240000)
+    ap.add_argument("--warmup", type=int, default=2400)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the rows sweep and the decode-loop step")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

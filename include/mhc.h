@@ -25,6 +25,14 @@
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and
  *     do not synchronise the host. Host-side argument checks happen before any
  *     launch; a call that returns an error launched nothing.
+ *   - Kernels are launched with programmatic stream serialization (dependent
+ *     launch): a boundary kernel may start while the kernel before it on the
+ *     stream is finishing, and reads the weights (fn, scale, base, norm_weight)
+ *     before waiting for that kernel. So weights must not be written by the
+ *     kernel launched immediately before on the same stream if that kernel
+ *     triggers dependent launches (no kernel of this library writes weights;
+ *     kernels that do not trigger, like ordinary library kernels, are waited
+ *     for in full). Activations are read only after the wait.
  *   - Errors are returned, never raised or aborted on. Errors found by a kernel
  *     (a wait that ran out, a gather index out of range) are recorded in the
  *     workspace and read with mhc_get_device_status.
@@ -61,7 +69,7 @@ typedef enum {
   MHC_ERR_UNSUPPORTED_SHAPE = 2, /* rows/hidden/hc_mult/P/top_k outside the limits */
   MHC_ERR_WORKSPACE = 3,         /* workspace NULL, misaligned or too small */
   MHC_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, query) */
-  MHC_ERR_DEVICE_TIMEOUT = 5,    /* device: a cross-block wait gave up */
+  MHC_ERR_DEVICE_TIMEOUT = 5,    /* device: a bounded wait gave up */
   MHC_ERR_DEVICE_INDEX = 6       /* device: expanded_idx_to_permuted_idx past the end */
 } mhc_status;
 
@@ -107,19 +115,21 @@ typedef struct {
   int swizzled_128x4;
 } mhc_mxfp8_out;
 
-/* Bytes of workspace the boundary entry points need for (rows, hidden, hc_mult).
- * A workspace sized for R rows serves every call with rows <= R and the same
- * hidden and hc_mult. It must be 256-byte aligned, zeroed once before first use
- * (mhc_workspace_init) and used by one stream at a time: calls sharing a
- * workspace must not overlap on the GPU. Returns 0 for unsupported shapes. */
+/* Bytes of workspace the boundary entry points need for (rows, hidden, hc_mult):
+ * a 1 KB header (the status word kernels record errors in) and the per-block
+ * partial sums that the tail of a boundary adds up. A workspace sized for R rows
+ * serves every call with rows <= R and the same hidden and hc_mult. It must be
+ * 256-byte aligned, zeroed once before first use (mhc_workspace_init; the
+ * partial sums are rewritten by every call) and used by one stream at a time:
+ * calls sharing a workspace must not overlap on the GPU. Returns 0 for
+ * unsupported shapes. */
 MHC_API size_t mhc_workspace_bytes(int rows, int hidden, int hc_mult);
 
 /* Bytes of the MXFP8 scale buffer: roundup(R,128) * roundup(H/32, 4) when
  * swizzled, R * H/32 when linear. Returns 0 for H not a multiple of 32. */
 MHC_API size_t mhc_mxfp8_scale_bytes(int rows, int hidden, int swizzled_128x4);
 
-/* Zero the workspace on `stream` (cudaMemsetAsync). Needed once before first use
- * and again after a call reported MHC_ERR_DEVICE_TIMEOUT. */
+/* Zero the workspace on `stream` (cudaMemsetAsync). Needed once before first use. */
 MHC_API mhc_status mhc_workspace_init(void* workspace, size_t ws_bytes, mhc_stream stream);
 
 /* Full boundary after a sublayer with TP-partial output ([all_reduce]
@@ -201,12 +211,13 @@ MHC_API mhc_status mhc_get_device_status(void* workspace, mhc_stream stream);
 /* Static, human-readable name of a status code. */
 MHC_API const char* mhc_status_string(mhc_status status);
 
-/* Test hook for the bounded waits: `budget_ns` > 0 sets the time a block waits
- * at a cross-block barrier before giving up (default 1e9 ns); `extra_arrivals`
- * makes the barrier expect that many blocks beyond the grid, so that it can
- * never complete and every wait runs out. Affects launches made after the call
- * by this process. Returns the previous budget. */
-MHC_API int64_t mhc_debug_set_wait(int64_t budget_ns, int extra_arrivals);
+/* Test hook for the bounded waits. A kernel waits on the TMA copies of its fn
+ * slice with a time limit: `budget_ns` > 0 sets it (default 1e9 ns, counted as
+ * 2 SM cycles per ns); `extra_units` makes that wait expect that many 16-byte
+ * units more than are copied, so that it can never complete and runs out
+ * (recording MHC_ERR_DEVICE_TIMEOUT). Affects launches made after the call by
+ * this process. Returns the previous budget. */
+MHC_API int64_t mhc_debug_set_wait(int64_t budget_ns, int extra_units);
 
 #ifdef __cplusplus
 }

@@ -1,24 +1,27 @@
 // mHC decode boundary on B200 (sm_100a): the fused kernel and the C ABI of
 // libmhc.so (declared in include/mhc.h).
 //
-// One launch does the whole boundary. Block g owns columns [64g, 64g+64) of H
-// for every row, so each weight of fn is read from HBM exactly once:
-//   1. TMA bulk copies bring the block's fn slice (n*64 rows of C floats) into
-//      shared memory while the threads stream the partials (or the MoE gather)
-//      and the residual streams with 128-bit loads;
-//   2. per (row, 8 columns) a lane sums the partials, applies the mHC post-mix
-//      (vllm ...boundary.boundary, Boundaries.post_only: mhc_post(x, residual,
-//      post, comb)), rounds the new streams to bf16 and stores them, collapses
-//      them with the carried pre (BoundaryState.pre) and accumulates, over its
-//      32 stream values, sum c^2, sum v^2 and the C dot products with fn
-//      (CUDA-core packed FMA);
-//   3. the 8 lanes of a row reduce their sums (shuffle reduce-scatter) and the
-//      block writes them to the workspace;
-//   4. one bounded grid barrier; then every block normalises its own columns
-//      into the layer input (and MXFP8), and block g finishes the coefficients
-//      (logits, sigmoid, Sinkhorn in registers) of rows g, g+G, ...
-// The residual-only variant stops after step 2 and needs no barrier.
-// All reductions run in a fixed order, so results are bitwise reproducible.
+// A boundary is two launches chained by programmatic dependent launch (PDL).
+// Block g of both owns columns [64g, 64g+64) of H for every row, so each
+// weight of fn is read from HBM exactly once.
+// The streaming kernel (boundary_kernel):
+//   1. TMA bulk copies bring the block's fn slice into shared memory and the
+//      block's activations are prefetched into L2, both before the kernel waits
+//      for its predecessor on the stream;
+//   2. per (row, 8 columns) a lane sums the partials (or finalizes the MoE
+//      output), applies the mHC post-mix (vllm ...boundary.boundary,
+//      Boundaries.post_only: mhc_post(x, residual, post, comb)), rounds the new
+//      streams to bf16, stores them, sums the squares of their collapse with the
+//      carried pre (BoundaryState.pre) and of the streams;
+//   3. the block projects its rows' n*64 stream values onto the C fn columns
+//      with register-tiled CUDA-core FMA (8 rows x C/4 columns per thread) and
+//      writes its partial sums to the workspace.
+// The tail kernel (boundary_tail_kernel), once the streaming kernel is done:
+//   4. every block normalises its own columns into the layer input (and MXFP8),
+//      and block g finishes the coefficients (logits, sigmoid, Sinkhorn with one
+//      comb element per lane) of rows g, g+G, ...
+// The residual-only variant is the streaming kernel alone. All reductions run
+// in a fixed order, so results are bitwise reproducible.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,22 +33,30 @@
 namespace mhc {
 
 constexpr int kCols = 64;      // columns of H per block
-constexpr int kThreads = 256;  // 8 warps; a warp covers 4 rows x 64 columns per step
+constexpr int kThreads = 256;  // 8 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRows = 128;
 constexpr int kMaxPartials = 16;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxIters = 1000;
-constexpr size_t kWsHeader = 1024;  // status, barrier count, barrier generation (own 128-B lines)
-constexpr int kStatusWord = 0, kBarCountWord = 32, kBarGenWord = 64;
+constexpr int kMaxBlocks = 148;  // H/64 blocks, all resident at once (one per SM)
+// Workspace header: the status word (byte 0); the partial sums follow.
+constexpr size_t kWsHeader = 1024;
+constexpr int kStatusWord = 0;
 
 enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3 };
 
 __host__ __device__ constexpr int logits_of(int n) { return 2 * n + n * n; }
-// Values reduced per row: C dot products, sum v^2, sum c^2, padded to a power of two >= 8.
+// logit columns padded to a multiple of 4: the projection's four column groups
+__host__ __device__ constexpr int cpad_of(int n) { return (logits_of(n) + 3) & ~3; }
+// Per-block record of a row in the workspace: C dot products, then sum v^2,
+// padded to a power of two >= 8 floats.
 __host__ __device__ constexpr int red_of(int n) {
-  return logits_of(n) + 2 <= 8 ? 8 : (logits_of(n) + 2 <= 16 ? 16 : 32);
+  return logits_of(n) + 1 <= 8 ? 8 : (logits_of(n) + 1 <= 16 ? 16 : 32);
 }
+// fn slice in shared memory as the bulk copies land it: pieces of 8 rows of C
+// floats followed by a 16-byte gap (the gap puts the rows that a half-warp of
+// the projection reads into distinct banks).
 __host__ __device__ constexpr int fn_piece_bytes(int n) { return 8 * logits_of(n) * 4 + 16; }
 
 struct Params {
@@ -86,61 +97,74 @@ struct Params {
   unsigned* ctl;
   float* sc2_part;  // [R][G]
   float* dot_part;  // [R][G][RED]
-  int extra_arrivals;
+  // the streams the tail normalises: the new streams, the given streams, or the
+  // embedding of the first layer (whose identity pre-mix selects it)
+  const __nv_bfloat16* tail_streams;
+  int tail_broadcast;
+  int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
   int64_t budget_ns;
 };
 
 struct SmemLayout {
-  int fn_off, mix_off, c_off, moe_off, inv_off, red_off, bar_off, total;
+  int fn_off, v_off, mix_off, moe_off, xs_off, misc_off, total;
 };
 
+// Shared memory of the streaming kernel.
 template <int N>
 __host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe) {
+  constexpr int CP = cpad_of(N);
   SmemLayout L{};
   int o = 0;
   L.fn_off = o;
   o += N * 8 * fn_piece_bytes(N);
-  L.mix_off = o;
+  L.v_off = o;  // new streams, bf16 [R][n*64]
+  o += R * N * kCols * 2;
+  L.mix_off = o;  // [R][post n | comb n*n | pre n]
   o += R * (2 * N + N * N) * 4;
   o = (o + 15) & ~15;
-  L.c_off = o;
-  o += R * kCols * 4;
   L.moe_off = o;
   if (moe) o += R * topk * 8;
   o = (o + 15) & ~15;
-  L.inv_off = o;
-  o += kMaxRows * 4;
-  L.red_off = o;
-  o += (kThreads + 64) * 4;
-  o = (o + 15) & ~15;
-  L.bar_off = o;
+  L.xs_off = o;  // projection: the second half-K warp's sums, [4][8][CP]
+  o += 4 * 8 * CP * 4;
+  L.misc_off = o;  // mbarrier
   o += 16;
   L.total = o;
   return L;
 }
 
-// Reduce-scatter `v` (M values) over the 8 lanes that share lane bits 3-4:
-// afterwards lane with (lane & 7) == q holds, in v[0 .. M/8), the sums of
-// values [q*M/8, (q+1)*M/8) over the 8 lanes. Fixed order: deterministic.
-template <int M>
-__device__ __forceinline__ void reduce_scatter8(float (&v)[M], int vec) {
-#pragma unroll
-  for (int s = 0; s < 3; ++s) {
-    const int mask = 4 >> s;
-    const int half = M >> (s + 1);
-    const bool up = (vec & mask) != 0;
-#pragma unroll
-    for (int k = 0; k < half; ++k) {
-      const float send = up ? v[k] : v[k + half];
-      const float keep = up ? v[k + half] : v[k];
-      v[k] = keep + __shfl_xor_sync(kFull, send, mask);
-    }
-  }
+// Shared memory of the tail kernel.
+struct TailLayout {
+  int inv_off, pre_off, part_off, cst_off, total;
+};
+
+template <int N>
+__host__ __device__ inline TailLayout tail_layout(int R) {
+  constexpr int CP = cpad_of(N);
+  TailLayout L{};
+  int o = 0;
+  L.inv_off = o;
+  o += kMaxRows * 4;
+  L.pre_off = o;
+  o += R * N * 4;
+  o = (o + 15) & ~15;
+  L.part_off = o;  // [warps][8] float4
+  o += kWarps * 8 * 16;
+  L.cst_off = o;  // norm weight [64] bf16, scale[4], base[CP]
+  o += kCols * 2 + (4 + CP) * 4;
+  L.total = (o + 15) & ~15;
+  return L;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  return v;
+}
+
+__device__ __forceinline__ float sum8_lanes(float v) {  // over the 8 lanes sharing lane bits 3-4
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
   return v;
 }
 
@@ -150,22 +174,100 @@ __device__ __forceinline__ int swizzled_scale_offset(int r, int c, int col_tiles
   return tile * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (c & 3);
 }
 
+// Sum over blocks of row r's per-block records ([r][g][RED] floats): thread t
+// loads the float4 number t % (RED/4) of records g = t/(RED/4) + k*kThreads/(RED/4)
+// (all loads issued before any add) and adds them in k order.
+template <int RED, int MAXK>
+__device__ __forceinline__ float4 sum_row_partials(const float* part, int r, int G, int tid) {
+  constexpr int V4 = RED / 4;
+  const float4* base = reinterpret_cast<const float4*>(part + static_cast<size_t>(r) * G * RED);
+  const int F = G * V4;
+  float4 v[MAXK];
+#pragma unroll
+  for (int k = 0; k < MAXK; ++k) {
+    const int f = tid + k * kThreads;
+    v[k] = f < F ? __ldcg(base + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float4 a = v[0];
+#pragma unroll
+  for (int k = 1; k < MAXK; ++k) {
+    a.x += v[k].x;
+    a.y += v[k].y;
+    a.z += v[k].z;
+    a.w += v[k].w;
+  }
+  return a;
+}
+
+template <int N>
+__device__ __forceinline__ float tree_sum(const float (&v)[N]) {
+  if constexpr (N == 4) {
+    return (v[0] + v[1]) + (v[2] + v[3]);
+  } else {
+    float s = v[0];
+#pragma unroll
+    for (int i = 1; i < N; ++i) s += v[i];
+    return s;
+  }
+}
+
+// Registers of one row-quad step of a lane: the stream vectors and up to 8
+// partial (or gathered) vectors, plus the shared-output / embedding vector.
+template <int N>
+struct QuadLoads {
+  uint4 rv[N];
+  uint4 pv[8];
+  uint4 sv;
+};
+
+template <int N, int FRONT>
+__device__ __forceinline__ void load_quad(const Params& p, int r, int h0, const int* e2p_s, QuadLoads<N>& Q) {
+  const int H = p.H;
+  if (r >= p.R) return;
+  if constexpr (FRONT == kBroadcast) {
+    Q.sv = ld_nc_v4(p.x + static_cast<size_t>(r) * H + h0);
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; ++j) Q.rv[j] = ld_v4(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
+  }
+  if (FRONT == kPartials) {
+    const __nv_bfloat16* base = p.partials + static_cast<size_t>(r) * H + h0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (u < p.P) Q.pv[u] = ld_nc_v4(base + u * p.pstride);
+  } else if (FRONT == kMoe) {
+    Q.sv = ld_nc_v4(p.shared_out + static_cast<size_t>(r) * H + h0);
+    const int* idx = e2p_s + r * p.topk;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (u < p.topk) {
+        const int e = idx[u];
+        Q.pv[u] = (e >= 0 && e < p.num_perm) ? ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0)
+                                             : make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+}
+
 template <int N, int FRONT>
 __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
   constexpr int C = logits_of(N);
+  constexpr int CP = cpad_of(N);
+  constexpr int CT = CP / 4;     // projection columns per thread
+  constexpr int KC = N * kCols;  // stream values per row in this block
+  constexpr int KPT = KC / 16;   // of which one projection thread owns KPT consecutive ones
   constexpr int RED = red_of(N);
+  constexpr int MIX = 2 * N + N * N;
   constexpr int PIECE = fn_piece_bytes(N);
   extern __shared__ __align__(128) unsigned char smem[];
   const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
   unsigned char* fn_s = smem + L.fn_off;
+  __nv_bfloat16* v_s = reinterpret_cast<__nv_bfloat16*>(smem + L.v_off);
   float* mix_s = reinterpret_cast<float*>(smem + L.mix_off);
-  float* c_s = reinterpret_cast<float*>(smem + L.c_off);
   int* e2p_s = reinterpret_cast<int*>(smem + L.moe_off);
   float* ew_s = reinterpret_cast<float*>(smem + L.moe_off) + p.R * p.topk;
-  float* inv_s = reinterpret_cast<float*>(smem + L.inv_off);
-  float* red_s = reinterpret_cast<float*>(smem + L.red_off);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  int* flag_s = reinterpret_cast<int*>(smem + L.bar_off + 8);
+  float* xs_s = reinterpret_cast<float*>(smem + L.xs_off);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.misc_off);
 
   const int g = blockIdx.x;
   const int G = gridDim.x;
@@ -173,127 +275,155 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
   const int R = p.R;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rq = lane >> 3, vec = lane & 7;
-  const int h0 = g * kCols + vec * 8;  // this lane's 8 columns
-  const uint64_t deadline = global_ns() + static_cast<uint64_t>(p.budget_ns);
+  const int h0 = g * kCols + vec * 8;  // this lane's 8 columns in the row-quad phase
+  const long long deadline = wait_deadline(p.budget_ns);
   unsigned* status = p.ctl + kStatusWord;
+  const int nquads = (R + 3) >> 2;
 
-  // ---- 1. start the fn slice copy (one bulk copy per 8 rows, 16 B gap between pieces)
+  // ---- 1. the block's fn slice by TMA bulk copies. Weights are never written by
+  // the kernel that precedes this one on the stream, so this runs before the
+  // wait on that kernel (programmatic dependent launch).
   if (p.do_coeff) {
     if (tid == 0) mbar_init(bar, 1);
     __syncthreads();
     if (warp == 0) {
-      if (lane == 0) mbar_arrive_expect_tx(bar, N * kCols * C * 4);
+      if (lane == 0) mbar_arrive_expect_tx(bar, KC * C * 4 + 16 * p.extra_tx);
       __syncwarp();
       for (int m = lane; m < N * 8; m += 32) {
         const int i = m >> 3, piece = m & 7;
-        const float* src = p.fn + (static_cast<size_t>(i) * H + g * kCols + piece * 8) * C;
-        bulk_g2s(fn_s + m * PIECE, src, 8 * C * 4, bar);
+        bulk_g2s(fn_s + m * PIECE, p.fn + (static_cast<size_t>(i) * H + g * kCols + piece * 8) * C, 8 * C * 4, bar);
       }
     }
   }
-  // ---- mixes (and MoE routing) of every row into shared memory
-  {
-    constexpr int MIX = 2 * N + N * N;
-    for (int k = tid; k < R * MIX; k += kThreads) {
-      const int r = k / MIX, c = k - r * MIX;
-      float v = 0.f;
-      if (c < N) {
-        v = (FRONT == kStreams || FRONT == kBroadcast) ? 0.f : p.post[r * N + c];
-      } else if (c < N + N * N) {
-        v = (FRONT == kStreams || FRONT == kBroadcast) ? 0.f : p.comb[r * N * N + (c - N)];
-      } else {
-        v = (p.pre != nullptr) ? p.pre[r * N + (c - N - N * N)] : 0.f;
-      }
-      mix_s[k] = v;
-    }
-    if (FRONT == kMoe) {
-      for (int k = tid; k < R * p.topk; k += kThreads) {
-        e2p_s[k] = p.e2p[k];
-        ew_s[k] = p.ew[k];
-      }
-    }
-  }
-  __syncthreads();
 
-  bool fn_ready = false;
-  bool aborted = false;
-  const int nquads = (R + 3) >> 2;
+  // ---- 2. bring this block's activations into L2 while the preceding kernel may
+  // still run: a prefetch is only a hint and L2 is the point of coherence, so
+  // it is safe before the wait; gather indices read now only steer prefetches.
+  if (vec == 0 || vec == 7) {
+    for (int q = warp; q < nquads; q += kWarps) {
+      const int r = q * 4 + rq;
+      if (r >= R) break;
+      if constexpr (FRONT == kBroadcast) {
+        prefetch_l2(p.x + static_cast<size_t>(r) * H + h0);
+      } else {
+        for (int j = 0; j < N; ++j) prefetch_l2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
+      }
+      if (FRONT == kPartials) {
+        for (int pp = 0; pp < p.P; ++pp) prefetch_l2(p.partials + pp * p.pstride + static_cast<size_t>(r) * H + h0);
+      } else if (FRONT == kMoe) {
+        prefetch_l2(p.shared_out + static_cast<size_t>(r) * H + h0);
+        for (int t = 0; t < p.topk; ++t) {
+          int e = p.e2p[r * p.topk + t];
+          e = e < 0 ? 0 : (e >= p.num_perm ? p.num_perm - 1 : e);
+          if (p.num_perm > 0) prefetch_l2(p.gemm2 + static_cast<size_t>(e) * H + h0);
+        }
+      }
+    }
+  }
+
+  // ---- 3. wait for the preceding kernel, let the next one launch, and read
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int k = tid; k < R * MIX; k += kThreads) {  // [R][post n | comb n*n | pre n]
+    const int r = k / MIX, c = k - r * MIX;
+    if (c < N + N * N) {
+      if (FRONT == kStreams || FRONT == kBroadcast) {
+        mix_s[k] = 0.f;
+      } else if (c < N) {
+        cp_async4(mix_s + k, p.post + r * N + c);
+      } else {
+        cp_async4(mix_s + k, p.comb + r * N * N + (c - N));
+      }
+    } else if (p.pre != nullptr) {
+      cp_async4(mix_s + k, p.pre + r * N + (c - N - N * N));
+    } else {
+      mix_s[k] = 0.f;
+    }
+  }
+  if (FRONT == kMoe) {
+    for (int k = tid; k < R * p.topk; k += kThreads) {
+      cp_async4(e2p_s + k, p.e2p + k);
+      cp_async4(ew_s + k, p.ew + k);
+    }
+  }
+  QuadLoads<N> cur;
+  if (FRONT != kMoe && warp < nquads) load_quad<N, FRONT>(p, warp * 4 + rq, h0, e2p_s, cur);
+  cp_async_wait_all();
+  __syncthreads();
+  if (FRONT == kMoe && warp < nquads) load_quad<N, FRONT>(p, warp * 4 + rq, h0, e2p_s, cur);
+
+  // ---- 4. row quads: sum / finalize, post-mix, store the streams, sum c^2
   for (int q = warp; q < nquads; q += kWarps) {
+    QuadLoads<N> nxt;
+    if (q + kWarps < nquads) load_quad<N, FRONT>(p, (q + kWarps) * 4 + rq, h0, e2p_s, nxt);
     const int r = q * 4 + rq;
     const bool valid = r < R;
-    const float* mix = mix_s + (valid ? r : 0) * (2 * N + N * N);
-
-    // ---- 2a. front end: the new streams nf[i][t] (bf16 values held as floats)
+    const float* mix = mix_s + (valid ? r : 0) * MIX;
     float nf[N][8];
     uint4 nb[N];
     float xs[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) xs[t] = 0.f;
     if (FRONT == kPartials || FRONT == kMoe) {
-      uint4 rv[N];
+      float rf[N][8];
       if (valid) {
 #pragma unroll
-        for (int j = 0; j < N; ++j) rv[j] = ld_v4(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
+        for (int j = 0; j < N; ++j) unpack8(cur.rv[j], rf[j]);
         if (FRONT == kPartials) {
-          const __nv_bfloat16* base = p.partials + static_cast<size_t>(r) * H + h0;
-          for (int p0 = 0; p0 < p.P; p0 += 8) {
-            uint4 pv[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              if (p0 + u < p.P) pv[u] = ld_nc_v4(base + (p0 + u) * p.pstride);
+          for (int u = 0; u < 8; ++u) {
+            if (u < p.P) {
+              float f[8];
+              unpack8(cur.pv[u], f);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              if (p0 + u < p.P) {
+              for (int t = 0; t < 8; ++t) xs[t] += f[t];
+            }
+          }
+          for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
+            float f[8];
+            unpack8(ld_nc_v4(p.partials + u * p.pstride + static_cast<size_t>(r) * H + h0), f);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) xs[t] += f[t];
+          }
+        } else {
+          unpack8(cur.sv, xs);
+          const int* idx = e2p_s + r * p.topk;
+          const float* wt = ew_s + r * p.topk;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {  // the first 8 slots, loaded ahead
+            if (u < p.topk) {
+              const int e = idx[u];
+              if (e >= p.num_perm) {
+                if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
+              } else if (e >= 0) {
                 float f[8];
-                unpack8(pv[u], f);
+                unpack8(cur.pv[u], f);
+                const float w = wt[u];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) xs[t] += f[t];
+                for (int t = 0; t < 8; ++t) xs[t] = fmaf(w, f[t], xs[t]);
               }
             }
           }
-        } else {
-          unpack8(ld_nc_v4(p.shared_out + static_cast<size_t>(r) * H + h0), xs);
-          const int* idx = e2p_s + r * p.topk;
-          const float* wt = ew_s + r * p.topk;
-          for (int t0 = 0; t0 < p.topk; t0 += 8) {
-            uint4 gv[8];
+          for (int u = 8; u < p.topk; ++u) {  // slots beyond 8
+            const int e = idx[u];
+            if (e >= p.num_perm) {
+              if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
+            } else if (e >= 0) {
+              float f[8];
+              unpack8(ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0), f);
+              const float w = wt[u];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int k = t0 + u;
-              if (k < p.topk) {
-                const int e = idx[k];
-                if (e >= 0 && e < p.num_perm) {
-                  gv[u] = ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0);
-                } else {
-                  gv[u] = make_uint4(0, 0, 0, 0);
-                  if (e >= p.num_perm && vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
-                }
-              }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int k = t0 + u;
-              if (k < p.topk) {
-                const int e = idx[k];
-                if (e >= 0 && e < p.num_perm) {
-                  float f[8];
-                  unpack8(gv[u], f);
-                  const float w = wt[k];
-#pragma unroll
-                  for (int t = 0; t < 8; ++t) xs[t] = fmaf(w, f[t], xs[t]);
-                }
-              }
+              for (int t = 0; t < 8; ++t) xs[t] = fmaf(w, f[t], xs[t]);
             }
           }
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < N; ++j) rv[j] = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < N; ++j)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) rf[j][t] = 0.f;
       }
       // mHC post: new[i] = bf16(post[i] * x + sum_j comb[j][i] * res[j])
-      float rf[N][8];
-#pragma unroll
-      for (int j = 0; j < N; ++j) unpack8(rv[j], rf[j]);
 #pragma unroll
       for (int i = 0; i < N; ++i) {
         float a[8];
@@ -310,11 +440,11 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
     } else if (FRONT == kStreams) {
 #pragma unroll
       for (int j = 0; j < N; ++j) {
-        nb[j] = valid ? ld_v4(p.residual + (static_cast<size_t>(r) * N + j) * H + h0) : make_uint4(0, 0, 0, 0);
+        nb[j] = valid ? cur.rv[j] : make_uint4(0, 0, 0, 0);
         unpack8(nb[j], nf[j]);
       }
     } else {  // kBroadcast: every stream is the embedding row
-      const uint4 xv = valid ? ld_nc_v4(p.x + static_cast<size_t>(r) * H + h0) : make_uint4(0, 0, 0, 0);
+      const uint4 xv = valid ? cur.sv : make_uint4(0, 0, 0, 0);
       unpack8(xv, xs);
 #pragma unroll
       for (int j = 0; j < N; ++j) {
@@ -323,18 +453,13 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
         for (int t = 0; t < 8; ++t) nf[j][t] = xs[t];
       }
     }
-
-    // ---- 2b. store the new streams
     if (p.write_res && valid) {
 #pragma unroll
       for (int i = 0; i < N; ++i) st_v4(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
     }
-    if (!p.do_layer && !p.do_coeff) continue;
-
-    // ---- 2c. collapse with the carried pre (identity pre-mix for the broadcast)
-    float sc2 = 0.f;
-    if (p.do_layer) {
+    if (p.do_layer) {  // collapse with the carried pre (identity pre-mix for the broadcast)
       float c[8];
+      float sc2 = 0.f;
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         if (FRONT == kBroadcast) {
@@ -347,121 +472,309 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
         }
         sc2 = fmaf(c[t], c[t], sc2);
       }
-      float4* cs = reinterpret_cast<float4*>(c_s + (valid ? r : 0) * kCols);
+      sc2 = sum8_lanes(sc2);
+      if (valid && vec == 0) p.sc2_part[r * G + g] = sc2;
+    }
+    if (p.do_coeff) {  // stage the streams for the projection; sum v^2 of the row
+      float sv2 = 0.f;
+#pragma unroll
+      for (int i = 0; i < N; ++i)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) sv2 = fmaf(nf[i][t], nf[i][t], sv2);
+      sv2 = sum8_lanes(sv2);
       if (valid) {
-        cs[vec] = make_float4(c[0], c[1], c[2], c[3]);
-        cs[8 + vec] = make_float4(c[4], c[5], c[6], c[7]);
+#pragma unroll
+        for (int i = 0; i < N; ++i) *reinterpret_cast<uint4*>(v_s + r * KC + i * kCols + vec * 8) = nb[i];
+        if (vec == 0) p.dot_part[(static_cast<size_t>(r) * G + g) * RED + C] = sv2;
       }
     }
+    cur = nxt;
+  }
+  if (!p.do_coeff) return;
 
-    if (p.do_coeff) {
-      // ---- 2d. projection of this lane's 8N stream values onto the C fn columns
-      if (!fn_ready) {
-        // warp-uniform decision: every lane of the warp shuffles below
-        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar, 0, deadline));
-        fn_ready = true;
-        if (!ok) {
-          if (lane == 0) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-          aborted = true;
-          break;
-        }
-      }
-      float red[RED];
+  // ---- 5. projection of this block's n*64 stream values per row onto the C fn
+  // columns (CUDA-core FMA). Thread (cg, ks, rs) owns 8 rows x C/4 columns over
+  // the KPT consecutive stream values from ks*KPT: each fn value it loads feeds
+  // 8 rows, each stream value C/4 columns. 64-bit loads of fn are bank-conflict
+  // free for a half-warp in the bulk-copy layout.
+  if (p.do_coeff) {
+    const bool ok = mbar_wait_bounded(bar, 0, deadline);
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
+    const int cg = tid & 3, ks = (tid >> 2) & 15, rs = tid >> 6, ksl = ks & 7, half = ks >> 3;
+    for (int rb = 0; rb < R; rb += 32) {
+      const int r0 = rb + rs * 8;
+      float acc[8][CT];
 #pragma unroll
-      for (int k = 0; k < RED; ++k) red[k] = 0.f;
-      float sv2 = 0.f;
-      if constexpr (C % 4 == 0) {
-        float2 acc[C / 2];
+      for (int j = 0; j < 8; ++j)
 #pragma unroll
-        for (int k = 0; k < C / 2; ++k) acc[k] = make_float2(0.f, 0.f);
+        for (int c = 0; c < CT; ++c) acc[j][c] = 0.f;
+      if (r0 < R) {  // uniform over the warp (rs is)
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-          const unsigned char* piece = fn_s + (i * 8 + vec) * PIECE;
+        for (int kk = 0; kk < KPT; kk += 2) {
+          const int k = ks * KPT + kk;
+          const float* frow = reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4) + cg * CT;
+          float f0[CT], f1[CT];
+          if constexpr (CT % 2 == 0) {
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float v = nf[i][t];
-            sv2 = fmaf(v, v, sv2);
-            const float2 vv = make_float2(v, v);
-            const float4* f = reinterpret_cast<const float4*>(piece + t * C * 4);
+            for (int c = 0; c < CT; c += 2) {
+              const float2 a = *reinterpret_cast<const float2*>(frow + c);
+              const float2 b = *reinterpret_cast<const float2*>(frow + C + c);
+              f0[c] = a.x;
+              f0[c + 1] = a.y;
+              f1[c] = b.x;
+              f1[c + 1] = b.y;
+            }
+          } else {
 #pragma unroll
-            for (int c4 = 0; c4 < C / 4; ++c4) {
-              const float4 w = f[c4];
-              acc[2 * c4] = __ffma2_rn(vv, make_float2(w.x, w.y), acc[2 * c4]);
-              acc[2 * c4 + 1] = __ffma2_rn(vv, make_float2(w.z, w.w), acc[2 * c4 + 1]);
+            for (int c = 0; c < CT; ++c) {
+              f0[c] = frow[c];
+              f1[c] = frow[C + c];
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int r = r0 + j;
+            const unsigned w2 = r < R ? *reinterpret_cast<const unsigned*>(v_s + r * KC + k) : 0u;
+            const float v0 = __uint_as_float(w2 << 16), v1 = __uint_as_float(w2 & 0xffff0000u);
+            if constexpr (CT % 2 == 0) {
+#pragma unroll
+              for (int c = 0; c < CT; c += 2) {
+                float2 a = make_float2(acc[j][c], acc[j][c + 1]);
+                a = __ffma2_rn(make_float2(v0, v0), make_float2(f0[c], f0[c + 1]), a);
+                a = __ffma2_rn(make_float2(v1, v1), make_float2(f1[c], f1[c + 1]), a);
+                acc[j][c] = a.x;
+                acc[j][c + 1] = a.y;
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < CT; ++c) acc[j][c] = fmaf(v1, f1[c], fmaf(v0, f0[c], acc[j][c]));
             }
           }
         }
+        // reduce over the 8 ks of this warp (lane bits 2-4), scattering the rows:
+        // lane with ksl keeps row r0 + ksl
 #pragma unroll
-        for (int k = 0; k < C / 2; ++k) {
-          red[2 * k] = acc[k].x;
-          red[2 * k + 1] = acc[k].y;
+        for (int s = 0; s < 3; ++s) {
+          const int mask = 16 >> s;
+          const int hj = 4 >> s;
+          const bool up = (ksl & (4 >> s)) != 0;
+#pragma unroll
+          for (int j = 0; j < hj; ++j)
+#pragma unroll
+            for (int c = 0; c < CT; ++c) {
+              const float send = up ? acc[j][c] : acc[j + hj][c];
+              const float keep = up ? acc[j + hj][c] : acc[j][c];
+              acc[j][c] = keep + __shfl_xor_sync(kFull, send, mask);
+            }
         }
-      } else {
+        if (half == 1) {
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-          const unsigned char* piece = fn_s + (i * 8 + vec) * PIECE;
+          for (int c = 0; c < CT; ++c) xs_s[(rs * 8 + ksl) * CP + cg * CT + c] = acc[0][c];
+        }
+      }
+      __syncthreads();
+      if (r0 < R && half == 0 && r0 + ksl < R) {
+        float* dst = p.dot_part + (static_cast<size_t>(r0 + ksl) * G + g) * RED;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float v = nf[i][t];
-            sv2 = fmaf(v, v, sv2);
-            const float* f = reinterpret_cast<const float*>(piece + t * C * 4);
+        for (int c = 0; c < CT; ++c) {
+          const int cc = cg * CT + c;
+          if (cc < C) dst[cc] = acc[0][c] + xs_s[(rs * 8 + ksl) * CP + cc];
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Sinkhorn normalisation of an n x n matrix in one thread's registers: `iters`
+// times, each row divided by (its sum + eps), then each column by (its sum +
+// eps). For n >= 2 rows are held as pairs and summed / scaled with packed
+// f32x2 arithmetic, which halves the instructions on the serial chain.
+template <int N>
+__device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, float eps) {
+  if constexpr (N == 1) {
+    for (int it = 0; it < iters; ++it) {
+      M[0][0] *= rcp_approx(M[0][0] + eps);
+      M[0][0] *= rcp_approx(M[0][0] + eps);
+    }
+  } else {
+    constexpr int H2 = N / 2;
+    float2 P[N][H2];
 #pragma unroll
-            for (int c = 0; c < C; ++c) red[c] = fmaf(v, f[c], red[c]);
+    for (int j = 0; j < N; ++j)
+#pragma unroll
+      for (int h = 0; h < H2; ++h) P[j][h] = make_float2(M[j][2 * h], M[j][2 * h + 1]);
+    const float2 e2 = make_float2(eps, eps);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int j = 0; j < N; ++j) {  // rows
+        float2 s2 = P[j][0];
+#pragma unroll
+        for (int h = 1; h < H2; ++h) s2 = __fadd2_rn(s2, P[j][h]);
+        const float rr = rcp_approx(s2.x + s2.y + eps);
+        const float2 r2 = make_float2(rr, rr);
+#pragma unroll
+        for (int h = 0; h < H2; ++h) P[j][h] = __fmul2_rn(P[j][h], r2);
+      }
+#pragma unroll
+      for (int h = 0; h < H2; ++h) {  // columns 2h, 2h+1
+        float2 c2;
+        if constexpr (N == 4) {
+          c2 = __fadd2_rn(__fadd2_rn(P[0][h], P[1][h]), __fadd2_rn(P[2][h], P[3][h]));
+        } else {
+          c2 = P[0][h];
+#pragma unroll
+          for (int j = 1; j < N; ++j) c2 = __fadd2_rn(c2, P[j][h]);
+        }
+        c2 = __fadd2_rn(c2, e2);
+        const float2 r2 = make_float2(rcp_approx(c2.x), rcp_approx(c2.y));
+#pragma unroll
+        for (int j = 0; j < N; ++j) P[j][h] = __fmul2_rn(P[j][h], r2);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+#pragma unroll
+      for (int h = 0; h < H2; ++h) {
+        M[j][2 * h] = P[j][h].x;
+        M[j][2 * h + 1] = P[j][h].y;
+      }
+  }
+}
+
+// The tail of a boundary, launched after the streaming kernel (programmatic
+// dependent launch): once every block's partial sums are in the workspace,
+// block g normalises columns [64g, 64g+64) of every row into the layer input
+// (and MXFP8), recomputing the collapse from the bf16 streams (L2-resident), and
+// finishes the coefficients of rows g, g+G, ...
+template <int N>
+__global__ void __launch_bounds__(kThreads, 1) boundary_tail_kernel(const Params p) {
+  constexpr int C = logits_of(N);
+  constexpr int CP = cpad_of(N);
+  constexpr int RED = red_of(N);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const TailLayout L = tail_layout<N>(p.R);
+  float* inv_s = reinterpret_cast<float*>(smem + L.inv_off);
+  float* pre_s = reinterpret_cast<float*>(smem + L.pre_off);
+  float* red_s = reinterpret_cast<float*>(smem + L.part_off);
+  __nv_bfloat16* nw_s = reinterpret_cast<__nv_bfloat16*>(smem + L.cst_off);
+  float* scale_s = reinterpret_cast<float*>(smem + L.cst_off + kCols * 2);
+  float* base_s = scale_s + 4;
+
+  const int g = blockIdx.x;
+  const int G = gridDim.x;
+  const int H = p.H;
+  const int R = p.R;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rq = lane >> 3, vec = lane & 7;
+  const int h0 = g * kCols + vec * 8;
+  const int nquads = (R + 3) >> 2;
+
+  // weights before the wait on the streaming kernel
+  if (p.do_layer && tid < 8) cp_async16(nw_s + tid * 8, p.norm_weight + g * kCols + tid * 8);
+  if (p.do_coeff) {
+    if (tid >= 32 && tid < 35) cp_async4(scale_s + tid - 32, p.scale + (tid - 32));
+    if (tid >= 64 && tid < 64 + C) cp_async4(base_s + tid - 64, p.base + (tid - 64));
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+
+  // coefficient rows: their loads go out first
+  constexpr int V4 = RED / 4;
+  constexpr int GPT = kThreads / V4;                  // record groups per pass
+  constexpr int MAXK = (kMaxBlocks + GPT - 1) / GPT;  // passes for G <= 148
+  float4 cacc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.do_coeff && g < R) cacc = sum_row_partials<RED, MAXK>(p.dot_part, g, G, tid);
+
+  if (p.do_layer) {
+    if (!p.tail_broadcast)
+      for (int k = tid; k < R * N; k += kThreads) cp_async4(pre_s + k, p.pre + k);
+    // the blocks' sums of c^2 of rows warp + 8j (j < 4) for the first 32 rows
+    constexpr int MAXM = (kMaxBlocks + 31) / 32;
+    float sq[4][MAXM];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = warp + j * kWarps;
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        const int k = lane + 32 * m;
+        sq[j][m] = (r < R && k < G) ? __ldcg(p.sc2_part + r * G + k) : 0.f;
+      }
+    }
+    // this lane's stream vectors of every quad it normalises (at most 4 per warp)
+    uint4 sv[4][N];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int r = (warp + m * kWarps) * 4 + rq;
+      if (r < R) {
+        if (p.tail_broadcast) {
+          sv[m][0] = ld_v4(p.tail_streams + static_cast<size_t>(r) * H + h0);
+        } else {
+#pragma unroll
+          for (int j = 0; j < N; ++j) sv[m][j] = ld_v4(p.tail_streams + (static_cast<size_t>(r) * N + j) * H + h0);
+        }
+      }
+    }
+    cp_async_wait_all();
+    // ---- 7. per-row inverse RMS of the collapse: block sums added in a fixed order.
+    // Rows r0 + 8j, j < 4, reduced together: two halving steps leave row
+    // 2*(lane bit 4) + (lane bit 3) in each lane, three more steps sum it.
+    for (int r0 = warp; r0 < R; r0 += 4 * kWarps) {
+      if (r0 != warp) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = r0 + j * kWarps;
+#pragma unroll
+          for (int m = 0; m < MAXM; ++m) {
+            const int k = lane + 32 * m;
+            sq[j][m] = (r < R && k < G) ? __ldcg(p.sc2_part + r * G + k) : 0.f;
           }
         }
       }
-      red[C] = sv2;
-      red[C + 1] = sc2;
-      // ---- 3. reduce over the row's 8 lanes and publish this block's partial sums
-      reduce_scatter8<RED>(red, vec);
-      if (valid) {
-        float* dst = p.dot_part + (static_cast<size_t>(r) * G + g) * RED + vec * (RED / 8);
+      float a[4];
 #pragma unroll
-        for (int k = 0; k < RED / 8; ++k) dst[k] = red[k];
-        if (p.do_layer && vec == (C + 1) / (RED / 8)) p.sc2_part[r * G + g] = red[(C + 1) % (RED / 8)];
+      for (int j = 0; j < 4; ++j) {
+        a[j] = 0.f;
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) a[j] += sq[j][m];
       }
-    } else {
-      // layer input only: reduce sum c^2 over the row's 8 lanes
+      const bool hi4 = (lane & 16) != 0, hi3 = (lane & 8) != 0;
+      float b0 = (hi4 ? a[2] : a[0]) + __shfl_xor_sync(kFull, hi4 ? a[0] : a[2], 16);
+      float b1 = (hi4 ? a[3] : a[1]) + __shfl_xor_sync(kFull, hi4 ? a[1] : a[3], 16);
+      float c = (hi3 ? b1 : b0) + __shfl_xor_sync(kFull, hi3 ? b0 : b1, 8);
 #pragma unroll
-      for (int m = 4; m >= 1; m >>= 1) sc2 += __shfl_xor_sync(kFull, sc2, m);
-      if (valid && vec == 0) p.sc2_part[r * G + g] = sc2;
-    }
-  }
-  if (!p.do_layer && !p.do_coeff) return;
-  if (p.do_coeff && !fn_ready) {
-    // a warp with no rows still waits for the copy in flight into shared memory
-    if (!mbar_wait_bounded(bar, 0, deadline)) {
-      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-      aborted = true;
-    }
-  }
-  if (__syncthreads_or(aborted)) return;  // block-uniform
-
-  // ---- 4. all blocks' partial sums are in the workspace after this barrier
-  if (!grid_barrier(p.ctl + kBarCountWord, p.ctl + kBarGenWord, G + p.extra_arrivals, status, deadline,
-                    MHC_ERR_DEVICE_TIMEOUT, flag_s))
-    return;
-
-  if (p.do_layer) {
-    // ---- 4a. per-row inverse RMS of the collapse, summed over blocks in a fixed order
-    for (int r = warp; r < R; r += kWarps) {
-      float s = 0.f;
-      for (int k = lane; k < G; k += 32) s += __ldcg(p.sc2_part + r * G + k);
-      s = warp_sum(s);
-      if (lane == 0) inv_s[r] = rsqrtf(__fdiv_rn(s, static_cast<float>(H)) + p.norm_eps);
+      for (int mm = 4; mm >= 1; mm >>= 1) c += __shfl_xor_sync(kFull, c, mm);
+      const int r = r0 + (2 * (hi4 ? 1 : 0) + (hi3 ? 1 : 0)) * kWarps;
+      if ((lane & 7) == 0 && r < R) inv_s[r] = rsqrtf(__fdiv_rn(c, static_cast<float>(H)) + p.norm_eps);
     }
     __syncthreads();
-    // ---- 4b. layer input (and MXFP8) of this block's columns
+    // ---- 7b. layer input (and MXFP8) of this block's columns: the collapse is
+    // recomputed from the bf16 streams exactly as the streaming kernel summed c^2
     float w[8];
-    unpack8(ld_nc_v4(p.norm_weight + h0), w);
+    unpack8(*reinterpret_cast<const uint4*>(nw_s + vec * 8), w);
     const int scols = H / 32;
     const int col_tiles = (scols + 3) / 4;
-    for (int q = warp; q < nquads; q += kWarps) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int q = warp + m * kWarps;
       const int r = q * 4 + rq;
-      if (r >= R) continue;  // whole 4-lane MXFP8 groups share r: no shuffle crosses this
-      const float4* cs = reinterpret_cast<const float4*>(c_s + r * kCols);
-      const float4 c0 = cs[vec], c1 = cs[8 + vec];
-      const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      if (q >= nquads || r >= R) continue;  // whole 4-lane MXFP8 groups share r
+      float c[8];
+      if (p.tail_broadcast) {
+        unpack8(sv[m][0], c);
+      } else {
+        float nf[N][8];
+#pragma unroll
+        for (int j = 0; j < N; ++j) unpack8(sv[m][j], nf[j]);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < N; ++j) s = fmaf(pre_s[r * N + j], nf[j][t], s);
+          c[t] = s;
+        }
+      }
       const float inv = inv_s[r];
       float y[8], yr[8];
 #pragma unroll
@@ -485,11 +798,11 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
         unsigned char sbyte;
         if (grp == 0xfu) {
           const int e = e8m0_exponent(amax);
-          const float s = exp2_neg(e);
-          d.x = static_cast<unsigned>(e4m3x2(yr[0] * s, yr[1] * s)) |
-                (static_cast<unsigned>(e4m3x2(yr[2] * s, yr[3] * s)) << 16);
-          d.y = static_cast<unsigned>(e4m3x2(yr[4] * s, yr[5] * s)) |
-                (static_cast<unsigned>(e4m3x2(yr[6] * s, yr[7] * s)) << 16);
+          const float sc = exp2_neg(e);
+          d.x = static_cast<unsigned>(e4m3x2(yr[0] * sc, yr[1] * sc)) |
+                (static_cast<unsigned>(e4m3x2(yr[2] * sc, yr[3] * sc)) << 16);
+          d.y = static_cast<unsigned>(e4m3x2(yr[4] * sc, yr[5] * sc)) |
+                (static_cast<unsigned>(e4m3x2(yr[6] * sc, yr[7] * sc)) << 16);
           sbyte = static_cast<unsigned char>(e + 127);
         } else {
           d.x = d.y = 0x7f7f7f7fu;
@@ -523,83 +836,72 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
   }
 
   if (p.do_coeff) {
-    // ---- 4c. coefficients of rows g, g+G, ...: sum the blocks' partials in a fixed order
-    float* tot_s = red_s + kThreads;  // [RED]
-    float* lg_s = tot_s + 32;         // comb logits [N*N]
+    // ---- 8. coefficients of rows g, g+G, ...: logits, sigmoid, Sinkhorn
+    cp_async_wait_all();  // scale and base (already waited for with a layer input)
+    __syncthreads();
+    float4* part4 = reinterpret_cast<float4*>(red_s);  // [kWarps][V4]
     for (int r = g; r < R; r += G) {
-      __syncthreads();
-      {
-        const int v = tid % RED, sub = tid / RED;
-        constexpr int SUBS = kThreads / RED;
-        float s = 0.f;
-        for (int k = sub; k < G; k += SUBS) s += __ldcg(p.dot_part + (static_cast<size_t>(r) * G + k) * RED + v);
-        red_s[sub * RED + v] = s;
+      if (r != g) cacc = sum_row_partials<RED, MAXK>(p.dot_part, r, G, tid);
+      // sum the record groups of a warp (lane bits above log2(V4)), then the warps
+#pragma unroll
+      for (int m = V4; m < 32; m <<= 1) {
+        cacc.x += __shfl_xor_sync(kFull, cacc.x, m);
+        cacc.y += __shfl_xor_sync(kFull, cacc.y, m);
+        cacc.z += __shfl_xor_sync(kFull, cacc.z, m);
+        cacc.w += __shfl_xor_sync(kFull, cacc.w, m);
       }
       __syncthreads();
-      if (tid < RED) {
-        constexpr int SUBS = kThreads / RED;
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < SUBS; ++k) s += red_s[k * RED + tid];
-        tot_s[tid] = s;
-      }
+      if (lane < V4) part4[warp * V4 + lane] = cacc;
       __syncthreads();
-      if (tid < C) {
-        const float inv = rsqrtf(__fdiv_rn(tot_s[C], static_cast<float>(N * H)) + p.rms_eps);
-        const int grp = tid < N ? 0 : (tid < 2 * N ? 1 : 2);
-        const float l = p.scale[grp] * inv * tot_s[tid] + p.base[tid];
-        if (tid < N) {
-          p.pre_out[r * N + tid] = 1.f / (1.f + expf(-l)) + p.pre_eps;
-        } else if (tid < 2 * N) {
-          p.post_out[r * N + (tid - N)] = p.alpha / (1.f + expf(-l));
-        } else {
-          lg_s[tid - 2 * N] = l;
-        }
-      }
-      __syncthreads();
-      if (tid == 0) {
-        // Sinkhorn in registers: M = exp(L - max L); rows then columns, iters times
-        float M[N][N];
-        float mx = lg_s[0];
+      if (warp == 0) {
+        float s = 0.f;  // lane v: value v of the record
+        if (lane < RED) {
 #pragma unroll
-        for (int k = 1; k < N * N; ++k) mx = fmaxf(mx, lg_s[k]);
-#pragma unroll
-        for (int j = 0; j < N; ++j)
-#pragma unroll
-          for (int i = 0; i < N; ++i) M[j][i] = expf(lg_s[j * N + i] - mx);
-        for (int it = 0; it < p.iters; ++it) {
-#pragma unroll
-          for (int j = 0; j < N; ++j) {
-            float s = 0.f;
-#pragma unroll
-            for (int i = 0; i < N; ++i) s += M[j][i];
-            const float rcp = __frcp_rn(s + p.sk_eps);
-#pragma unroll
-            for (int i = 0; i < N; ++i) M[j][i] *= rcp;
-          }
-#pragma unroll
-          for (int i = 0; i < N; ++i) {
-            float s = 0.f;
-#pragma unroll
-            for (int j = 0; j < N; ++j) s += M[j][i];
-            const float rcp = __frcp_rn(s + p.sk_eps);
-#pragma unroll
-            for (int j = 0; j < N; ++j) M[j][i] *= rcp;
+          for (int w = 0; w < kWarps; ++w) {
+            const float4 a = part4[w * V4 + lane / 4];
+            s += (lane & 3) == 0 ? a.x : ((lane & 3) == 1 ? a.y : ((lane & 3) == 2 ? a.z : a.w));
           }
         }
+        const float inv = rsqrtf(__fdiv_rn(__shfl_sync(kFull, s, C), static_cast<float>(N * H)) + p.rms_eps);
+        const int grp = lane < N ? 0 : (lane < 2 * N ? 1 : 2);
+        const float l = lane < C ? scale_s[grp] * inv * s + base_s[lane] : 0.f;
+        if (lane < N) {
+          p.pre_out[r * N + lane] = 1.f / (1.f + expf(-l)) + p.pre_eps;
+        } else if (lane < 2 * N) {
+          p.post_out[r * N + (lane - N)] = p.alpha / (1.f + expf(-l));
+        }
+        // Sinkhorn in one thread: M = exp(L - max L); rows then columns, iters times
+        constexpr int NN = N * N;
+        float lc[NN];
 #pragma unroll
-        for (int j = 0; j < N; ++j)
+        for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, l, 2 * N + k);
+        if (lane == 0) {
+          float mx = lc[0];
 #pragma unroll
-          for (int i = 0; i < N; ++i) p.comb_out[(r * N + j) * N + i] = M[j][i];
+          for (int k = 1; k < NN; ++k) mx = fmaxf(mx, lc[k]);
+          float M[N][N];
+#pragma unroll
+          for (int j = 0; j < N; ++j)
+#pragma unroll
+            for (int i = 0; i < N; ++i) M[j][i] = expf(lc[j * N + i] - mx);
+          sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
+#pragma unroll
+          for (int j = 0; j < N; ++j)
+#pragma unroll
+            for (int i = 0; i < N; ++i) p.comb_out[r * NN + j * N + i] = M[j][i];
+        }
       }
     }
   }
 }
 
+
 // MXFP8 of a bf16 [R, H] matrix: a lane quantises 8 columns, 4 lanes a block.
 __global__ void __launch_bounds__(256) mxfp8_rows_kernel(const __nv_bfloat16* __restrict__ x, int R, int H,
                                                           uint8_t* __restrict__ data, uint8_t* __restrict__ scale,
                                                           int swizzled) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lanes_per_row = H / 8;
   const int scols = H / 32;
   const int col_tiles = (scols + 3) / 4;
@@ -651,6 +953,8 @@ __global__ void __launch_bounds__(256) mxfp8_rows_kernel(const __nv_bfloat16* __
 
 // Zero the padding bytes of a swizzled scale buffer (rows >= R or columns >= H/32).
 __global__ void scale_padding_kernel(uint8_t* scale, int R, int H) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int scols = H / 32;
   const int col_tiles = (scols + 3) / 4;
   const int rows_p = (R + 127) & ~127;
@@ -672,7 +976,7 @@ namespace {
 using namespace mhc;
 
 int64_t g_budget_ns = 1000000000LL;
-int g_extra_arrivals = 0;
+int g_extra_tx = 0;
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -705,41 +1009,58 @@ mhc_status check_mxfp8(const mhc_mxfp8_out* q) {
   return MHC_OK;
 }
 
-template <int N, int FRONT>
-mhc_status launch_boundary(Params& p, cudaStream_t stream) {
-  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
-  auto kern = boundary_kernel<N, FRONT>;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MHC_ERR_CUDA;
-  static int configured[64] = {0};
-  if (dev < 64 && configured[dev] < L.total) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
-      return MHC_ERR_CUDA;
-    configured[dev] = 200 * 1024;
-  }
-  const bool needs_barrier = p.do_layer || p.do_coeff;
-  p.extra_arrivals = g_extra_arrivals;
-  p.budget_ns = g_budget_ns;
+// Launch with programmatic stream serialization: the kernel may start while the
+// preceding kernel on the stream finishes, and waits for it (griddepcontrol.wait)
+// before reading anything that kernel may have written.
+template <typename Kern>
+mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const Params& p) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.H / kCols);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L.total;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = needs_barrier ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
-  if (e == cudaErrorCooperativeLaunchTooLarge) {
-    (void)cudaGetLastError();
-    return MHC_ERR_UNSUPPORTED_SHAPE;
-  }
-  if (e != cudaSuccess) {
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return MHC_ERR_CUDA;
   }
   return MHC_OK;
+}
+
+// Raise a kernel's dynamic shared memory limit once per device.
+template <typename Kern>
+bool allow_smem(Kern kern, int bytes, int* configured) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 64 || configured[dev] >= bytes) return dev < 64;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+    return false;
+  configured[dev] = 200 * 1024;
+  return true;
+}
+
+template <int N, int FRONT>
+mhc_status launch_boundary(Params& p, cudaStream_t stream) {
+  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
+  static int configured[64] = {0};
+  if (!allow_smem(boundary_kernel<N, FRONT>, L.total, configured)) return MHC_ERR_CUDA;
+  p.extra_tx = g_extra_tx;
+  p.budget_ns = g_budget_ns;
+  const int G = p.H / kCols;
+  mhc_status st = launch_pdl(boundary_kernel<N, FRONT>, G, L.total, stream, p);
+  if (st != MHC_OK || !(p.do_layer || p.do_coeff)) return st;
+  if (FRONT == kBroadcast) {
+    p.tail_streams = p.x;
+    p.tail_broadcast = 1;
+  } else {
+    p.tail_streams = FRONT == kStreams ? p.residual : p.residual_out;
+    p.tail_broadcast = 0;
+  }
+  return launch_pdl(boundary_tail_kernel<N>, G, tail_layout<N>(p.R).total, stream, p);
 }
 
 template <int FRONT>
@@ -988,19 +1309,31 @@ mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden, const mh
   if (rows < 1 || rows > 65535 || hidden < 32 || hidden % 32 != 0) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!x || !aligned(x, 16) || check_mxfp8(out) != MHC_OK || out == nullptr) return MHC_ERR_INVALID_ARG;
   const long long lanes = static_cast<long long>(rows) * (hidden / 8);
-  const int blocks = static_cast<int>((lanes + 255) / 256);
-  mxfp8_rows_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), rows, hidden, out->data,
-                                                 out->scale, out->swizzled_128x4 != 0);
-  if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((lanes + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, mxfp8_rows_kernel, reinterpret_cast<const __nv_bfloat16*>(x), rows, hidden, out->data,
+                         out->scale, static_cast<int>(out->swizzled_128x4 != 0)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MHC_ERR_CUDA;
+  }
   if (out->swizzled_128x4) {
     const int scols = hidden / 32;
     const int rows_p = (rows + 127) / 128 * 128;
     const int cols_p = (scols + 3) / 4 * 4;
     if (rows_p != rows || cols_p != scols) {
       const int total = rows_p * cols_p;
-      scale_padding_kernel<<<(total + 255) / 256 < 1024 ? (total + 255) / 256 : 1024, 256, 0, stream>>>(
-          out->scale, rows, hidden);
-      if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
+      cfg.gridDim = dim3((total + 255) / 256 < 1024 ? (total + 255) / 256 : 1024);
+      if (cudaLaunchKernelEx(&cfg, scale_padding_kernel, out->scale, rows, hidden) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MHC_ERR_CUDA;
+      }
     }
   }
   return MHC_OK;
@@ -1028,10 +1361,10 @@ const char* mhc_status_string(mhc_status s) {
   return "MHC_ERR_UNKNOWN";
 }
 
-int64_t mhc_debug_set_wait(int64_t budget_ns, int extra_arrivals) {
+int64_t mhc_debug_set_wait(int64_t budget_ns, int extra_units) {
   const int64_t old = g_budget_ns;
   if (budget_ns > 0) g_budget_ns = budget_ns;
-  g_extra_arrivals = extra_arrivals < 0 ? 0 : extra_arrivals;
+  g_extra_tx = extra_units < 0 ? 0 : extra_units;
   return old;
 }
 

@@ -11,13 +11,12 @@ namespace mhc {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-// ---------------------------------------------------------------- timers / waits
+// ---------------------------------------------------------------- waits
 
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+// The bounded waits count SM cycles (clock64 is a register read; %globaltimer
+// costs about a microsecond per read on this part). A budget of T ns is granted
+// as 2*T cycles: at clocks up to 2 GHz the wait lasts at least T ns.
+__device__ __forceinline__ long long wait_deadline(int64_t budget_ns) { return clock64() + 2 * budget_ns; }
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -37,7 +36,8 @@ __device__ __forceinline__ unsigned smem_u32(const void* p) {
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  // make the initialised barrier visible to the async proxy (the TMA engine)
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
@@ -67,13 +67,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`, giving up at `deadline` (globaltimer ns).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, uint64_t deadline) {
+// Wait for phase `parity` of `bar`, giving up at `deadline` (clock64 cycles).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, long long deadline) {
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() > deadline) return false;
+    if (clock64() > deadline) return false;
   }
   return true;
 }
+
+// ---------------------------------------------------------------- small async copies / L2 prefetch
+
+// 4-byte global -> shared copy that does not occupy a register (LDGSTS); all
+// copies of a thread complete at cp_async_wait_all.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most one (the most recent) committed group of this thread is in flight.
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // ---------------------------------------------------------------- global vector loads / stores
 
@@ -126,6 +147,13 @@ __device__ __forceinline__ uint4 round8(const float (&f)[8], float (&r)[8]) {
   return v;
 }
 
+// Approximate reciprocal (MUFU, <= 1 ulp): the Sinkhorn normalisations.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // ---------------------------------------------------------------- MXFP8 encoders
 
 // Exponent e of an MXFP8 block whose largest magnitude is `amax` (a finite,
@@ -153,42 +181,24 @@ __device__ __forceinline__ unsigned short e4m3x2(float lo, float hi) {
   return r;
 }
 
-// ---------------------------------------------------------------- grid barrier
+// ---------------------------------------------------------------- cross-block flags, dependent launch
 
-// Self-resetting barrier over all blocks of the grid, with a bounded wait.
-// ctl[kBarCount] counts arrivals, ctl[kBarGen] is the generation. A block reads
-// the generation before it arrives; the last arriver resets the count and then
-// bumps the generation, which releases the others. Every block must call it the
-// same number of times. Returns false (and records MHC_ERR_DEVICE_TIMEOUT) when
-// the wait ran past `deadline`; the barrier state is then unusable until the
-// workspace is zeroed again.
-__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned* gen, unsigned expected,
-                                             unsigned* status, uint64_t deadline, unsigned timeout_code,
-                                             int* flag_smem) {
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    bool ok = true;
-    const unsigned my_gen = ld_acquire_gpu(gen);
-    const unsigned old = atomicAdd(count, 1u);
-    if (old == expected - 1) {
-      atomicExch(count, 0u);
-      __threadfence();
-      atomicAdd(gen, 1u);
-    } else {
-      while (ld_acquire_gpu(gen) == my_gen) {
-        if (global_ns() > deadline) {
-          record_error(status, timeout_code);
-          ok = false;
-          break;
-        }
-        __nanosleep(20);
-      }
-    }
-    *flag_smem = ok ? 1 : 0;
-  }
-  __syncthreads();
-  return *flag_smem != 0;
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Programmatic dependent launch: wait for the preceding grid on the stream to
+// complete (and its memory to be visible); a no-op when launched normally.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid on the stream (launched with programmatic serialization)
+// to start once every block of this grid has executed this.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 }  // namespace mhc

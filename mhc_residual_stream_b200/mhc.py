@@ -188,8 +188,10 @@ def mhc_get_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().mhc_get_device_status(_p(workspace), _stream(stream)))
 
 
-def mhc_debug_set_wait(budget_ns: int, extra_arrivals: int) -> int:
-    return int(lib().mhc_debug_set_wait(int(budget_ns), int(extra_arrivals)))
+def mhc_debug_set_wait(budget_ns: int, extra_units: int) -> int:
+    """Test hook: the time limit of the kernels' bounded wait, and extra 16-byte
+    units that wait should expect (so that it runs out)."""
+    return int(lib().mhc_debug_set_wait(int(budget_ns), int(extra_units)))
 
 
 # ------------------------------------------------------------------ entry points

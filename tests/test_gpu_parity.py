@@ -306,10 +306,13 @@ def test_mxfp8_nonfinite_block():
 
 # ---------------------------------------------------------------- bounded waits
 
-def test_barrier_wait_times_out_and_recovers():
+def test_weight_copy_wait_times_out_and_recovers():
+    # the wait on the fn slice's TMA copies expects one 16-byte unit that never
+    # comes: it must give up after its budget and record the timeout, and the
+    # next boundary must be correct
     d = S.draw_boundary(4, 256, n=4, partials=2, seed=9)
     ws = M.new_workspace(4, 256, 4, DEV)
-    old = M.mhc_debug_set_wait(20_000_000, 1)  # 20 ms, one arrival that never comes
+    old = M.mhc_debug_set_wait(20_000_000, 1)  # 20 ms
     try:
         g = to_dev(d)
         out = alloc_outputs(4, 4, 256)
@@ -320,7 +323,7 @@ def test_barrier_wait_times_out_and_recovers():
         assert M.mhc_get_device_status(ws) == M.DEVICE_TIMEOUT
     finally:
         M.mhc_debug_set_wait(old, 0)
-    M.mhc_workspace_init(ws)
+    assert M.mhc_get_device_status(ws) == M.OK  # reading cleared it
     gpu = gpu_post_pre(d, ws=ws)
     orc = oracle_post_pre(d)
     check_tail(d, gpu, orc, what="after recovery")
