@@ -204,6 +204,31 @@ MHC_API mhc_status mhc_coeffs(
 MHC_API mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden,
                                const mhc_mxfp8_out* out, mhc_stream stream);
 
+/* mhc_boundary_post_pre for callers that cannot allocate device memory.
+ * The pages have no counterpart: this entry point exists for callers such as a
+ * plugin hosted by a runtime that owns all device memory (it is only handed
+ * tensors), code running while a CUDA graph is captured (cudaMalloc is not a
+ * stream operation), or a serving loop that must not take the allocator's locks.
+ * Arguments and results are those of mhc_boundary_post_pre without the
+ * workspace: the scratch is a fixed device array inside the library, 1,893,376
+ * bytes (the workspace of rows 128, hidden 7168, hc_mult 4), which every GPU
+ * that loads the library holds until the process exits. Limits: rows <= 128,
+ * hidden <= 7168, hc_mult <= 4; larger shapes return MHC_ERR_WORKSPACE.
+ * The first call on a device looks up the array's device address (one
+ * cudaGetSymbolAddress per device, with that device current); make that first
+ * call before any stream capture. Every call on a device shares the array:
+ * calls that overlap on the GPU (other streams, other threads) race on it and
+ * must be serialised by the caller. A kernel-side error (a wait that ran out) is
+ * recorded in the array and not reported; use mhc_boundary_post_pre with a
+ * workspace to read it. Allocates nothing. */
+MHC_API mhc_status mhc_boundary_post_pre_noalloc(
+    const mhc_bf16* partials, int num_partials, int64_t partial_stride,
+    const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
+    const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+    mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    float* post_out, float* comb_out, float* pre_out,
+    int rows, int hidden, int hc_mult, mhc_stream stream);
+
 /* Wait for `stream`, then read and clear the error a kernel recorded in
  * `workspace` (MHC_OK when none). The only entry point that synchronises. */
 MHC_API mhc_status mhc_get_device_status(void* workspace, mhc_stream stream);

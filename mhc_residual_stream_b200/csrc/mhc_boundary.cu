@@ -27,6 +27,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/mhc.h"
 #include "mhc_device.cuh"
 
@@ -1366,6 +1368,73 @@ int64_t mhc_debug_set_wait(int64_t budget_ns, int extra_units) {
   if (budget_ns > 0) g_budget_ns = budget_ns;
   g_extra_tx = extra_units < 0 ? 0 : extra_units;
   return old;
+}
+
+// ---------------------------------------------------------------------------
+// Boundary without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory: a plugin hosted by a runtime
+// that owns all device memory and only hands it tensors, code that runs while
+// a CUDA graph is being captured (cudaMalloc is not a stream operation), or a
+// serving loop that must never take the allocator's locks. For them the
+// scratch of mhc_boundary_post_pre lives in the fixed array below, which every
+// GPU that loads the library holds until the process exits.
+
+}  // extern "C"
+
+namespace {
+
+constexpr int kNoAllocMaxRows = 128;
+constexpr int kNoAllocMaxHidden = 7168;
+constexpr int kNoAllocMaxHc = 4;
+// mhc_workspace_bytes(128, 7168, 4): header, c^2 sums [128][112] (rounded to
+// 256 bytes), projection sums [128][112][32] floats
+constexpr size_t kNoAllocBytes = kWsHeader + ((static_cast<size_t>(kNoAllocMaxRows) * (kNoAllocMaxHidden / kCols) * 4 + 255) & ~static_cast<size_t>(255)) +
+                                 static_cast<size_t>(kNoAllocMaxRows) * (kNoAllocMaxHidden / kCols) * red_of(kNoAllocMaxHc) * 4;
+
+// The array is zero at module load. A kernel never needs its contents to start
+// at zero except the status word, which only a failed wait writes.
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of the array on the current device, looked up once per device.
+// In host code the symbol is only a host-side stand-in; the kernels get this.
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+mhc_status mhc_boundary_post_pre_noalloc(const mhc_bf16* partials, int num_partials, int64_t partial_stride,
+                                         const mhc_bf16* residual, const float* post, const float* comb,
+                                         const float* pre, const mhc_bf16* norm_weight, float norm_eps,
+                                         const mhc_coeff_args* coeffs, mhc_bf16* residual_out,
+                                         mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out,
+                                         float* comb_out, float* pre_out, int rows, int hidden, int hc_mult,
+                                         mhc_stream stream) {
+  if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (rows > kNoAllocMaxRows || hidden > kNoAllocMaxHidden || hc_mult > kNoAllocMaxHc ||
+      ws_layout(rows, hidden, hc_mult, nullptr, nullptr) > kNoAllocBytes)
+    return MHC_ERR_WORKSPACE;  // needs more scratch than the fixed array holds
+  void* ws = noalloc_scratch();
+  if (ws == nullptr) return MHC_ERR_CUDA;
+  return mhc_boundary_post_pre(partials, num_partials, partial_stride, residual, post, comb, pre, norm_weight,
+                               norm_eps, coeffs, residual_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
+                               hidden, hc_mult, ws, kNoAllocBytes, stream);
 }
 
 }  // extern "C"

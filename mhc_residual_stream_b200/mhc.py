@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         "mhc_workspace_init": (_i, [_vp, _sz, _vp]),
         "mhc_boundary_post_pre": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+        "mhc_boundary_post_pre_noalloc": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+                                               _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
         "mhc_boundary_moe_finalize": (_i, [_vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _f, _vp,
                                            _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
         "mhc_boundary_residual_only": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
@@ -242,6 +244,25 @@ def mhc_boundary_post_pre(partials, residual, post, comb, pre, norm_weight, norm
         _ref(cs), _p(residual_out), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
         R, H, n, _p(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "mhc_boundary_post_pre")
+
+
+def mhc_boundary_post_pre_noalloc(partials, residual, post, comb, pre, norm_weight, norm_eps,
+                                  coeffs: Optional[Coeffs], residual_out, layer_input=None, mxfp8=None,
+                                  post_out=None, comb_out=None, pre_out=None, stream=None):
+    """mhc_boundary_post_pre without a workspace, for callers that cannot allocate
+    device memory (a runtime that owns all memory, graph capture, allocation-free
+    serving loops): the scratch is a fixed array inside the library. Limits:
+    rows <= 128, hidden <= 7168, hc_mult <= 4. Calls on one device must not
+    overlap on the GPU."""
+    R, n, H = _mix_args(residual, post, comb, residual_out)
+    P, stride = _partials_args(partials, R, H)
+    _tail_args(pre, norm_weight, layer_input, post_out, comb_out, pre_out, R, n, H)
+    cs, qs = _coeff_struct(coeffs), _mxfp8_struct(mxfp8)
+    st = lib().mhc_boundary_post_pre_noalloc(
+        _p(partials), P, stride, _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight), float(norm_eps),
+        _ref(cs), _p(residual_out), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
+        R, H, n, _stream(stream))
+    _check(st, "mhc_boundary_post_pre_noalloc")
 
 
 def mhc_boundary_moe_finalize(gemm2_permuted, expert_weights, expanded_idx_to_permuted_idx, shared_output,
