@@ -17,9 +17,9 @@
 //      with register-tiled CUDA-core FMA (8 rows x C/4 columns per thread) and
 //      writes its partial sums to the workspace.
 // The tail kernel (boundary_tail_kernel), once the streaming kernel is done:
-//   4. every block normalises its own columns into the layer input (and MXFP8),
-//      and block g finishes the coefficients (logits, sigmoid, Sinkhorn with one
-//      comb element per lane) of rows g, g+G, ...
+//   4. blocks 0..G-1 normalise their columns into the layer input (and MXFP8);
+//      at the same time further blocks finish the coefficients (logits, sigmoid,
+//      Sinkhorn in one thread) of rows j, j + Gc, ...
 // The residual-only variant is the streaming kernel alone. All reductions run
 // in a fixed order, so results are bitwise reproducible.
 
@@ -103,32 +103,41 @@ struct Params {
   // embedding of the first layer (whose identity pre-mix selects it)
   const __nv_bfloat16* tail_streams;
   int tail_broadcast;
+  int tail_layer_blocks;  // tail blocks [0, this) write the layer input (G or 0)
+  int tail_coeff_blocks;  // the next ones finish the coefficients of rows j, j + this, ...
   int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
   int64_t budget_ns;
 };
 
 struct SmemLayout {
-  int fn_off, v_off, mix_off, moe_off, xs_off, misc_off, total;
+  int fn_off, bs_off, v_off, mix_off, moe_off, red_off, misc_off, total;
 };
+
+// Projection operands: n-tiles of 8 logit columns; staged stream rows and fn
+// columns are n*64 bf16 plus a 16-byte gap (ldmatrix rows in distinct banks).
+__host__ __device__ constexpr int ntiles_of(int n) { return (logits_of(n) + 7) / 8; }
+__host__ __device__ constexpr int kstride_of(int n) { return n * kCols + 8; }
 
 // Shared memory of the streaming kernel.
 template <int N>
 __host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe) {
-  constexpr int CP = cpad_of(N);
+  constexpr int CP8 = ntiles_of(N) * 8;
   SmemLayout L{};
   int o = 0;
-  L.fn_off = o;
+  L.fn_off = o;  // fn slice as the bulk copies land it
   o += N * 8 * fn_piece_bytes(N);
-  L.v_off = o;  // new streams, bf16 [R][n*64]
-  o += R * N * kCols * 2;
+  L.bs_off = o;  // fn slice as three bf16 terms, [3][CP8][n*64 + 8]
+  o += 3 * CP8 * kstride_of(N) * 2;
+  L.v_off = o;  // new streams, bf16 [roundup(R, 16)][n*64 + 8]
+  o += ((R + 15) & ~15) * kstride_of(N) * 2;
   L.mix_off = o;  // [R][post n | comb n*n | pre n]
   o += R * (2 * N + N * N) * 4;
   o = (o + 15) & ~15;
   L.moe_off = o;
   if (moe) o += R * topk * 8;
   o = (o + 15) & ~15;
-  L.xs_off = o;  // projection: the second half-K warp's sums, [4][8][CP]
-  o += 4 * 8 * CP * 4;
+  L.red_off = o;  // per-warp projection sums of a 32-row chunk, [8][32][CP8]
+  o += kWarps * 32 * CP8 * 4;
   L.misc_off = o;  // mbarrier
   o += 16;
   L.total = o;
@@ -252,23 +261,24 @@ __device__ __forceinline__ void load_quad(const Params& p, int r, int h0, const 
 }
 
 template <int N, int FRONT>
-__global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   constexpr int C = logits_of(N);
-  constexpr int CP = cpad_of(N);
-  constexpr int CT = CP / 4;     // projection columns per thread
-  constexpr int KC = N * kCols;  // stream values per row in this block
-  constexpr int KPT = KC / 16;   // of which one projection thread owns KPT consecutive ones
+  constexpr int KC = N * kCols;       // stream values per row in this block
+  constexpr int KS = kstride_of(N);   // staged row stride (bf16)
+  constexpr int NT = ntiles_of(N);    // 8-column tiles of the projection
+  constexpr int CP8 = NT * 8;
   constexpr int RED = red_of(N);
   constexpr int MIX = 2 * N + N * N;
   constexpr int PIECE = fn_piece_bytes(N);
   extern __shared__ __align__(128) unsigned char smem[];
   const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
   unsigned char* fn_s = smem + L.fn_off;
+  __nv_bfloat16* bs_s = reinterpret_cast<__nv_bfloat16*>(smem + L.bs_off);
   __nv_bfloat16* v_s = reinterpret_cast<__nv_bfloat16*>(smem + L.v_off);
   float* mix_s = reinterpret_cast<float*>(smem + L.mix_off);
   int* e2p_s = reinterpret_cast<int*>(smem + L.moe_off);
   float* ew_s = reinterpret_cast<float*>(smem + L.moe_off) + p.R * p.topk;
-  float* xs_s = reinterpret_cast<float*>(smem + L.xs_off);
+  float* red_s = reinterpret_cast<float*>(smem + L.red_off);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.misc_off);
 
   const int g = blockIdx.x;
@@ -323,6 +333,26 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
     }
   }
 
+  if (p.do_coeff) {
+    // Split the fn slice into three bf16 terms, f = hi + mid + lo to 2^-24,
+    // stored column-major for the MMA's B operand (weights only: before the wait).
+    // Each bf16 x bf16 product is exact in fp32, so the tensor cores return the
+    // fp32 projection up to the order of the fp32 additions.
+    const bool ok = mbar_wait_bounded(bar, 0, deadline);
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
+    for (int e = tid; e < CP8 * KC; e += kThreads) {
+      const int c = e / KC, k = e - c * KC;
+      const float f = c < C ? reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4)[c] : 0.f;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(f);
+      const float r1 = f - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+      bs_s[(0 * CP8 + c) * KS + k] = hi;
+      bs_s[(1 * CP8 + c) * KS + k] = mid;
+      bs_s[(2 * CP8 + c) * KS + k] = lo;
+    }
+  }
   // ---- 3. wait for the preceding kernel, let the next one launch, and read
   griddep_wait();
   griddep_launch_dependents();
@@ -486,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
       sv2 = sum8_lanes(sv2);
       if (valid) {
 #pragma unroll
-        for (int i = 0; i < N; ++i) *reinterpret_cast<uint4*>(v_s + r * KC + i * kCols + vec * 8) = nb[i];
+        for (int i = 0; i < N; ++i) *reinterpret_cast<uint4*>(v_s + r * KS + i * kCols + vec * 8) = nb[i];
         if (vec == 0) p.dot_part[(static_cast<size_t>(r) * G + g) * RED + C] = sv2;
       }
     }
@@ -495,97 +525,59 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_kernel(const Params p) {
   if (!p.do_coeff) return;
 
   // ---- 5. projection of this block's n*64 stream values per row onto the C fn
-  // columns (CUDA-core FMA). Thread (cg, ks, rs) owns 8 rows x C/4 columns over
-  // the KPT consecutive stream values from ks*KPT: each fn value it loads feeds
-  // 8 rows, each stream value C/4 columns. 64-bit loads of fn are bank-conflict
-  // free for a half-warp in the bulk-copy layout.
-  if (p.do_coeff) {
-    const bool ok = mbar_wait_bounded(bar, 0, deadline);
-    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-    if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
-    const int cg = tid & 3, ks = (tid >> 2) & 15, rs = tid >> 6, ksl = ks & 7, half = ks >> 3;
-    for (int rb = 0; rb < R; rb += 32) {
-      const int r0 = rb + rs * 8;
-      float acc[8][CT];
+  // columns on the tensor cores: [rows x n*64] bf16 x [n*64 x C] as three bf16
+  // terms, fp32 accumulation (mma.sync m16n8k16). Warp w takes the k-steps
+  // w, w+8, ... of every 16-row tile and 8-column tile of a 32-row chunk; the
+  // warps' sums are added in warp order.
+  __syncthreads();  // staged streams
+  for (int rb = 0; rb < R; rb += 32) {
+    float acc[2][NT][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int c = 0; c < CT; ++c) acc[j][c] = 0.f;
-      if (r0 < R) {  // uniform over the warp (rs is)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int kk = 0; kk < KPT; kk += 2) {
-          const int k = ks * KPT + kk;
-          const float* frow = reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4) + cg * CT;
-          float f0[CT], f1[CT];
-          if constexpr (CT % 2 == 0) {
+        for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.f;
+    const bool two = rb + 16 < R;  // second 16-row tile of the chunk in use
+    for (int kstep = warp; kstep < KC / 16; kstep += kWarps) {
+      const int k0 = kstep * 16;
+      unsigned a[2][4];
+      ldmatrix_x4(a[0], v_s + (rb + (lane & 15)) * KS + k0 + (lane >> 4) * 8);
+      if (two) ldmatrix_x4(a[1], v_s + (rb + 16 + (lane & 15)) * KS + k0 + (lane >> 4) * 8);
 #pragma unroll
-            for (int c = 0; c < CT; c += 2) {
-              const float2 a = *reinterpret_cast<const float2*>(frow + c);
-              const float2 b = *reinterpret_cast<const float2*>(frow + C + c);
-              f0[c] = a.x;
-              f0[c + 1] = a.y;
-              f1[c] = b.x;
-              f1[c + 1] = b.y;
-            }
-          } else {
+      for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-            for (int c = 0; c < CT; ++c) {
-              f0[c] = frow[c];
-              f1[c] = frow[C + c];
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int r = r0 + j;
-            const unsigned w2 = r < R ? *reinterpret_cast<const unsigned*>(v_s + r * KC + k) : 0u;
-            const float v0 = __uint_as_float(w2 << 16), v1 = __uint_as_float(w2 & 0xffff0000u);
-            if constexpr (CT % 2 == 0) {
-#pragma unroll
-              for (int c = 0; c < CT; c += 2) {
-                float2 a = make_float2(acc[j][c], acc[j][c + 1]);
-                a = __ffma2_rn(make_float2(v0, v0), make_float2(f0[c], f0[c + 1]), a);
-                a = __ffma2_rn(make_float2(v1, v1), make_float2(f1[c], f1[c + 1]), a);
-                acc[j][c] = a.x;
-                acc[j][c + 1] = a.y;
-              }
-            } else {
-#pragma unroll
-              for (int c = 0; c < CT; ++c) acc[j][c] = fmaf(v1, f1[c], fmaf(v0, f0[c], acc[j][c]));
-            }
-          }
-        }
-        // reduce over the 8 ks of this warp (lane bits 2-4), scattering the rows:
-        // lane with ksl keeps row r0 + ksl
-#pragma unroll
-        for (int s = 0; s < 3; ++s) {
-          const int mask = 16 >> s;
-          const int hj = 4 >> s;
-          const bool up = (ksl & (4 >> s)) != 0;
-#pragma unroll
-          for (int j = 0; j < hj; ++j)
-#pragma unroll
-            for (int c = 0; c < CT; ++c) {
-              const float send = up ? acc[j][c] : acc[j + hj][c];
-              const float keep = up ? acc[j + hj][c] : acc[j][c];
-              acc[j][c] = keep + __shfl_xor_sync(kFull, send, mask);
-            }
-        }
-        if (half == 1) {
-#pragma unroll
-          for (int c = 0; c < CT; ++c) xs_s[(rs * 8 + ksl) * CP + cg * CT + c] = acc[0][c];
+        for (int sp = 0; sp < 3; ++sp) {
+          unsigned b[2];
+          ldmatrix_x2(b, bs_s + (sp * CP8 + nt * 8 + (lane & 7)) * KS + k0 + ((lane >> 3) & 1) * 8);
+          mma_bf16_16816(acc[0][nt], a[0], b);
+          if (two) mma_bf16_16816(acc[1][nt], a[1], b);
         }
       }
-      __syncthreads();
-      if (r0 < R && half == 0 && r0 + ksl < R) {
-        float* dst = p.dot_part + (static_cast<size_t>(r0 + ksl) * G + g) * RED;
-#pragma unroll
-        for (int c = 0; c < CT; ++c) {
-          const int cc = cg * CT + c;
-          if (cc < C) dst[cc] = acc[0][c] + xs_s[(rs * 8 + ksl) * CP + cc];
-        }
-      }
-      __syncthreads();
     }
+    // C fragment: lane holds rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int row = mt * 16 + (lane >> 2), col = nt * 8 + 2 * (lane & 3);
+        float* dst = red_s + (warp * 32 + row) * CP8 + col;
+        dst[0] = acc[mt][nt][0];
+        dst[1] = acc[mt][nt][1];
+        dst[8 * CP8] = acc[mt][nt][2];
+        dst[8 * CP8 + 1] = acc[mt][nt][3];
+      }
+    __syncthreads();
+    for (int e = tid; e < 32 * C; e += kThreads) {
+      const int row = e / C, col = e - row * C, r = rb + row;
+      if (r < R) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) sum += red_s[(w * 32 + row) * CP8 + col];
+        p.dot_part[(static_cast<size_t>(r) * G + g) * RED + col] = sum;
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -646,12 +638,12 @@ __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, fl
 }
 
 // The tail of a boundary, launched after the streaming kernel (programmatic
-// dependent launch): once every block's partial sums are in the workspace,
-// block g normalises columns [64g, 64g+64) of every row into the layer input
-// (and MXFP8), recomputing the collapse from the bf16 streams (L2-resident), and
-// finishes the coefficients of rows g, g+G, ...
+// dependent launch). Once every block's partial sums are in the workspace,
+// layer-input block g normalises columns [64g, 64g+64) of every row into the
+// layer input (and MXFP8), recomputing the collapse from the bf16 streams
+// (L2-resident), while coefficient block j finishes rows j, j + Gc, ...
 template <int N>
-__global__ void __launch_bounds__(kThreads, 1) boundary_tail_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params p) {
   constexpr int C = logits_of(N);
   constexpr int CP = cpad_of(N);
   constexpr int RED = red_of(N);
@@ -664,32 +656,20 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_tail_kernel(const Params
   float* scale_s = reinterpret_cast<float*>(smem + L.cst_off + kCols * 2);
   float* base_s = scale_s + 4;
 
-  const int g = blockIdx.x;
-  const int G = gridDim.x;
+  const int G = p.H / kCols;
   const int H = p.H;
   const int R = p.R;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rq = lane >> 3, vec = lane & 7;
-  const int h0 = g * kCols + vec * 8;
   const int nquads = (R + 3) >> 2;
+  const bool layer_role = static_cast<int>(blockIdx.x) < p.tail_layer_blocks;
 
-  // weights before the wait on the streaming kernel
-  if (p.do_layer && tid < 8) cp_async16(nw_s + tid * 8, p.norm_weight + g * kCols + tid * 8);
-  if (p.do_coeff) {
-    if (tid >= 32 && tid < 35) cp_async4(scale_s + tid - 32, p.scale + (tid - 32));
-    if (tid >= 64 && tid < 64 + C) cp_async4(base_s + tid - 64, p.base + (tid - 64));
-  }
-  griddep_wait();
-  griddep_launch_dependents();
-
-  // coefficient rows: their loads go out first
-  constexpr int V4 = RED / 4;
-  constexpr int GPT = kThreads / V4;                  // record groups per pass
-  constexpr int MAXK = (kMaxBlocks + GPT - 1) / GPT;  // passes for G <= 148
-  float4 cacc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (p.do_coeff && g < R) cacc = sum_row_partials<RED, MAXK>(p.dot_part, g, G, tid);
-
-  if (p.do_layer) {
+  if (layer_role) {
+    const int g = blockIdx.x;
+    const int h0 = g * kCols + vec * 8;
+    if (tid < 8) cp_async16(nw_s + tid * 8, p.norm_weight + g * kCols + tid * 8);  // weights: before the wait
+    griddep_wait();
+    griddep_launch_dependents();
     if (!p.tail_broadcast)
       for (int k = tid; k < R * N; k += kThreads) cp_async4(pre_s + k, p.pre + k);
     // the blocks' sums of c^2 of rows warp + 8j (j < 4) for the first 32 rows
@@ -835,15 +815,22 @@ __global__ void __launch_bounds__(kThreads, 1) boundary_tail_kernel(const Params
         }
       }
     }
-  }
-
-  if (p.do_coeff) {
-    // ---- 8. coefficients of rows g, g+G, ...: logits, sigmoid, Sinkhorn
-    cp_async_wait_all();  // scale and base (already waited for with a layer input)
+  } else {
+    // coefficient rows j, j + tail_coeff_blocks, ...: sum the blocks' partials in a
+    // fixed order, logits, sigmoid, Sinkhorn
+    const int jb = blockIdx.x - p.tail_layer_blocks;
+    if (tid < 3) cp_async4(scale_s + tid, p.scale + tid);  // weights: before the wait
+    if (tid >= 32 && tid < 32 + C) cp_async4(base_s + tid - 32, p.base + (tid - 32));
+    griddep_wait();
+    griddep_launch_dependents();
+    constexpr int V4 = RED / 4;
+    constexpr int GPT = kThreads / V4;                  // record groups per pass
+    constexpr int MAXK = (kMaxBlocks + GPT - 1) / GPT;  // passes for G <= 148
+    cp_async_wait_all();
     __syncthreads();
     float4* part4 = reinterpret_cast<float4*>(red_s);  // [kWarps][V4]
-    for (int r = g; r < R; r += G) {
-      if (r != g) cacc = sum_row_partials<RED, MAXK>(p.dot_part, r, G, tid);
+    for (int r = jb; r < R; r += p.tail_coeff_blocks) {
+      float4 cacc = sum_row_partials<RED, MAXK>(p.dot_part, r, G, tid);
       // sum the record groups of a warp (lane bits above log2(V4)), then the warps
 #pragma unroll
       for (int m = V4; m < 32; m <<= 1) {
@@ -1033,6 +1020,19 @@ mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const 
   return MHC_OK;
 }
 
+// Number of SMs of the current device (cached per device).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kMaxBlocks;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return kMaxBlocks;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 // Raise a kernel's dynamic shared memory limit once per device.
 template <typename Kern>
 bool allow_smem(Kern kern, int bytes, int* configured) {
@@ -1062,7 +1062,12 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
     p.tail_streams = FRONT == kStreams ? p.residual : p.residual_out;
     p.tail_broadcast = 0;
   }
-  return launch_pdl(boundary_tail_kernel<N>, G, tail_layout<N>(p.R).total, stream, p);
+  // coefficient blocks run beside the G layer-input blocks, on the SMs those leave
+  p.tail_layer_blocks = p.do_layer ? G : 0;
+  const int spare = sm_count() - p.tail_layer_blocks;
+  p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
+  return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>(p.R).total,
+                    stream, p);
 }
 
 template <int FRONT>
