@@ -366,7 +366,9 @@ def ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": load_traffic(),
                      "algorithmic_bytes": bpb, "peak_kind": f"{peak_kind} (copy bandwidth)",
-                     "kernel": "boundary_kernel<4, partials>"},
+                     "kernel": "boundary_kernel<4, partials> + boundary_tail_kernel<4>: the two launches "
+                               "of one boundary, timed together; traffic is the streaming kernel's "
+                               "DRAM bytes per launch (the tail reads L2)"},
         "gpu_launches": args.steps,
     }
     if sampler is not None:
