@@ -153,6 +153,11 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
+# fn is packed once, at weight-load time, into the projection's bf16-term tiles
+# (mhc_projection_pack); --unpacked-fn times the kernels splitting fp32 fn per call
+PACK_FN = True
+
+
 class BoundarySet:
     """Device buffers of one boundary of the benchmark workload."""
 
@@ -167,7 +172,9 @@ class BoundarySet:
         self.comb = d["comb"].to(device)
         self.pre = d["pre"].to(device)
         self.norm_weight = d["norm_weight"].to(device)
-        self.coeffs = M.Coeffs.from_weights(d["coeff"], device)
+        self.coeffs = M.Coeffs.from_weights(d["coeff"], device, packed=PACK_FN)
+        if PACK_FN:
+            self.coeffs.fn = None  # the kernels read the packed form only
         self.residual_out = torch.empty_like(self.residual)
         self.layer_input = torch.empty(R, HIDDEN, dtype=torch.bfloat16, device=device)
         self.q_data = torch.empty(R, HIDDEN, dtype=torch.uint8, device=device) if mxfp8 else None
@@ -335,7 +342,8 @@ def ours(args):
     sets = [BoundarySet(ROWS, 900000 + 97 * i + 1000 * rank, device) for i in range(nsets)]
     ws = M.new_workspace(ROWS, HIDDEN, HC, device)
     set_bytes = sum(t.numel() * t.element_size() for s in sets[:1] for t in
-                    (s.partials, s.residual, s.coeffs.fn, s.residual_out, s.layer_input, s.q_data))
+                    (s.partials, s.residual, s.coeffs.fn if s.coeffs.fn is not None else s.coeffs.fn_packed,
+                     s.residual_out, s.layer_input, s.q_data))
     assert set_bytes * nsets > 2 * L2_BYTES
     graph_len = 240
     main, tail = timed_graph_steps(sets, ws, args.steps, args.warmup, graph_len)
@@ -361,6 +369,8 @@ def ours(args):
                    "rows": ROWS, "hidden": HIDDEN, "hc_mult": HC, "partials": PARTIALS,
                    "l2": f"inputs larger than L2: {nsets} rotating buffer sets, {set_bytes * nsets / 1e6:.0f} MB",
                    "timing": "CUDA graphs of 240 boundaries, CUDA events on the launching stream",
+                   "fn": ("packed once at weight load (mhc_projection_pack)" if PACK_FN
+                          else "fp32, split into bf16 terms in every call"),
                    "parallelism": f"replicas x{world}"},
         "gb_per_s": round(achieved * world, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -369,7 +379,7 @@ def ours(args):
                      "kernel": "boundary_kernel<4, partials> + boundary_tail_kernel<4>: the two launches "
                                "of one boundary, timed together; traffic is the streaming kernel's "
                                "DRAM bytes per launch (the tail reads L2)"},
-        "gpu_launches": args.steps,
+        "gpu_launches": 2 * args.steps,
     }
     if sampler is not None:
         result["clocks"] = sampler.summary()
@@ -390,7 +400,7 @@ def ours(args):
         result["rows_sweep"] = sweep
         # one decode step: the 123 chained boundaries of the 61-layer loop at rows 32
         from mhc_residual_stream_b200.decode import DecodeLoop
-        loop = DecodeLoop(rows=ROWS, device=str(device))
+        loop = DecodeLoop(rows=ROWS, device=str(device), pack_fn=PACK_FN)
         g = capture(lambda i: loop.run(), 1)
         for _ in range(3):
             g.replay()
@@ -479,7 +489,11 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rows sweep and the decode-loop step")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--unpacked-fn", action="store_true",
+                    help="pass fp32 fn (split into bf16 terms in every call) instead of the packed form")
     args = ap.parse_args()
+    global PACK_FN
+    PACK_FN = not args.unpacked_fn
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -86,7 +86,11 @@ typedef enum {
  *   pre  = sigmoid(l_pre) + pre_eps;     post = post_alpha * sigmoid(l_post)
  *   comb = Sinkhorn(l_comb, sinkhorn_iters, sinkhorn_eps):
  *          M = exp(L - max L); repeat: rows /= (row sum + eps), then columns /= (column sum + eps).
- * Constraints: eps values >= 0, 0 <= sinkhorn_iters <= 1000. */
+ *   fn_packed  optional: fn as mhc_projection_pack wrote it. When set, the
+ *         boundary reads it instead of fn (fn may then be NULL) and gives
+ *         bitwise the same results; it spares the kernel the split of fn into
+ *         bf16 terms at every call, at 1.55x the bytes of fn for n = 4.
+ * Constraints: fn or fn_packed set, eps values >= 0, 0 <= sinkhorn_iters <= 1000. */
 typedef struct {
   const float* fn;
   const float* scale;
@@ -96,6 +100,7 @@ typedef struct {
   float sinkhorn_eps;
   float post_alpha;
   int sinkhorn_iters;
+  const void* fn_packed;
 } mhc_coeff_args;
 
 /* MXFP8 layer input ([boundary] empty_quantized_layer_input: E4M3 data [R, H] and
@@ -131,6 +136,21 @@ MHC_API size_t mhc_mxfp8_scale_bytes(int rows, int hidden, int swizzled_128x4);
 
 /* Zero the workspace on `stream` (cudaMemsetAsync). Needed once before first use. */
 MHC_API mhc_status mhc_workspace_init(void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* fn [n*H, C] fp32 rewritten once, at weight-load time, into the form the
+ * projection's tensor-core tiles read (no counterpart in the method: a layout
+ * of the same weights). Each value f becomes three bf16 terms hi + mid + lo
+ * equal to f to 2^-24 (hi = bf16(f), mid = bf16(f - hi), lo = bf16(f - hi - mid)),
+ * grouped per 64-column block of H as [3][CP8][n*64 + 8] with CP8 = C rounded
+ * up to 8 and zeros in the padding. The layout is private to this library
+ * version: pass the result only as mhc_coeff_args.fn_packed.
+ *   mhc_projection_pack_bytes: H/64 * 3 * CP8 * (n*64 + 8) * 2 bytes, 0 for an
+ *     unsupported (hidden, hc_mult).
+ *   mhc_projection_pack: fn 4-byte aligned, packed 16-byte aligned and
+ *     mhc_projection_pack_bytes long; asynchronous on stream, an ordinary
+ *     launch (a boundary launched after it on the stream sees the result). */
+MHC_API size_t mhc_projection_pack_bytes(int hidden, int hc_mult);
+MHC_API mhc_status mhc_projection_pack(const float* fn, void* packed, int hidden, int hc_mult, mhc_stream stream);
 
 /* Full boundary after a sublayer with TP-partial output ([all_reduce]
  * BoundaryAllReduce.__call__, [boundary] Boundaries.sublayer / _reduce):

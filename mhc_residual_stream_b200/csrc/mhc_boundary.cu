@@ -2,10 +2,10 @@
 // libmhc.so (declared in include/mhc.h).
 //
 // A boundary is two launches chained by programmatic dependent launch (PDL).
-// Block g of both owns columns [64g, 64g+64) of H for every row, so each
-// weight of fn is read from HBM exactly once.
-// The streaming kernel (boundary_kernel):
-//   1. TMA bulk copies bring the block's fn slice into shared memory and the
+// The streaming kernel (boundary_kernel): block g owns columns [64g, 64g+64)
+// of H for every row, so each weight of fn is read from HBM exactly once.
+//   1. A TMA bulk copy brings the block's fn slice into shared memory (packed
+//      bf16 terms, or fp32 that the block splits into bf16 terms) and the
 //      block's activations are prefetched into L2, both before the kernel waits
 //      for its predecessor on the stream;
 //   2. per (row, 8 columns) a lane sums the partials (or finalizes the MoE
@@ -13,13 +13,13 @@
 //      Boundaries.post_only: mhc_post(x, residual, post, comb)), rounds the new
 //      streams to bf16, stores them, sums the squares of their collapse with the
 //      carried pre (BoundaryState.pre) and of the streams;
-//   3. the block projects its rows' n*64 stream values onto the C fn columns
-//      with register-tiled CUDA-core FMA (8 rows x C/4 columns per thread) and
-//      writes its partial sums to the workspace.
+//   3. the block projects its rows' n*64 stream values onto the C fn columns on
+//      the tensor cores (mma.sync bf16, fn as three bf16 terms) and writes its
+//      partial sums to the workspace.
 // The tail kernel (boundary_tail_kernel), once the streaming kernel is done:
-//   4. blocks 0..G-1 normalise their columns into the layer input (and MXFP8);
-//      at the same time further blocks finish the coefficients (logits, sigmoid,
-//      Sinkhorn in one thread) of rows j, j + Gc, ...
+//   4. layer-input blocks normalise 256-column tasks of the rows into the layer
+//      input (and MXFP8); beside them, coefficient blocks finish the rows'
+//      coefficients (logits, sigmoid, Sinkhorn with one matrix entry per lane).
 // The residual-only variant is the streaming kernel alone. All reductions run
 // in a fixed order, so results are bitwise reproducible.
 
@@ -41,7 +41,7 @@ constexpr int kMaxRows = 128;
 constexpr int kMaxPartials = 16;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxIters = 1000;
-constexpr int kMaxBlocks = 148;  // H/64 blocks, all resident at once (one per SM)
+constexpr int kMaxBlocks = 148;  // most H/64 blocks: the tail's per-lane loads are sized for it
 // Workspace header: the status word (byte 0); the partial sums follow.
 constexpr size_t kWsHeader = 1024;
 constexpr int kStatusWord = 0;
@@ -81,6 +81,7 @@ struct Params {
   const __nv_bfloat16* norm_weight;
   float norm_eps;
   const float* fn;
+  const __nv_bfloat16* fn_packed;  // [G][3][CP8][n*64 + 8] bf16 terms of fn, or null
   const float* scale;
   const float* base;
   float rms_eps, pre_eps, sk_eps, alpha;
@@ -103,7 +104,7 @@ struct Params {
   // embedding of the first layer (whose identity pre-mix selects it)
   const __nv_bfloat16* tail_streams;
   int tail_broadcast;
-  int tail_layer_blocks;  // tail blocks [0, this) write the layer input (G or 0)
+  int tail_layer_blocks;  // tail blocks [0, this) write the layer input (at most G, or 0)
   int tail_coeff_blocks;  // the next ones finish the coefficients of rows j, j + this, ...
   int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
   int64_t budget_ns;
@@ -146,23 +147,18 @@ __host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe) {
 
 // Shared memory of the tail kernel.
 struct TailLayout {
-  int inv_off, pre_off, part_off, cst_off, total;
+  int part_off, cst_off, total;
 };
 
 template <int N>
-__host__ __device__ inline TailLayout tail_layout(int R) {
+__host__ __device__ inline TailLayout tail_layout() {
   constexpr int CP = cpad_of(N);
   TailLayout L{};
   int o = 0;
-  L.inv_off = o;
-  o += kMaxRows * 4;
-  L.pre_off = o;
-  o += R * N * 4;
-  o = (o + 15) & ~15;
-  L.part_off = o;  // [warps][8] float4
-  o += kWarps * 8 * 16;
-  L.cst_off = o;  // norm weight [64] bf16, scale[4], base[CP]
-  o += kCols * 2 + (4 + CP) * 4;
+  L.part_off = o;  // [kWarps rows][kWarps][RED] floats: the warps' shares of a row's records
+  o += kWarps * kWarps * red_of(N) * 4;
+  L.cst_off = o;  // scale[4], base[CP]
+  o += (4 + CP) * 4;
   L.total = (o + 15) & ~15;
   return L;
 }
@@ -260,6 +256,22 @@ __device__ __forceinline__ void load_quad(const Params& p, int r, int h0, const 
   }
 }
 
+// fn as three bf16 terms, f = hi + mid + lo to 2^-24: each bf16 x bf16 product is
+// exact in fp32, so three tensor-core products return the fp32 projection up to
+// the order of the fp32 additions.
+__device__ __forceinline__ void split3(float f, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(f);
+  const float r1 = f - __bfloat162float(hi);
+  mid = __float2bfloat16_rn(r1);
+  lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+}
+
+// Bytes of a block's packed fn slice: the B operand of the projection exactly as
+// it sits in shared memory, [3][CP8][n*64 + 8] bf16.
+__host__ __device__ constexpr int packed_slice_bytes(int n) { return 3 * ntiles_of(n) * 8 * kstride_of(n) * 2; }
+static_assert(packed_slice_bytes(1) % 16 == 0 && packed_slice_bytes(2) % 16 == 0 && packed_slice_bytes(4) % 16 == 0,
+              "a bulk copy moves a multiple of 16 bytes");
+
 template <int N, int FRONT>
 __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   constexpr int C = logits_of(N);
@@ -295,10 +307,17 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   // ---- 1. the block's fn slice by TMA bulk copies. Weights are never written by
   // the kernel that precedes this one on the stream, so this runs before the
   // wait on that kernel (programmatic dependent launch).
+  const bool packed = p.fn_packed != nullptr;
   if (p.do_coeff) {
     if (tid == 0) mbar_init(bar, 1);
     __syncthreads();
-    if (warp == 0) {
+    if (packed) {  // pre-split terms (mhc_projection_pack): one copy, waited for at step 5
+      if (tid == 0) {
+        constexpr int PB = packed_slice_bytes(N);
+        mbar_arrive_expect_tx(bar, PB + 16 * p.extra_tx);
+        bulk_g2s(bs_s, reinterpret_cast<const unsigned char*>(p.fn_packed) + static_cast<size_t>(g) * PB, PB, bar);
+      }
+    } else if (warp == 0) {
       if (lane == 0) mbar_arrive_expect_tx(bar, KC * C * 4 + 16 * p.extra_tx);
       __syncwarp();
       for (int m = lane; m < N * 8; m += 32) {
@@ -333,21 +352,17 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
     }
   }
 
-  if (p.do_coeff) {
-    // Split the fn slice into three bf16 terms, f = hi + mid + lo to 2^-24,
-    // stored column-major for the MMA's B operand (weights only: before the wait).
-    // Each bf16 x bf16 product is exact in fp32, so the tensor cores return the
-    // fp32 projection up to the order of the fp32 additions.
+  if (p.do_coeff && !packed) {
+    // Split the fn slice into three bf16 terms (split3), stored column-major for
+    // the MMA's B operand (weights only: before the wait).
     const bool ok = mbar_wait_bounded(bar, 0, deadline);
     if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
     if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
     for (int e = tid; e < CP8 * KC; e += kThreads) {
       const int c = e / KC, k = e - c * KC;
       const float f = c < C ? reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4)[c] : 0.f;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(f);
-      const float r1 = f - __bfloat162float(hi);
-      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+      __nv_bfloat16 hi, mid, lo;
+      split3(f, hi, mid, lo);
       bs_s[(0 * CP8 + c) * KS + k] = hi;
       bs_s[(1 * CP8 + c) * KS + k] = mid;
       bs_s[(2 * CP8 + c) * KS + k] = lo;
@@ -529,7 +544,13 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   // terms, fp32 accumulation (mma.sync m16n8k16). Warp w takes the k-steps
   // w, w+8, ... of every 16-row tile and 8-column tile of a 32-row chunk; the
   // warps' sums are added in warp order.
-  __syncthreads();  // staged streams
+  if (packed) {  // the packed slice, copied before the wait, has surely landed by now
+    const bool ok = mbar_wait_bounded(bar, 0, deadline);
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (__syncthreads_or(!ok)) return;  // also the barrier for the staged streams
+  } else {
+    __syncthreads();  // staged streams
+  }
   for (int rb = 0; rb < R; rb += 32) {
     float acc[2][NT][4];
 #pragma unroll
@@ -583,8 +604,12 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
 
 // Sinkhorn normalisation of an n x n matrix in one thread's registers: `iters`
 // times, each row divided by (its sum + eps), then each column by (its sum +
-// eps). For n >= 2 rows are held as pairs and summed / scaled with packed
-// f32x2 arithmetic, which halves the instructions on the serial chain.
+// eps). For n = 4, eps rides in copies of column 0 (row sums) and row 0 (column
+// sums) made by a fused multiply-add from the previous step's scaling, instead
+// of an add on the dependency chain. Measured on this part, scalar code beats
+// packed f32x2 pairs, and neither sharing the matrix between lanes (a shuffle
+// costs about 27 cycles) nor taking a step's four reciprocals from one (batch
+// inversion) is faster.
 template <int N>
 __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, float eps) {
   if constexpr (N == 1) {
@@ -592,68 +617,100 @@ __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, fl
       M[0][0] *= rcp_approx(M[0][0] + eps);
       M[0][0] *= rcp_approx(M[0][0] + eps);
     }
-  } else {
-    constexpr int H2 = N / 2;
-    float2 P[N][H2];
-#pragma unroll
-    for (int j = 0; j < N; ++j)
-#pragma unroll
-      for (int h = 0; h < H2; ++h) P[j][h] = make_float2(M[j][2 * h], M[j][2 * h + 1]);
+  } else if constexpr (N == 2) {
+    float2 P[2] = {make_float2(M[0][0], M[0][1]), make_float2(M[1][0], M[1][1])};
     const float2 e2 = make_float2(eps, eps);
     for (int it = 0; it < iters; ++it) {
 #pragma unroll
-      for (int j = 0; j < N; ++j) {  // rows
-        float2 s2 = P[j][0];
-#pragma unroll
-        for (int h = 1; h < H2; ++h) s2 = __fadd2_rn(s2, P[j][h]);
-        const float rr = rcp_approx(s2.x + s2.y + eps);
-        const float2 r2 = make_float2(rr, rr);
-#pragma unroll
-        for (int h = 0; h < H2; ++h) P[j][h] = __fmul2_rn(P[j][h], r2);
+      for (int j = 0; j < 2; ++j) {
+        const float rr = rcp_approx(P[j].x + P[j].y + eps);
+        P[j] = __fmul2_rn(P[j], make_float2(rr, rr));
       }
-#pragma unroll
-      for (int h = 0; h < H2; ++h) {  // columns 2h, 2h+1
-        float2 c2;
-        if constexpr (N == 4) {
-          c2 = __fadd2_rn(__fadd2_rn(P[0][h], P[1][h]), __fadd2_rn(P[2][h], P[3][h]));
-        } else {
-          c2 = P[0][h];
-#pragma unroll
-          for (int j = 1; j < N; ++j) c2 = __fadd2_rn(c2, P[j][h]);
-        }
-        c2 = __fadd2_rn(c2, e2);
-        const float2 r2 = make_float2(rcp_approx(c2.x), rcp_approx(c2.y));
-#pragma unroll
-        for (int j = 0; j < N; ++j) P[j][h] = __fmul2_rn(P[j][h], r2);
-      }
+      const float2 c2 = __fadd2_rn(__fadd2_rn(P[0], P[1]), e2);
+      const float2 r2 = make_float2(rcp_approx(c2.x), rcp_approx(c2.y));
+      P[0] = __fmul2_rn(P[0], r2);
+      P[1] = __fmul2_rn(P[1], r2);
     }
 #pragma unroll
-    for (int j = 0; j < N; ++j)
+    for (int j = 0; j < 2; ++j) {
+      M[j][0] = P[j].x;
+      M[j][1] = P[j].y;
+    }
+  } else {
+    static_assert(N == 4, "hc_mult 1, 2 or 4");
+    float e0[4];  // column 0 plus eps: the row sums' eps
 #pragma unroll
-      for (int h = 0; h < H2; ++h) {
-        M[j][2 * h] = P[j][h].x;
-        M[j][2 * h + 1] = P[j][h].y;
-      }
+    for (int j = 0; j < 4; ++j) e0[j] = M[j][0] + eps;
+    for (int it = 0; it < iters; ++it) {
+      float r[4], c0[4], c[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) r[j] = rcp_approx((e0[j] + M[j][1]) + (M[j][2] + M[j][3]));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c0[i] = fmaf(M[0][i], r[0], eps);  // row 0 plus eps: the column sums' eps
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) M[j][i] *= r[j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[i] = rcp_approx((c0[i] + M[1][i]) + (M[2][i] + M[3][i]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) e0[j] = fmaf(M[j][0], c[0], eps);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) M[j][i] *= c[i];
+    }
+  }
+}
+
+// Loads of one layer-input task of a lane (row r, 8 columns): the row's
+// per-block sums of c^2, its carried pre, the stream vectors and norm weights.
+template <int N>
+struct LayerLoads {
+  static constexpr int MAXM = (kMaxBlocks + 31) / 32;
+  float sq[MAXM];
+  float pr[N];
+  uint4 sv[N];
+  uint4 nw;
+};
+
+template <int N>
+__device__ __forceinline__ void layer_load(const Params& p, int r, int g, int lane, bool weights,
+                                           LayerLoads<N>& Q) {
+  const int G = p.H / kCols;
+#pragma unroll
+  for (int m = 0; m < LayerLoads<N>::MAXM; ++m) {
+    const int k = lane + 32 * m;
+    Q.sq[m] = k < G ? __ldcg(p.sc2_part + r * G + k) : 0.f;
+  }
+  if (g >= G) return;
+  const int h0 = g * kCols + (lane & 7) * 8;
+  if (weights) Q.nw = ld_nc_v4(p.norm_weight + h0);
+  if (p.tail_broadcast) {
+    Q.sv[0] = ld_v4(p.tail_streams + static_cast<size_t>(r) * p.H + h0);
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      Q.pr[j] = p.pre[r * N + j];
+      Q.sv[j] = ld_v4(p.tail_streams + (static_cast<size_t>(r) * N + j) * p.H + h0);
+    }
   }
 }
 
 // The tail of a boundary, launched after the streaming kernel (programmatic
-// dependent launch). Once every block's partial sums are in the workspace,
-// layer-input block g normalises columns [64g, 64g+64) of every row into the
-// layer input (and MXFP8), recomputing the collapse from the bf16 streams
-// (L2-resident), while coefficient block j finishes rows j, j + Gc, ...
+// dependent launch). Layer-input blocks split the rows into tasks of 256
+// columns (4 units of 64), one task per warp at a time: a lane normalises 8
+// columns of the row into the layer input (and MXFP8), recomputing the
+// collapse from the bf16 streams, after summing the row's per-block c^2 itself.
+// Coefficient blocks finish rows j, j + Gc, ... (logits, sigmoid, Sinkhorn).
 template <int N>
 __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params p) {
   constexpr int C = logits_of(N);
-  constexpr int CP = cpad_of(N);
   constexpr int RED = red_of(N);
   extern __shared__ __align__(128) unsigned char smem[];
-  const TailLayout L = tail_layout<N>(p.R);
-  float* inv_s = reinterpret_cast<float*>(smem + L.inv_off);
-  float* pre_s = reinterpret_cast<float*>(smem + L.pre_off);
-  float* red_s = reinterpret_cast<float*>(smem + L.part_off);
-  __nv_bfloat16* nw_s = reinterpret_cast<__nv_bfloat16*>(smem + L.cst_off);
-  float* scale_s = reinterpret_cast<float*>(smem + L.cst_off + kCols * 2);
+  const TailLayout L = tail_layout<N>();
+  float* slot_s = reinterpret_cast<float*>(smem + L.part_off);  // [kWarps rows][kWarps][RED]
+  float* scale_s = reinterpret_cast<float*>(smem + L.cst_off);
   float* base_s = scale_s + 4;
 
   const int G = p.H / kCols;
@@ -661,195 +718,187 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
   const int R = p.R;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rq = lane >> 3, vec = lane & 7;
-  const int nquads = (R + 3) >> 2;
-  const bool layer_role = static_cast<int>(blockIdx.x) < p.tail_layer_blocks;
 
-  if (layer_role) {
-    const int g = blockIdx.x;
-    const int h0 = g * kCols + vec * 8;
-    if (tid < 8) cp_async16(nw_s + tid * 8, p.norm_weight + g * kCols + tid * 8);  // weights: before the wait
+  if (static_cast<int>(blockIdx.x) < p.tail_layer_blocks) {
+    const int GT = (G + 3) >> 2;  // tasks per row
+    const int T = R * GT;
+    const int W = p.tail_layer_blocks * kWarps;
+    const int w0 = blockIdx.x * kWarps + warp;
+    LayerLoads<N> cur;
+    if (w0 < T) {  // norm weights of the first task: weights, so before the wait
+      const int g = (w0 % GT) * 4 + rq;
+      if (g < G) cur.nw = ld_nc_v4(p.norm_weight + g * kCols + vec * 8);
+    }
     griddep_wait();
     griddep_launch_dependents();
-    if (!p.tail_broadcast)
-      for (int k = tid; k < R * N; k += kThreads) cp_async4(pre_s + k, p.pre + k);
-    // the blocks' sums of c^2 of rows warp + 8j (j < 4) for the first 32 rows
-    constexpr int MAXM = (kMaxBlocks + 31) / 32;
-    float sq[4][MAXM];
+    if (w0 < T) layer_load<N>(p, w0 / GT, (w0 % GT) * 4 + rq, lane, false, cur);
+    const int scols = H / 32;
+    const int col_tiles = (scols + 3) / 4;
+    for (int t = w0; t < T; t += W) {
+      LayerLoads<N> nxt;
+      if (t + W < T) layer_load<N>(p, (t + W) / GT, ((t + W) % GT) * 4 + rq, lane, true, nxt);
+      const int r = t / GT;
+      const int g = (t - r * GT) * 4 + rq;
+      // ---- 7. the row's inverse RMS of the collapse: block sums in a fixed order
+      float a = cur.sq[0];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = warp + j * kWarps;
-#pragma unroll
-      for (int m = 0; m < MAXM; ++m) {
-        const int k = lane + 32 * m;
-        sq[j][m] = (r < R && k < G) ? __ldcg(p.sc2_part + r * G + k) : 0.f;
-      }
-    }
-    // this lane's stream vectors of every quad it normalises (at most 4 per warp)
-    uint4 sv[4][N];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int r = (warp + m * kWarps) * 4 + rq;
-      if (r < R) {
+      for (int m = 1; m < LayerLoads<N>::MAXM; ++m) a += cur.sq[m];
+      a = warp_sum(a);
+      const float inv = rsqrtf(__fdiv_rn(a, static_cast<float>(H)) + p.norm_eps);
+      if (g < G) {  // the 8 lanes of a unit share g: whole MXFP8 groups
+        const int h0 = g * kCols + vec * 8;
+        // ---- 7b. layer input: the collapse recomputed from the bf16 streams exactly
+        // as the streaming kernel summed its squares
+        float c[8];
         if (p.tail_broadcast) {
-          sv[m][0] = ld_v4(p.tail_streams + static_cast<size_t>(r) * H + h0);
+          unpack8(cur.sv[0], c);
         } else {
+          float nf[N][8];
 #pragma unroll
-          for (int j = 0; j < N; ++j) sv[m][j] = ld_v4(p.tail_streams + (static_cast<size_t>(r) * N + j) * H + h0);
+          for (int j = 0; j < N; ++j) unpack8(cur.sv[j], nf[j]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < N; ++j) s = fmaf(cur.pr[j], nf[j][e], s);
+            c[e] = s;
+          }
         }
-      }
-    }
-    cp_async_wait_all();
-    // ---- 7. per-row inverse RMS of the collapse: block sums added in a fixed order.
-    // Rows r0 + 8j, j < 4, reduced together: two halving steps leave row
-    // 2*(lane bit 4) + (lane bit 3) in each lane, three more steps sum it.
-    for (int r0 = warp; r0 < R; r0 += 4 * kWarps) {
-      if (r0 != warp) {
+        float w[8], y[8], yr[8];
+        unpack8(cur.nw, w);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = r0 + j * kWarps;
+        for (int e = 0; e < 8; ++e) y[e] = c[e] * inv * w[e];
+        const uint4 yb = round8(y, yr);
+        st_v4(p.layer_input + static_cast<size_t>(r) * H + h0, yb);
+        if (p.q_data != nullptr) {
+          float amax = 0.f;
+          bool finite = true;
 #pragma unroll
-          for (int m = 0; m < MAXM; ++m) {
-            const int k = lane + 32 * m;
-            sq[j][m] = (r < R && k < G) ? __ldcg(p.sc2_part + r * G + k) : 0.f;
+          for (int e = 0; e < 8; ++e) {
+            amax = fmaxf(amax, fabsf(yr[e]));
+            finite = finite && isfinite(yr[e]);
+          }
+          // the 4 lanes of a 32-column block are vec 0-3 or 4-7 of the same unit
+          const unsigned grp_mask = 0xffu << (lane & 24);
+          amax = fmaxf(amax, __shfl_xor_sync(grp_mask, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(grp_mask, amax, 2));
+          const unsigned fin_mask = __ballot_sync(grp_mask, finite);
+          const unsigned grp = (fin_mask >> (lane & 28)) & 0xfu;
+          uint2 d;
+          unsigned char sbyte;
+          if (grp == 0xfu) {
+            const int e = e8m0_exponent(amax);
+            const float sc = exp2_neg(e);
+            d.x = static_cast<unsigned>(e4m3x2(yr[0] * sc, yr[1] * sc)) |
+                  (static_cast<unsigned>(e4m3x2(yr[2] * sc, yr[3] * sc)) << 16);
+            d.y = static_cast<unsigned>(e4m3x2(yr[4] * sc, yr[5] * sc)) |
+                  (static_cast<unsigned>(e4m3x2(yr[6] * sc, yr[7] * sc)) << 16);
+            sbyte = static_cast<unsigned char>(e + 127);
+          } else {
+            d.x = d.y = 0x7f7f7f7fu;
+            sbyte = 0xff;
+          }
+          *reinterpret_cast<uint2*>(p.q_data + static_cast<size_t>(r) * H + h0) = d;
+          if ((vec & 3) == 0) {
+            const int sc = h0 / 32;
+            const int off = p.q_swizzled ? swizzled_scale_offset(r, sc, col_tiles) : r * scols + sc;
+            p.q_scale[off] = sbyte;
           }
         }
       }
-      float a[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        a[j] = 0.f;
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) a[j] += sq[j][m];
-      }
-      const bool hi4 = (lane & 16) != 0, hi3 = (lane & 8) != 0;
-      float b0 = (hi4 ? a[2] : a[0]) + __shfl_xor_sync(kFull, hi4 ? a[0] : a[2], 16);
-      float b1 = (hi4 ? a[3] : a[1]) + __shfl_xor_sync(kFull, hi4 ? a[1] : a[3], 16);
-      float c = (hi3 ? b1 : b0) + __shfl_xor_sync(kFull, hi3 ? b0 : b1, 8);
-#pragma unroll
-      for (int mm = 4; mm >= 1; mm >>= 1) c += __shfl_xor_sync(kFull, c, mm);
-      const int r = r0 + (2 * (hi4 ? 1 : 0) + (hi3 ? 1 : 0)) * kWarps;
-      if ((lane & 7) == 0 && r < R) inv_s[r] = rsqrtf(__fdiv_rn(c, static_cast<float>(H)) + p.norm_eps);
-    }
-    __syncthreads();
-    // ---- 7b. layer input (and MXFP8) of this block's columns: the collapse is
-    // recomputed from the bf16 streams exactly as the streaming kernel summed c^2
-    float w[8];
-    unpack8(*reinterpret_cast<const uint4*>(nw_s + vec * 8), w);
-    const int scols = H / 32;
-    const int col_tiles = (scols + 3) / 4;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int q = warp + m * kWarps;
-      const int r = q * 4 + rq;
-      if (q >= nquads || r >= R) continue;  // whole 4-lane MXFP8 groups share r
-      float c[8];
-      if (p.tail_broadcast) {
-        unpack8(sv[m][0], c);
-      } else {
-        float nf[N][8];
-#pragma unroll
-        for (int j = 0; j < N; ++j) unpack8(sv[m][j], nf[j]);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          float s = 0.f;
-#pragma unroll
-          for (int j = 0; j < N; ++j) s = fmaf(pre_s[r * N + j], nf[j][t], s);
-          c[t] = s;
-        }
-      }
-      const float inv = inv_s[r];
-      float y[8], yr[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) y[t] = c[t] * inv * w[t];
-      const uint4 yb = round8(y, yr);
-      st_v4(p.layer_input + static_cast<size_t>(r) * H + h0, yb);
-      if (p.q_data != nullptr) {
-        float amax = 0.f;
-        bool finite = true;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          amax = fmaxf(amax, fabsf(yr[t]));
-          finite = finite && isfinite(yr[t]);
-        }
-        // the 4 lanes of a 32-column block are vec 0-3 or 4-7 of the same row
-        amax = fmaxf(amax, __shfl_xor_sync(0xffu << (lane & 24), amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffu << (lane & 24), amax, 2));
-        const unsigned fin_mask = __ballot_sync(0xffu << (lane & 24), finite);
-        const unsigned grp = (fin_mask >> (lane & 28)) & 0xfu;
-        uint2 d;
-        unsigned char sbyte;
-        if (grp == 0xfu) {
-          const int e = e8m0_exponent(amax);
-          const float sc = exp2_neg(e);
-          d.x = static_cast<unsigned>(e4m3x2(yr[0] * sc, yr[1] * sc)) |
-                (static_cast<unsigned>(e4m3x2(yr[2] * sc, yr[3] * sc)) << 16);
-          d.y = static_cast<unsigned>(e4m3x2(yr[4] * sc, yr[5] * sc)) |
-                (static_cast<unsigned>(e4m3x2(yr[6] * sc, yr[7] * sc)) << 16);
-          sbyte = static_cast<unsigned char>(e + 127);
-        } else {
-          d.x = d.y = 0x7f7f7f7fu;
-          sbyte = 0xff;
-        }
-        *reinterpret_cast<uint2*>(p.q_data + static_cast<size_t>(r) * H + h0) = d;
-        if ((vec & 3) == 0) {
-          const int sc = h0 / 32;
-          const int off = p.q_swizzled ? swizzled_scale_offset(r, sc, col_tiles) : r * scols + sc;
-          p.q_scale[off] = sbyte;
-        }
-      }
+      cur = nxt;
     }
     if (p.q_data != nullptr && p.q_swizzled) {
-      // zero the padding of the swizzled scale buffer: rows R.. of this block's two
-      // scale columns, and (last block) the padding columns of every row
+      // zero the padding of the swizzled scale buffer: rows R.. whole (4-byte words
+      // of a tile row when the buffer is 4-byte aligned), then the padding columns
+      // of rows below R
       const int rows_p = (R + 127) & ~127;
-      const int sc0 = g * 2;
-      for (int k = tid; k < (rows_p - R) * 2; k += kThreads) {
-        const int r = R + (k >> 1), sc = sc0 + (k & 1);
-        p.q_scale[swizzled_scale_offset(r, sc, col_tiles)] = 0;
-      }
-      if (g == G - 1) {
-        const int pad_cols = col_tiles * 4 - scols;
-        for (int k = tid; k < rows_p * pad_cols; k += kThreads) {
-          const int r = k / pad_cols, sc = scols + (k - r * pad_cols);
+      const int pad_cols = col_tiles * 4 - scols;
+      const bool words = (reinterpret_cast<uintptr_t>(p.q_scale) & 3) == 0;
+      const int per_row = words ? col_tiles : col_tiles * 4;
+      const int n_rows = (rows_p - R) * per_row;
+      const int n_cols = R * pad_cols;
+      for (int k = w0 * 32 + lane; k < n_rows + n_cols; k += W * 32) {
+        if (k < n_rows) {
+          const int r = R + k / per_row, u = k % per_row;
+          if (words)
+            *reinterpret_cast<uint32_t*>(p.q_scale + swizzled_scale_offset(r, u * 4, col_tiles)) = 0u;
+          else
+            p.q_scale[swizzled_scale_offset(r, u, col_tiles)] = 0;
+        } else {
+          const int kk = k - n_rows;
+          const int r = kk / pad_cols, sc = scols + kk % pad_cols;
           p.q_scale[swizzled_scale_offset(r, sc, col_tiles)] = 0;
         }
       }
     }
   } else {
-    // coefficient rows j, j + tail_coeff_blocks, ...: sum the blocks' partials in a
-    // fixed order, logits, sigmoid, Sinkhorn
+    // Coefficient rows jb, jb + CB, ...: in batches of up to kWarps rows, every
+    // warp adds a share of each row's per-block records (fixed order) into a
+    // slot, then warp s finishes row s of the batch: logits, sigmoid, Sinkhorn.
     const int jb = blockIdx.x - p.tail_layer_blocks;
+    const int CB = p.tail_coeff_blocks;
     if (tid < 3) cp_async4(scale_s + tid, p.scale + tid);  // weights: before the wait
     if (tid >= 32 && tid < 32 + C) cp_async4(base_s + tid - 32, p.base + (tid - 32));
     griddep_wait();
     griddep_launch_dependents();
     constexpr int V4 = RED / 4;
-    constexpr int GPT = kThreads / V4;                  // record groups per pass
-    constexpr int MAXK = (kMaxBlocks + GPT - 1) / GPT;  // passes for G <= 148
+    constexpr int MAXK = (kMaxBlocks * V4 + kThreads - 1) / kThreads;
+    constexpr int NN = N * N;
+    const int F = G * V4;
+    const int rho = (R - jb + CB - 1) / CB;
     cp_async_wait_all();
-    __syncthreads();
-    float4* part4 = reinterpret_cast<float4*>(red_s);  // [kWarps][V4]
-    for (int r = jb; r < R; r += p.tail_coeff_blocks) {
-      float4 cacc = sum_row_partials<RED, MAXK>(p.dot_part, r, G, tid);
-      // sum the record groups of a warp (lane bits above log2(V4)), then the warps
+    for (int k0 = 0; k0 < rho; k0 += kWarps) {
+      const int nk = rho - k0 < kWarps ? rho - k0 : kWarps;
+      float4 v[MAXK];
+      {
+        const float4* base = reinterpret_cast<const float4*>(p.dot_part + static_cast<size_t>(jb + k0 * CB) * G * RED);
 #pragma unroll
-      for (int m = V4; m < 32; m <<= 1) {
-        cacc.x += __shfl_xor_sync(kFull, cacc.x, m);
-        cacc.y += __shfl_xor_sync(kFull, cacc.y, m);
-        cacc.z += __shfl_xor_sync(kFull, cacc.z, m);
-        cacc.w += __shfl_xor_sync(kFull, cacc.w, m);
+        for (int k = 0; k < MAXK; ++k) {
+          const int f = tid + k * kThreads;
+          v[k] = f < F ? __ldcg(base + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      for (int s = 0; s < nk; ++s) {
+        float4 nx[MAXK];
+        if (s + 1 < nk) {  // the next row's loads go out before this row is added up
+          const float4* base =
+              reinterpret_cast<const float4*>(p.dot_part + static_cast<size_t>(jb + (k0 + s + 1) * CB) * G * RED);
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int f = tid + k * kThreads;
+            nx[k] = f < F ? __ldcg(base + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float4 a = v[0];
+#pragma unroll
+        for (int k = 1; k < MAXK; ++k) {
+          a.x += v[k].x;
+          a.y += v[k].y;
+          a.z += v[k].z;
+          a.w += v[k].w;
+        }
+        // lanes sharing lane % V4 hold the same 4 record values: add them up
+#pragma unroll
+        for (int m = V4; m < 32; m <<= 1) {
+          a.x += __shfl_xor_sync(kFull, a.x, m);
+          a.y += __shfl_xor_sync(kFull, a.y, m);
+          a.z += __shfl_xor_sync(kFull, a.z, m);
+          a.w += __shfl_xor_sync(kFull, a.w, m);
+        }
+        if (lane < V4) reinterpret_cast<float4*>(slot_s + (s * kWarps + warp) * RED)[lane] = a;
+        if (s + 1 < nk) {
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) v[k] = nx[k];
+        }
       }
       __syncthreads();
-      if (lane < V4) part4[warp * V4 + lane] = cacc;
-      __syncthreads();
-      if (warp == 0) {
-        float s = 0.f;  // lane v: value v of the record
+      if (warp < nk) {
+        const int r = jb + (k0 + warp) * CB;
+        float s = 0.f;  // lane c: record value c, the warps' shares added in order
         if (lane < RED) {
 #pragma unroll
-          for (int w = 0; w < kWarps; ++w) {
-            const float4 a = part4[w * V4 + lane / 4];
-            s += (lane & 3) == 0 ? a.x : ((lane & 3) == 1 ? a.y : ((lane & 3) == 2 ? a.z : a.w));
-          }
+          for (int w = 0; w < kWarps; ++w) s += slot_s[(warp * kWarps + w) * RED + lane];
         }
         const float inv = rsqrtf(__fdiv_rn(__shfl_sync(kFull, s, C), static_cast<float>(N * H)) + p.rms_eps);
         const int grp = lane < N ? 0 : (lane < 2 * N ? 1 : 2);
@@ -860,19 +909,22 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
           p.post_out[r * N + (lane - N)] = p.alpha / (1.f + expf(-l));
         }
         // Sinkhorn in one thread: M = exp(L - max L); rows then columns, iters times
-        constexpr int NN = N * N;
         float lc[NN];
 #pragma unroll
         for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, l, 2 * N + k);
         if (lane == 0) {
-          float mx = lc[0];
+          float t[NN];
 #pragma unroll
-          for (int k = 1; k < NN; ++k) mx = fmaxf(mx, lc[k]);
+          for (int k = 0; k < NN; ++k) t[k] = lc[k];
+#pragma unroll
+          for (int w = NN / 2; w >= 1; w >>= 1)
+#pragma unroll
+            for (int k = 0; k < w; ++k) t[k] = fmaxf(t[k], t[k + w]);
           float M[N][N];
 #pragma unroll
           for (int j = 0; j < N; ++j)
 #pragma unroll
-            for (int i = 0; i < N; ++i) M[j][i] = expf(lc[j * N + i] - mx);
+            for (int i = 0; i < N; ++i) M[j][i] = expf(lc[j * N + i] - t[0]);
           sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
 #pragma unroll
           for (int j = 0; j < N; ++j)
@@ -880,10 +932,34 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
             for (int i = 0; i < N; ++i) p.comb_out[r * NN + j * N + i] = M[j][i];
         }
       }
+      __syncthreads();  // the slots are refilled by the next batch
     }
   }
 }
 
+
+// fn [n*H, C] fp32 -> per block g the B operand of its projection as three bf16
+// terms, [G][3][CP8][n*64 + 8]: entry (t, c, k) is term t of fn[(k/64)*H + 64g + k%64][c];
+// columns c >= C and the 8-entry gap after each column are zero.
+template <int N>
+__global__ void __launch_bounds__(256) pack_projection_kernel(const float* __restrict__ fn, int H,
+                                                              __nv_bfloat16* __restrict__ out) {
+  constexpr int C = logits_of(N);
+  constexpr int KS = kstride_of(N);
+  constexpr int CP8 = ntiles_of(N) * 8;
+  const int g = blockIdx.x;
+  __nv_bfloat16* dst = out + static_cast<size_t>(g) * (packed_slice_bytes(N) / 2);
+  for (int e = threadIdx.x; e < CP8 * KS; e += blockDim.x) {
+    const int c = e / KS, k = e - c * KS;
+    float f = 0.f;
+    if (c < C && k < N * kCols) f = fn[(static_cast<size_t>(k / kCols) * H + g * kCols + k % kCols) * C + c];
+    __nv_bfloat16 hi, mid, lo;
+    split3(f, hi, mid, lo);
+    dst[(0 * CP8 + c) * KS + k] = hi;
+    dst[(1 * CP8 + c) * KS + k] = mid;
+    dst[(2 * CP8 + c) * KS + k] = lo;
+  }
+}
 
 // MXFP8 of a bf16 [R, H] matrix: a lane quantises 8 columns, 4 lanes a block.
 __global__ void __launch_bounds__(256) mxfp8_rows_kernel(const __nv_bfloat16* __restrict__ x, int R, int H,
@@ -980,13 +1056,15 @@ size_t ws_layout(int R, int H, int n, size_t* sc2_off, size_t* dot_off) {
 }
 
 bool shape_ok(int R, int H, int n) {
-  return R >= 1 && R <= kMaxRows && H >= kCols && H % kCols == 0 && (n == 1 || n == 2 || n == 4);
+  return R >= 1 && R <= kMaxRows && H >= kCols && H % kCols == 0 && H / kCols <= kMaxBlocks &&
+         (n == 1 || n == 2 || n == 4);
 }
 
 mhc_status check_coeff(const mhc_coeff_args* a) {
   if (a == nullptr) return MHC_OK;
-  if (!a->fn || !a->scale || !a->base) return MHC_ERR_INVALID_ARG;
-  if (!aligned(a->fn, 16) || !aligned(a->scale, 4) || !aligned(a->base, 4)) return MHC_ERR_INVALID_ARG;
+  if ((!a->fn && !a->fn_packed) || !a->scale || !a->base) return MHC_ERR_INVALID_ARG;
+  if (!aligned(a->fn, 16) || !aligned(a->fn_packed, 16) || !aligned(a->scale, 4) || !aligned(a->base, 4))
+    return MHC_ERR_INVALID_ARG;
   if (!(a->rms_eps >= 0.f) || !(a->pre_eps >= 0.f) || !(a->sinkhorn_eps >= 0.f)) return MHC_ERR_INVALID_ARG;
   if (a->sinkhorn_iters < 0 || a->sinkhorn_iters > kMaxIters) return MHC_ERR_INVALID_ARG;
   return MHC_OK;
@@ -1062,11 +1140,14 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
     p.tail_streams = FRONT == kStreams ? p.residual : p.residual_out;
     p.tail_broadcast = 0;
   }
-  // coefficient blocks run beside the G layer-input blocks, on the SMs those leave
-  p.tail_layer_blocks = p.do_layer ? G : 0;
+  // layer-input blocks: one 256-column task per warp, at most G blocks; coefficient
+  // blocks run beside them, on the SMs those leave
+  const int tasks = p.R * ((G + 3) / 4);
+  const int lb = (tasks + kWarps - 1) / kWarps;
+  p.tail_layer_blocks = p.do_layer ? (lb < G ? lb : G) : 0;
   const int spare = sm_count() - p.tail_layer_blocks;
   p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
-  return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>(p.R).total,
+  return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>().total,
                     stream, p);
 }
 
@@ -1116,6 +1197,7 @@ mhc_status fill_tail(Params& p, const float* pre, const mhc_bf16* norm_weight, f
   if (coeffs) {
     p.do_coeff = 1;
     p.fn = coeffs->fn;
+    p.fn_packed = static_cast<const __nv_bfloat16*>(coeffs->fn_packed);
     p.scale = coeffs->scale;
     p.base = coeffs->base;
     p.rms_eps = coeffs->rms_eps;
@@ -1275,6 +1357,7 @@ mhc_status mhc_coeffs(const mhc_bf16* residual, const mhc_coeff_args* coeffs, co
   p.H = hidden;
   p.do_coeff = 1;
   p.fn = coeffs->fn;
+  p.fn_packed = static_cast<const __nv_bfloat16*>(coeffs->fn_packed);
   p.scale = coeffs->scale;
   p.base = coeffs->base;
   p.rms_eps = coeffs->rms_eps;
@@ -1343,6 +1426,27 @@ mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden, const mh
       }
     }
   }
+  return MHC_OK;
+}
+
+size_t mhc_projection_pack_bytes(int hidden, int hc_mult) {
+  if (!shape_ok(1, hidden, hc_mult)) return 0;
+  const int G = hidden / kCols;
+  const int pb = hc_mult == 1 ? packed_slice_bytes(1) : (hc_mult == 2 ? packed_slice_bytes(2) : packed_slice_bytes(4));
+  return static_cast<size_t>(G) * pb;
+}
+
+mhc_status mhc_projection_pack(const float* fn, void* packed, int hidden, int hc_mult, mhc_stream stream) {
+  if (!shape_ok(1, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (!fn || !packed || !aligned(fn, 4) || !aligned(packed, 16)) return MHC_ERR_INVALID_ARG;
+  const int G = hidden / kCols;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(packed);
+  switch (hc_mult) {
+    case 1: pack_projection_kernel<1><<<G, 256, 0, stream>>>(fn, hidden, out); break;
+    case 2: pack_projection_kernel<2><<<G, 256, 0, stream>>>(fn, hidden, out); break;
+    default: pack_projection_kernel<4><<<G, 256, 0, stream>>>(fn, hidden, out); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
   return MHC_OK;
 }
 

@@ -62,6 +62,7 @@ class DecodeLoop:
     top_k: int = 8
     seed: int = 5000
     device: str = "cuda"
+    pack_fn: bool = True  # fn packed once at weight load (mhc_projection_pack)
     steps: List[Step] = field(default_factory=list)
 
     def __post_init__(self):
@@ -83,7 +84,7 @@ class DecodeLoop:
             g = S.gen(seed)
             cw = S.draw_coeff_weights(g, H, n, 0.01, affine=True)
             nw = (1.0 + torch.randn(H, generator=g) * 0.1).to(torch.bfloat16)
-            return BoundaryWeights(M.Coeffs.from_weights(cw, dev), nw.to(dev))
+            return BoundaryWeights(M.Coeffs.from_weights(cw, dev, packed=self.pack_fn), nw.to(dev))
 
         def attn_pending(seed):
             g = S.gen(seed)

@@ -39,7 +39,7 @@ class CoeffArgs(ctypes.Structure):
     _fields_ = [("fn", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("base", ctypes.c_void_p),
                 ("rms_eps", ctypes.c_float), ("pre_eps", ctypes.c_float),
                 ("sinkhorn_eps", ctypes.c_float), ("post_alpha", ctypes.c_float),
-                ("sinkhorn_iters", ctypes.c_int)]
+                ("sinkhorn_iters", ctypes.c_int), ("fn_packed", ctypes.c_void_p)]
 
 
 class Mxfp8Out(ctypes.Structure):
@@ -48,8 +48,10 @@ class Mxfp8Out(ctypes.Structure):
 
 @dataclass
 class Coeffs:
-    """Device tensors and scalars of the next-coefficient step (mhc_coeff_args)."""
-    fn: torch.Tensor
+    """Device tensors and scalars of the next-coefficient step (mhc_coeff_args).
+    `fn_packed` (optional) is fn as mhc_projection_pack wrote it; with it set the
+    kernels read it instead of fn, and fn may be None."""
+    fn: Optional[torch.Tensor]
     scale: torch.Tensor
     base: torch.Tensor
     rms_eps: float = 1e-6
@@ -57,13 +59,20 @@ class Coeffs:
     sinkhorn_eps: float = 1e-6
     post_alpha: float = 2.0
     sinkhorn_iters: int = 20
+    fn_packed: Optional[torch.Tensor] = None
 
     @classmethod
-    def from_weights(cls, w, device) -> "Coeffs":
-        """From any object with the same fields (e.g. synthetic.CoeffWeights) on the CPU."""
-        return cls(fn=w.fn.to(device).contiguous(), scale=w.scale.to(device).contiguous(),
-                   base=w.base.to(device).contiguous(), rms_eps=w.rms_eps, pre_eps=w.pre_eps,
-                   sinkhorn_eps=w.sinkhorn_eps, post_alpha=w.post_alpha, sinkhorn_iters=w.sinkhorn_iters)
+    def from_weights(cls, w, device, packed: bool = False) -> "Coeffs":
+        """From any object with the same fields (e.g. synthetic.CoeffWeights) on the CPU;
+        `packed` also packs fn (mhc_projection_pack) on `device`."""
+        fn = w.fn.to(device).contiguous()
+        c = cls(fn=fn, scale=w.scale.to(device).contiguous(), base=w.base.to(device).contiguous(),
+                rms_eps=w.rms_eps, pre_eps=w.pre_eps, sinkhorn_eps=w.sinkhorn_eps, post_alpha=w.post_alpha,
+                sinkhorn_iters=w.sinkhorn_iters)
+        if packed:
+            n = int(round((fn.shape[1] + 1) ** 0.5)) - 1  # C = n^2 + 2n
+            c.fn_packed = mhc_projection_pack(fn, fn.shape[0] // n, n)
+        return c
 
 
 _lib = None
@@ -95,6 +104,8 @@ def lib() -> ctypes.CDLL:
         "mhc_get_device_status": (_i, [_vp, _vp]),
         "mhc_status_string": (ctypes.c_char_p, [_i]),
         "mhc_debug_set_wait": (_i64, [_i64, _i]),
+        "mhc_projection_pack_bytes": (_sz, [_i, _i]),
+        "mhc_projection_pack": (_i, [_vp, _vp, _i, _i, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -140,12 +151,13 @@ def _coeff_struct(c: Optional[Coeffs]):
     if c is None:
         return None
     _need(c.fn, torch.float32, "fn", 2)
+    _need(c.fn_packed, torch.uint8, "fn_packed", 1)
     _need(c.scale, torch.float32, "scale", 1)
     _need(c.base, torch.float32, "base", 1)
-    for t, n in ((c.fn, "fn"), (c.scale, "scale"), (c.base, "base")):
+    for t, n in ((c.fn, "fn"), (c.fn_packed, "fn_packed"), (c.scale, "scale"), (c.base, "base")):
         _contig(t, n)
-    return CoeffArgs(c.fn.data_ptr(), c.scale.data_ptr(), c.base.data_ptr(), c.rms_eps, c.pre_eps,
-                     c.sinkhorn_eps, c.post_alpha, int(c.sinkhorn_iters))
+    return CoeffArgs(_p(c.fn), c.scale.data_ptr(), c.base.data_ptr(), c.rms_eps, c.pre_eps,
+                     c.sinkhorn_eps, c.post_alpha, int(c.sinkhorn_iters), _p(c.fn_packed))
 
 
 def _mxfp8_struct(q):
@@ -188,6 +200,31 @@ def mhc_workspace_init(workspace: torch.Tensor, stream=None):
 def mhc_get_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise `stream`, then read and clear the status a kernel recorded."""
     return int(lib().mhc_get_device_status(_p(workspace), _stream(stream)))
+
+
+def mhc_projection_pack_bytes(hidden: int, hc_mult: int) -> int:
+    return int(lib().mhc_projection_pack_bytes(hidden, hc_mult))
+
+
+def mhc_projection_pack(fn: torch.Tensor, hidden: int, hc_mult: int, out: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """fn [n*H, C] fp32 rewritten into the projection's tile form (a uint8 device
+    tensor of mhc_projection_pack_bytes); done once per weight, at load time."""
+    _need(fn, torch.float32, "fn", 2)
+    _contig(fn, "fn")
+    n = mhc_projection_pack_bytes(hidden, hc_mult)
+    if n == 0:
+        raise MhcError(UNSUPPORTED_SHAPE, "mhc_projection_pack_bytes")
+    C = 2 * hc_mult + hc_mult * hc_mult
+    if tuple(fn.shape) != (hc_mult * hidden, C):
+        raise ValueError(f"fn must be [{hc_mult * hidden}, {C}], got {tuple(fn.shape)}")
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=fn.device)
+    _need(out, torch.uint8, "packed", 1)
+    if out.numel() < n:
+        raise ValueError(f"packed needs {n} bytes")
+    _check(lib().mhc_projection_pack(_p(fn), _p(out), hidden, hc_mult, _stream(stream)), "mhc_projection_pack")
+    return out
 
 
 def mhc_debug_set_wait(budget_ns: int, extra_units: int) -> int:

@@ -75,7 +75,7 @@ def alloc_outputs(R, n, H, mxfp8=True, swizzled=True, coeff=True):
 
 
 def gpu_post_pre(d: dict, *, mxfp8=True, swizzled=True, coeff=True, residual_only=False, ws=None,
-                 in_place=False, partials=None):
+                 in_place=False, partials=None, packed=False):
     """Run mhc_boundary_post_pre on the inputs of synthetic.draw_boundary; CPU results."""
     g = to_dev({k: d[k] for k in ("partials", "residual", "post", "comb", "pre", "norm_weight")})
     R, n, H = g["residual"].shape
@@ -86,7 +86,7 @@ def gpu_post_pre(d: dict, *, mxfp8=True, swizzled=True, coeff=True, residual_onl
         out["residual_out"] = g["residual"]
     if ws is None:
         ws = M.new_workspace(R, H, n, DEV)
-    cw = None if (not coeff or residual_only) else M.Coeffs.from_weights(d["coeff"], DEV)
+    cw = None if (not coeff or residual_only) else M.Coeffs.from_weights(d["coeff"], DEV, packed=packed)
     M.mhc_boundary_post_pre(
         g["partials"], g["residual"], g["post"], g["comb"], None if residual_only else g["pre"],
         None if residual_only else g["norm_weight"], d["norm_eps"], cw, out["residual_out"],

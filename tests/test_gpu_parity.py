@@ -124,7 +124,7 @@ def test_sinkhorn_iteration_counts_and_eps():
 
 # ---------------------------------------------------------------- MoE finalize
 
-def _moe_gpu(d, pre=True, mxfp8=False, coeff=True, ws=None, check_status=True):
+def _moe_gpu(d, pre=True, mxfp8=False, coeff=True, ws=None, check_status=True, packed=False):
     g = to_dev(d)
     R, n, H = g["residual"].shape
     out = alloc_outputs(R, n, H, mxfp8, True, coeff)
@@ -132,7 +132,8 @@ def _moe_gpu(d, pre=True, mxfp8=False, coeff=True, ws=None, check_status=True):
     M.mhc_boundary_moe_finalize(
         g["gemm2_permuted"], g["expert_weights"], g["expanded_idx_to_permuted_idx"], g["shared_output"],
         g["residual"], g["post"], g["comb"], g["pre"] if pre else None, g["norm_weight"] if pre else None,
-        d["norm_eps"], M.Coeffs.from_weights(d["coeff"], DEV) if (coeff and pre) else None, out["residual_out"],
+        d["norm_eps"], M.Coeffs.from_weights(d["coeff"], DEV, packed=packed) if (coeff and pre) else None,
+        out["residual_out"],
         layer_input=out["layer_input"] if pre else None,
         mxfp8=(out["q_data"], out["q_scale"], True) if mxfp8 else None,
         post_out=out.get("post"), comb_out=out.get("comb"), pre_out=out.get("pre"), workspace=ws)
@@ -304,6 +305,70 @@ def test_mxfp8_nonfinite_block():
     assert np.array_equal(scale.cpu().numpy(), osc.reshape(-1))
 
 
+# ---------------------------------------------------------------- packed projection weights
+
+@pytest.mark.parametrize("R,H,n,P", [(1, 7168, 4, 8), (5, 192, 4, 3), (13, 320, 2, 16), (7, 64, 1, 2),
+                                     (32, 7168, 4, 8), (128, 7168, 4, 8), (100, 9472, 4, 4)])
+def test_packed_projection_matches_fn_bitwise(R, H, n, P):
+    # fn packed once into bf16 terms gives the same bits as the in-kernel split,
+    # and so the oracle's results at the parity tolerances
+    d = S.draw_boundary(R, H, n=n, partials=P, seed=4100 + R + n)
+    a = gpu_post_pre(d)
+    b = gpu_post_pre(d, packed=True)
+    for k in a:
+        assert torch.equal(a[k], b[k]), f"R={R} H={H} n={n}: {k} differs with packed fn"
+    if R <= 32:
+        orc = oracle_post_pre(d)
+        assert_bf16_close(f64(b["residual_out"]), orc["residual"], "packed residual")
+        check_tail(d, b, orc, what=f"packed R={R} H={H} n={n}")
+
+
+def test_packed_projection_moe_and_coeffs_entry():
+    d = S.draw_moe(32, 7168, n=4, top_k=8, seed=4232)
+    a, _ = _moe_gpu(d, mxfp8=True)
+    b, _ = _moe_gpu(d, mxfp8=True, packed=True)
+    for k in a:
+        assert torch.equal(a[k], b[k]), f"moe: {k} differs with packed fn"
+    d = S.draw_boundary(24, 7168, n=4, partials=1, seed=4824)
+    g = to_dev(d)
+    outs = []
+    for packed in (False, True):
+        cw = M.Coeffs.from_weights(d["coeff"], DEV, packed=packed)
+        if packed:
+            cw.fn = None  # the packed form alone is enough
+        out = alloc_outputs(24, 4, 7168, False, True, True)
+        ws = M.new_workspace(24, 7168, 4, DEV)
+        M.mhc_coeffs(cw, out["post"], out["comb"], out["pre"], residual=g["residual"], pre_mix=g["pre"],
+                     norm_weight=g["norm_weight"], norm_eps=d["norm_eps"], layer_input=out["layer_input"],
+                     workspace=ws)
+        torch.cuda.synchronize()
+        assert M.mhc_get_device_status(ws) == M.OK
+        outs.append({k: out[k].cpu() for k in ("post", "comb", "pre", "layer_input")})
+    for k in outs[0]:
+        assert torch.equal(outs[0][k], outs[1][k]), f"coeffs entry: {k} differs with packed fn"
+
+
+@pytest.mark.parametrize("n", [1, 4])
+def test_packed_layout_holds_the_three_bf16_terms(n):
+    # element (t, c, k) of block g is term t of fn[(k/64)*H + 64g + k%64][c]; terms add back to fn
+    H = 128
+    C = 2 * n + n * n
+    fn = torch.randn(n * H, C, dtype=torch.float32) * 0.02
+    pk = M.mhc_projection_pack(fn.to(DEV), H, n)
+    torch.cuda.synchronize()
+    KS, CP8 = n * 64 + 8, ((C + 7) // 8) * 8
+    t = pk.cpu().view(torch.bfloat16).view(H // 64, 3, CP8, KS).to(torch.float64)
+    for g in range(H // 64):
+        for k in [k for k in (0, 5, 63, 64, 200, n * 64 - 1) if k < n * 64]:
+            row = (k // 64) * H + 64 * g + k % 64
+            s = t[g, 0, :C, k] + t[g, 1, :C, k] + t[g, 2, :C, k]
+            assert torch.allclose(s, fn[row].double(), rtol=2 ** -22, atol=0), (g, k)
+            hi = fn[row].to(torch.bfloat16).double()
+            assert torch.equal(t[g, 0, :C, k], hi), (g, k)
+    for pad in (t[:, :, C:, :], t[:, :, :, n * 64:]):  # padding columns and gaps are zero
+        assert pad.numel() == 0 or float(pad.abs().max()) == 0.0
+
+
 # ---------------------------------------------------------------- bounded waits
 
 def test_weight_copy_wait_times_out_and_recovers():
@@ -327,3 +392,24 @@ def test_weight_copy_wait_times_out_and_recovers():
     gpu = gpu_post_pre(d, ws=ws)
     orc = oracle_post_pre(d)
     check_tail(d, gpu, orc, what="after recovery")
+
+
+def test_packed_weight_copy_wait_times_out_and_recovers():
+    # the same with packed fn, whose copy is waited for only before the projection
+    d = S.draw_boundary(4, 256, n=4, partials=2, seed=19)
+    ws = M.new_workspace(4, 256, 4, DEV)
+    old = M.mhc_debug_set_wait(20_000_000, 1)  # 20 ms
+    try:
+        g = to_dev(d)
+        out = alloc_outputs(4, 4, 256)
+        M.mhc_boundary_post_pre(g["partials"], g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"],
+                                d["norm_eps"], M.Coeffs.from_weights(d["coeff"], DEV, packed=True),
+                                out["residual_out"], layer_input=out["layer_input"], post_out=out["post"],
+                                comb_out=out["comb"], pre_out=out["pre"], workspace=ws)
+        assert M.mhc_get_device_status(ws) == M.DEVICE_TIMEOUT
+    finally:
+        M.mhc_debug_set_wait(old, 0)
+    assert M.mhc_get_device_status(ws) == M.OK
+    gpu = gpu_post_pre(d, ws=ws, packed=True)
+    orc = oracle_post_pre(d)
+    check_tail(d, gpu, orc, what="packed, after recovery")

@@ -52,8 +52,15 @@ def test_sizes(L):
     ws = M.mhc_workspace_bytes(32, 7168, 4)
     assert ws >= 1024 + 32 * 112 * 4 + 32 * 112 * 32 * 4
     assert M.mhc_workspace_bytes(16, 7168, 4) <= ws  # smaller rows fit a larger workspace
-    for bad in ((0, 7168, 4), (129, 7168, 4), (4, 7100, 4), (4, 7168, 3), (4, 7168, 8)):
+    for bad in ((0, 7168, 4), (129, 7168, 4), (4, 7100, 4), (4, 7168, 3), (4, 7168, 8), (4, 9536, 4)):
         assert M.mhc_workspace_bytes(*bad) == 0
+    assert M.mhc_workspace_bytes(4, 9472, 4) > 0  # H/64 = 148 blocks is the largest
+    # packed fn: per 64-column block [3][CP8][n*64 + 8] bf16, CP8 = C rounded up to 8
+    assert M.mhc_projection_pack_bytes(7168, 4) == 112 * 3 * 24 * 264 * 2
+    assert M.mhc_projection_pack_bytes(320, 2) == 5 * 3 * 8 * 136 * 2
+    assert M.mhc_projection_pack_bytes(64, 1) == 1 * 3 * 8 * 72 * 2
+    for bad in ((7100, 4), (7168, 3), (9536, 4), (0, 4)):
+        assert M.mhc_projection_pack_bytes(*bad) == 0
 
 
 def test_status_strings(L):
@@ -123,5 +130,13 @@ def test_other_entry_points_host_checks(L):
     assert L.mxfp8_quantize_rows(a, 4, 48, ctypes.byref(q), None) == M.UNSUPPORTED_SHAPE
     assert L.mxfp8_quantize_rows(None, 4, 64, ctypes.byref(q), None) == M.INVALID_ARG
     assert L.mxfp8_quantize_rows(a, 4, 64, None, None) == M.INVALID_ARG
+    assert L.mhc_projection_pack(a, a, 7100, 4, None) == M.UNSUPPORTED_SHAPE
+    assert L.mhc_projection_pack(None, a, 7168, 4, None) == M.INVALID_ARG
+    assert L.mhc_projection_pack(a, _fake(0x10008), 7168, 4, None) == M.INVALID_ARG  # packed not 16-aligned
+    # coefficients with neither fn nor packed fn, or a misaligned packed fn
+    for bad in (M.CoeffArgs(None, 0x10000, 0x10000, 1e-6, 1e-6, 1e-6, 2.0, 20, None),
+                M.CoeffArgs(None, 0x10000, 0x10000, 1e-6, 1e-6, 1e-6, 2.0, 20, 0x10008)):
+        assert L.mhc_coeffs(a, ctypes.byref(bad), None, None, None, None, 0.0, None, a, a, a, 4, 256, 4, a,
+                            1 << 20, None) == M.INVALID_ARG
     assert L.mhc_workspace_init(None, 4096, None) == M.WORKSPACE
     assert L.mhc_get_device_status(None, None) == M.WORKSPACE
