@@ -368,6 +368,10 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
       bs_s[(2 * CP8 + c) * KS + k] = lo;
     }
   }
+  if (warp == 1 && lane < 3) {  // the mixes' first lines: L2 and address translation warm before the wait
+    const float* mp = lane == 0 ? p.post : (lane == 1 ? p.comb : p.pre);
+    if (mp != nullptr) prefetch_l2(mp);
+  }
   // ---- 3. wait for the preceding kernel, let the next one launch, and read
   griddep_wait();
   griddep_launch_dependents();
@@ -406,34 +410,36 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
     const int r = q * 4 + rq;
     const bool valid = r < R;
     const float* mix = mix_s + (valid ? r : 0) * MIX;
-    float nf[N][8];
+    // Pairs of columns in packed f32x2 arithmetic (each element the same fp32
+    // operations, in the same order, as one at a time).
+    float2 nf[N][4];  // the new streams, as rounded to bf16
     uint4 nb[N];
-    float xs[8];
+    float2 xs[4];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) xs[t] = 0.f;
+    for (int t = 0; t < 4; ++t) xs[t] = make_float2(0.f, 0.f);
     if (FRONT == kPartials || FRONT == kMoe) {
-      float rf[N][8];
+      float2 rf[N][4];
       if (valid) {
 #pragma unroll
-        for (int j = 0; j < N; ++j) unpack8(cur.rv[j], rf[j]);
+        for (int j = 0; j < N; ++j) unpack8x2(cur.rv[j], rf[j]);
         if (FRONT == kPartials) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             if (u < p.P) {
-              float f[8];
-              unpack8(cur.pv[u], f);
+              float2 f[4];
+              unpack8x2(cur.pv[u], f);
 #pragma unroll
-              for (int t = 0; t < 8; ++t) xs[t] += f[t];
+              for (int t = 0; t < 4; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
             }
           }
           for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
-            float f[8];
-            unpack8(ld_nc_v4(p.partials + u * p.pstride + static_cast<size_t>(r) * H + h0), f);
+            float2 f[4];
+            unpack8x2(ld_nc_v4(p.partials + u * p.pstride + static_cast<size_t>(r) * H + h0), f);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) xs[t] += f[t];
+            for (int t = 0; t < 4; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
           }
         } else {
-          unpack8(cur.sv, xs);
+          unpack8x2(cur.sv, xs);
           const int* idx = e2p_s + r * p.topk;
           const float* wt = ew_s + r * p.topk;
 #pragma unroll
@@ -443,11 +449,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
               if (e >= p.num_perm) {
                 if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
               } else if (e >= 0) {
-                float f[8];
-                unpack8(cur.pv[u], f);
-                const float w = wt[u];
+                float2 f[4];
+                unpack8x2(cur.pv[u], f);
+                const float2 w2 = make_float2(wt[u], wt[u]);
 #pragma unroll
-                for (int t = 0; t < 8; ++t) xs[t] = fmaf(w, f[t], xs[t]);
+                for (int t = 0; t < 4; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
               }
             }
           }
@@ -456,11 +462,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
             if (e >= p.num_perm) {
               if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
             } else if (e >= 0) {
-              float f[8];
-              unpack8(ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0), f);
-              const float w = wt[u];
+              float2 f[4];
+              unpack8x2(ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0), f);
+              const float2 w2 = make_float2(wt[u], wt[u]);
 #pragma unroll
-              for (int t = 0; t < 8; ++t) xs[t] = fmaf(w, f[t], xs[t]);
+              for (int t = 0; t < 4; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
             }
           }
         }
@@ -468,36 +474,39 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
 #pragma unroll
         for (int j = 0; j < N; ++j)
 #pragma unroll
-          for (int t = 0; t < 8; ++t) rf[j][t] = 0.f;
+          for (int t = 0; t < 4; ++t) rf[j][t] = make_float2(0.f, 0.f);
       }
       // mHC post: new[i] = bf16(post[i] * x + sum_j comb[j][i] * res[j])
 #pragma unroll
       for (int i = 0; i < N; ++i) {
-        float a[8];
-        const float po = mix[i];
+        float2 a[4];
+        const float2 po = make_float2(mix[i], mix[i]);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          float s = po * xs[t];
+        for (int t = 0; t < 4; ++t) {
+          float2 s2 = __fmul2_rn(po, xs[t]);
 #pragma unroll
-          for (int j = 0; j < N; ++j) s = fmaf(mix[N + j * N + i], rf[j][t], s);
-          a[t] = s;
+          for (int j = 0; j < N; ++j) {
+            const float cj = mix[N + j * N + i];
+            s2 = __ffma2_rn(make_float2(cj, cj), rf[j][t], s2);
+          }
+          a[t] = s2;
         }
-        nb[i] = round8(a, nf[i]);
+        nb[i] = round8x2(a, nf[i]);
       }
     } else if (FRONT == kStreams) {
 #pragma unroll
       for (int j = 0; j < N; ++j) {
         nb[j] = valid ? cur.rv[j] : make_uint4(0, 0, 0, 0);
-        unpack8(nb[j], nf[j]);
+        unpack8x2(nb[j], nf[j]);
       }
     } else {  // kBroadcast: every stream is the embedding row
       const uint4 xv = valid ? cur.sv : make_uint4(0, 0, 0, 0);
-      unpack8(xv, xs);
+      unpack8x2(xv, xs);
 #pragma unroll
       for (int j = 0; j < N; ++j) {
         nb[j] = xv;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) nf[j][t] = xs[t];
+        for (int t = 0; t < 4; ++t) nf[j][t] = xs[t];
       }
     }
     if (p.write_res && valid) {
@@ -505,30 +514,32 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
       for (int i = 0; i < N; ++i) st_v4(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
     }
     if (p.do_layer) {  // collapse with the carried pre (identity pre-mix for the broadcast)
-      float c[8];
-      float sc2 = 0.f;
+      float2 sq = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
+      for (int t = 0; t < 4; ++t) {
+        float2 c;
         if (FRONT == kBroadcast) {
-          c[t] = xs[t];
+          c = xs[t];
         } else {
-          float s = 0.f;
+          c = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int j = 0; j < N; ++j) s = fmaf(mix[N + N * N + j], nf[j][t], s);
-          c[t] = s;
+          for (int j = 0; j < N; ++j) {
+            const float pj = mix[N + N * N + j];
+            c = __ffma2_rn(make_float2(pj, pj), nf[j][t], c);
+          }
         }
-        sc2 = fmaf(c[t], c[t], sc2);
+        sq = __ffma2_rn(c, c, sq);
       }
-      sc2 = sum8_lanes(sc2);
+      const float sc2 = sum8_lanes(sq.x + sq.y);
       if (valid && vec == 0) p.sc2_part[r * G + g] = sc2;
     }
     if (p.do_coeff) {  // stage the streams for the projection; sum v^2 of the row
-      float sv2 = 0.f;
+      float2 sv = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < N; ++i)
 #pragma unroll
-        for (int t = 0; t < 8; ++t) sv2 = fmaf(nf[i][t], nf[i][t], sv2);
-      sv2 = sum8_lanes(sv2);
+        for (int t = 0; t < 4; ++t) sv = __ffma2_rn(nf[i][t], nf[i][t], sv);
+      const float sv2 = sum8_lanes(sv.x + sv.y);
       if (valid) {
 #pragma unroll
         for (int i = 0; i < N; ++i) *reinterpret_cast<uint4*>(v_s + r * KS + i * kCols + vec * 8) = nb[i];
@@ -728,6 +739,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
     if (w0 < T) {  // norm weights of the first task: weights, so before the wait
       const int g = (w0 % GT) * 4 + rq;
       if (g < G) cur.nw = ld_nc_v4(p.norm_weight + g * kCols + vec * 8);
+      // lines the first task reads after the wait: L2 and address translation warm
+      const int r = w0 / GT;
+      if (lane == 0) prefetch_l2(p.sc2_part + r * G);
+      if (lane == 1 && !p.tail_broadcast) prefetch_l2(p.pre + r * N);
+      if (lane == 2) prefetch_l2(p.tail_streams + static_cast<size_t>(r) * (p.tail_broadcast ? 1 : N) * H);
     }
     griddep_wait();
     griddep_launch_dependents();
@@ -840,6 +856,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
     const int CB = p.tail_coeff_blocks;
     if (tid < 3) cp_async4(scale_s + tid, p.scale + tid);  // weights: before the wait
     if (tid >= 32 && tid < 32 + C) cp_async4(base_s + tid - 32, p.base + (tid - 32));
+    if (tid == 64) prefetch_l2(p.dot_part + static_cast<size_t>(jb) * G * RED);  // warm, as above
     griddep_wait();
     griddep_launch_dependents();
     constexpr int V4 = RED / 4;
@@ -893,43 +910,52 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
         }
       }
       __syncthreads();
-      if (warp < nk) {
-        const int r = jb + (k0 + warp) * CB;
+      // warp s < nk: the comb (Sinkhorn) of row s of the batch; the pre and post of
+      // row s go to warp s + nk where there is one, else warp s does them after
+      const int s_comb = warp < nk ? warp : -1;
+      const int s_pp = warp < nk ? (warp + nk < kWarps ? -1 : warp) : (warp - nk < nk ? warp - nk : -1);
+      if (s_comb >= 0 || s_pp >= 0) {
+        const int sl = s_comb >= 0 ? s_comb : s_pp;
+        const int r = jb + (k0 + sl) * CB;
         float s = 0.f;  // lane c: record value c, the warps' shares added in order
         if (lane < RED) {
 #pragma unroll
-          for (int w = 0; w < kWarps; ++w) s += slot_s[(warp * kWarps + w) * RED + lane];
+          for (int w = 0; w < kWarps; ++w) s += slot_s[(sl * kWarps + w) * RED + lane];
         }
         const float inv = rsqrtf(__fdiv_rn(__shfl_sync(kFull, s, C), static_cast<float>(N * H)) + p.rms_eps);
         const int grp = lane < N ? 0 : (lane < 2 * N ? 1 : 2);
         const float l = lane < C ? scale_s[grp] * inv * s + base_s[lane] : 0.f;
-        if (lane < N) {
-          p.pre_out[r * N + lane] = 1.f / (1.f + expf(-l)) + p.pre_eps;
-        } else if (lane < 2 * N) {
-          p.post_out[r * N + (lane - N)] = p.alpha / (1.f + expf(-l));
+        if (s_comb >= 0) {
+          // Sinkhorn in one thread: M = exp(L - max L); rows then columns, iters times
+          float lc[NN];
+#pragma unroll
+          for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, l, 2 * N + k);
+          if (lane == 0) {
+            float t[NN];
+#pragma unroll
+            for (int k = 0; k < NN; ++k) t[k] = lc[k];
+#pragma unroll
+            for (int w = NN / 2; w >= 1; w >>= 1)
+#pragma unroll
+              for (int k = 0; k < w; ++k) t[k] = fmaxf(t[k], t[k + w]);
+            float M[N][N];
+#pragma unroll
+            for (int j = 0; j < N; ++j)
+#pragma unroll
+              for (int i = 0; i < N; ++i) M[j][i] = expf(lc[j * N + i] - t[0]);
+            sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
+#pragma unroll
+            for (int j = 0; j < N; ++j)
+#pragma unroll
+              for (int i = 0; i < N; ++i) p.comb_out[r * NN + j * N + i] = M[j][i];
+          }
         }
-        // Sinkhorn in one thread: M = exp(L - max L); rows then columns, iters times
-        float lc[NN];
-#pragma unroll
-        for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, l, 2 * N + k);
-        if (lane == 0) {
-          float t[NN];
-#pragma unroll
-          for (int k = 0; k < NN; ++k) t[k] = lc[k];
-#pragma unroll
-          for (int w = NN / 2; w >= 1; w >>= 1)
-#pragma unroll
-            for (int k = 0; k < w; ++k) t[k] = fmaxf(t[k], t[k + w]);
-          float M[N][N];
-#pragma unroll
-          for (int j = 0; j < N; ++j)
-#pragma unroll
-            for (int i = 0; i < N; ++i) M[j][i] = expf(lc[j * N + i] - t[0]);
-          sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
-#pragma unroll
-          for (int j = 0; j < N; ++j)
-#pragma unroll
-            for (int i = 0; i < N; ++i) p.comb_out[r * NN + j * N + i] = M[j][i];
+        if (s_pp >= 0) {
+          if (lane < N) {
+            p.pre_out[r * N + lane] = 1.f / (1.f + expf(-l)) + p.pre_eps;
+          } else if (lane < 2 * N) {
+            p.post_out[r * N + (lane - N)] = p.alpha / (1.f + expf(-l));
+          }
         }
       }
       __syncthreads();  // the slots are refilled by the next batch

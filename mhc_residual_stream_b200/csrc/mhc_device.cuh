@@ -157,6 +157,13 @@ __device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8]) {
   }
 }
 
+// The same as column pairs: f[m] = (element 2m, element 2m + 1).
+__device__ __forceinline__ void unpack8x2(const uint4 v, float2 (&f)[4]) {
+  const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int m = 0; m < 4; ++m) f[m] = make_float2(__uint_as_float(w[m] << 16), __uint_as_float(w[m] & 0xffff0000u));
+}
+
 __device__ __forceinline__ unsigned pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<unsigned*>(&b);
@@ -170,6 +177,16 @@ __device__ __forceinline__ uint4 round8(const float (&f)[8], float (&r)[8]) {
   v.z = pack_bf16x2(f[4], f[5]);
   v.w = pack_bf16x2(f[6], f[7]);
   unpack8(v, r);
+  return v;
+}
+
+__device__ __forceinline__ uint4 round8x2(const float2 (&f)[4], float2 (&r)[4]) {
+  uint4 v;
+  v.x = pack_bf16x2(f[0].x, f[0].y);
+  v.y = pack_bf16x2(f[1].x, f[1].y);
+  v.z = pack_bf16x2(f[2].x, f[2].y);
+  v.w = pack_bf16x2(f[3].x, f[3].y);
+  unpack8x2(v, r);
   return v;
 }
 

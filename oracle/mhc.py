@@ -41,6 +41,8 @@ __all__ = [
     "rms_norm",
     "logit_groups",
     "mhc_coefficients",
+    "stream_mean",
+    "final_head",
     "boundary",
     "coeffs_entry",
 ]
@@ -397,9 +399,29 @@ def rms_norm(c, weight, eps):
     return bf16_round(c * inv[:, None] * np.asarray(weight, dtype=np.float64)[None, :])
 
 
+def stream_mean(streams):
+    """aux[r, h] = bf16(mean over j of streams[r, j, h]).
+
+    The hidden state a boundary keeps for the layers that capture it
+    ([boundary: Boundaries.sublayer] with capture_aux: the mean over dim 1 of
+    the new streams; [decode: SpecializedDecode.run] the same after the last
+    post_only). READING: the exact mean rounded once to bf16 (torch reduces
+    bf16 in fp32 and rounds the result once; for n <= 4 bf16 inputs the fp32
+    sum is exact unless the inputs span more than 16 binades).
+    """
+    return bf16_round(np.mean(np.asarray(streams, dtype=np.float64), axis=1))
+
+
+def final_head(streams, pre, norm_weight, norm_eps):
+    """The decode step's hidden state after the last layer ([decode:
+    SpecializedDecode._head]): the final norm of hc_collapse(streams, pre),
+    with the pre carried from the last boundary that computed one."""
+    return rms_norm(collapse(streams, pre), norm_weight, norm_eps)
+
+
 def boundary(*, residual, post, comb, partials=None, moe=None, pre=None,
              norm_weight=None, norm_eps=0.0, coeff=None, mxfp8=False,
-             swizzled=True):
+             swizzled=True, aux=False):
     """One boundary: reduce pending, post-mix, and with ``pre`` the layer input
     and (with ``coeff``) the next coefficients.
 
@@ -410,6 +432,8 @@ def boundary(*, residual, post, comb, partials=None, moe=None, pre=None,
     no pre, no norm); it returns the streams only.
     ``coeff`` = dict(fn, scale, base, rms_eps, pre_eps, sinkhorn_eps,
     post_alpha, sinkhorn_iters) or None.
+
+    ``aux`` also returns 'aux', the stream mean of the new streams.
 
     Returns a dict with 'residual' and, with pre: 'layer_input', and with
     mxfp8: 'mxfp8_data', 'mxfp8_scale' (swizzled or linear bytes), and with
@@ -423,6 +447,8 @@ def boundary(*, residual, post, comb, partials=None, moe=None, pre=None,
                          moe["expanded_idx_to_permuted_idx"], moe["shared_output"])
     new = post_mix(residual, x, post, comb)
     out = {"residual": new}
+    if aux:
+        out["aux"] = stream_mean(new)
     if pre is None:
         return out
     y = rms_norm(collapse(new, pre), norm_weight, norm_eps)

@@ -321,6 +321,38 @@ def test_first_layer_broadcast_identity_pre_and_fold():
     assert np.allclose(out["post"], post, rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------- aux stream mean / final head
+
+def test_stream_mean_hand_values_and_special_cases():
+    # hand-computed: means of bf16-exact values, rounded once to bf16
+    st = np.array([[[1.0, 3.0, -2.0], [2.0, 5.0, 2.0], [4.0, 0.5, -1.0], [5.0, 0.5, 1.0]]])  # [1, 4, 3]
+    assert np.array_equal(O.stream_mean(st)[0], np.array([3.0, 2.25, 0.0]))
+    # 1 + 2^-8 is not a bf16 value: the mean of (1, 1, 1, 1 + 2^-6) = 1 + 2^-8 rounds to even, 1.0
+    st2 = np.array([[[1.0], [1.0], [1.0], [1.0 + 2.0 ** -6]]])
+    assert O.stream_mean(st2)[0, 0] == 1.0
+    # mean 1 + 3 * 2^-9 is 0.75 ulp above 1 (a bf16 ulp there is 2^-7): rounds up to 1 + 2^-7
+    st3 = np.array([[[1.0 + 2.0 ** -7], [1.0 + 2.0 ** -7], [1.0 + 2.0 ** -7], [1.0]]])
+    assert O.stream_mean(st3)[0, 0] == 1.0 + 2.0 ** -7
+    # n identical streams: the mean is the stream; n = 1: the identity
+    x = O.bf16_round(np.random.default_rng(11).standard_normal((3, 40)))
+    assert np.array_equal(O.stream_mean(np.repeat(x[:, None, :], 4, axis=1)), x)
+    assert np.array_equal(O.stream_mean(x[:, None, :]), x)
+
+
+def test_final_head_is_the_norm_of_one_stream_for_a_one_hot_pre():
+    rng = np.random.default_rng(12)
+    st = O.bf16_round(rng.standard_normal((2, 4, 64)))
+    w = O.bf16_round(1.0 + rng.standard_normal(64) * 0.1)
+    for j in range(4):
+        pre = np.zeros((2, 4))
+        pre[:, j] = 1.0
+        assert np.array_equal(O.final_head(st, pre, w, 1e-6), O.rms_norm(st[:, j], w, 1e-6))
+    # a constant row collapses to sign * weight (see the RMSNorm pin)
+    st2 = np.full((1, 4, 64), 0.5)
+    pre = np.full((1, 4), 0.25)
+    assert np.array_equal(O.final_head(st2, pre, w, 1e-12)[0], O.bf16_round(w))
+
+
 def test_residual_only_streams_equal_full_path():
     d, f = _small_boundary(R=4, H=96, P=2)
     coeff = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v)
