@@ -166,15 +166,60 @@ MHC_API mhc_status mhc_projection_pack(const float* fn, void* packed, int hidden
  *     computed from the new streams (see mhc_coeff_args).
  * pre == NULL is the residual-only variant ([boundary] Boundaries._reduce with no
  * pre and no norm): then norm_weight, layer_input, mxfp8 and coeffs must be NULL.
+ * aux_out (optional, may be NULL; 16-byte aligned) receives the hidden state a
+ * capturing layer keeps ([boundary] Boundaries.sublayer with capture_aux, and
+ * [decode] SpecializedDecode.run after the last layer): the mean of the new
+ * streams, aux[r,h] = bf16( (sum_j new[r,j,h]) / n ), summed in stream order in
+ * fp32 and rounded once.  [R, H]
+ * The decode step's final head ([decode] SpecializedDecode._head:
+ * norm(hc_collapse(streams, pre))) is this call with the carried pre, the final
+ * norm's weight and coeffs = NULL: layer_input is then the step's hidden state.
  * Inputs post [R,n], comb [R,n,n], pre [R,n] are fp32; norm_weight [H] bf16.
  * workspace: see mhc_workspace_bytes. */
 MHC_API mhc_status mhc_boundary_post_pre(
     const mhc_bf16* partials, int num_partials, int64_t partial_stride,
     const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
     const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
-    mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
     float* post_out, float* comb_out, float* pre_out,
     int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* mhc_boundary_post_pre with the partials given as a table: partials is a HOST
+ * array of num_partials DEVICE pointers, each to a [R, H] bf16 partial (16-byte
+ * aligned). A pointer may be another GPU's memory (peer access or
+ * mhc_ipc_import): this is the tensor-parallel boundary, where every rank's
+ * kernel sums all ranks' partials itself with plain peer loads, in pointer
+ * order, instead of an all-reduce before it ([boundary] Boundaries.post_only:
+ * tensor_model_parallel_all_reduce then mhc_post; [all_reduce]
+ * BoundaryAllReduce.__call__). The table is read during the call only. The
+ * caller orders the accesses: every partial complete before the call (e.g. a
+ * barrier across the ranks after their sublayers) and no partial overwritten
+ * until every rank's boundary has read it. pre == NULL is the residual-only
+ * form, which needs no workspace. */
+MHC_API mhc_status mhc_boundary_post_pre_ptrs(
+    const mhc_bf16* const* partials, int num_partials,
+    const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
+    const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+    mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    float* post_out, float* comb_out, float* pre_out,
+    int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream);
+
+/* Device memory shared between processes (one process per GPU), for the
+ * partial table above (no counterpart on the pages, which use a multicast
+ * mailbox; nothing here uses multicast).
+ *   mhc_ipc_handle_bytes: size of a handle (a CUDA IPC handle of the
+ *     allocation holding the pointer, plus the pointer's offset into it).
+ *   mhc_ipc_export: write the handle of dev_ptr (device memory from cudaMalloc
+ *     or a caching allocator built on it) into handle_out.
+ *   mhc_ipc_import: map a handle exported by ANOTHER process; *dev_ptr_out is
+ *     the same byte the exporter's pointer names. Opening a handle of the
+ *     calling process fails (MHC_ERR_CUDA).
+ *   mhc_ipc_release: unmap a pointer from mhc_ipc_import.
+ * The exporter must keep the memory allocated until every importer released it. */
+MHC_API size_t mhc_ipc_handle_bytes(void);
+MHC_API mhc_status mhc_ipc_export(const void* dev_ptr, void* handle_out);
+MHC_API mhc_status mhc_ipc_import(const void* handle, void** dev_ptr_out);
+MHC_API mhc_status mhc_ipc_release(void* dev_ptr);
 
 /* Boundary after a MoE sublayer whose output was left unfinalized ([all_reduce]
  * BoundaryAllReduce.finalize, [boundary] Boundaries._reduce):
@@ -190,17 +235,18 @@ MHC_API mhc_status mhc_boundary_moe_finalize(
     const int32_t* expanded_idx_to_permuted_idx, int top_k, const mhc_bf16* shared_output,
     const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
     const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
-    mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
     float* post_out, float* comb_out, float* pre_out,
     int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream);
 
 /* Residual-only boundary ([boundary] Boundaries.post_only: all-reduce then mHC
  * post, streams only): residual_out = bf16(comb-mix of residual + post * sum of
- * partials). Needs no workspace. */
+ * partials), and aux_out (may be NULL) as in mhc_boundary_post_pre. Needs no
+ * workspace. */
 MHC_API mhc_status mhc_boundary_residual_only(
     const mhc_bf16* partials, int num_partials, int64_t partial_stride,
     const mhc_bf16* residual, const float* post, const float* comb,
-    mhc_bf16* residual_out, int rows, int hidden, int hc_mult, mhc_stream stream);
+    mhc_bf16* residual_out, mhc_bf16* aux_out, int rows, int hidden, int hc_mult, mhc_stream stream);
 
 /* The stock mHC pre without a reduction ([boundary] Boundaries._pre), two forms:
  *   residual != NULL, x == NULL: coefficients of the given streams [R, n, H]; with
@@ -245,7 +291,7 @@ MHC_API mhc_status mhc_boundary_post_pre_noalloc(
     const mhc_bf16* partials, int num_partials, int64_t partial_stride,
     const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
     const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
-    mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+    mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
     float* post_out, float* comb_out, float* pre_out,
     int rows, int hidden, int hc_mult, mhc_stream stream);
 

@@ -27,6 +27,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
+#include <map>
 #include <mutex>
 
 #include "../../include/mhc.h"
@@ -63,8 +65,8 @@ __host__ __device__ constexpr int fn_piece_bytes(int n) { return 8 * logits_of(n
 
 struct Params {
   // front ends
-  const __nv_bfloat16* partials;
-  int64_t pstride;
+  const __nv_bfloat16* pptr[kMaxPartials];  // partial u: [R, H] at pptr[u]
+  int premote;  // partials may be other GPUs' memory: plain loads, no L2 prefetch
   int P;
   const __nv_bfloat16* gemm2;
   int num_perm;
@@ -87,6 +89,7 @@ struct Params {
   float rms_eps, pre_eps, sk_eps, alpha;
   int iters;
   __nv_bfloat16* residual_out;
+  __nv_bfloat16* aux_out;  // stream mean of the new streams [R, H], or null
   __nv_bfloat16* layer_input;
   uint8_t* q_data;
   uint8_t* q_scale;
@@ -238,10 +241,16 @@ __device__ __forceinline__ void load_quad(const Params& p, int r, int h0, const 
     for (int j = 0; j < N; ++j) Q.rv[j] = ld_v4(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
   }
   if (FRONT == kPartials) {
-    const __nv_bfloat16* base = p.partials + static_cast<size_t>(r) * H + h0;
+    const size_t off = static_cast<size_t>(r) * H + h0;
+    if (p.premote) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (u < p.P) Q.pv[u] = ld_nc_v4(base + u * p.pstride);
+      for (int u = 0; u < 8; ++u)
+        if (u < p.P) Q.pv[u] = ld_v4(p.pptr[u] + off);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < p.P) Q.pv[u] = ld_nc_v4(p.pptr[u] + off);
+    }
   } else if (FRONT == kMoe) {
     Q.sv = ld_nc_v4(p.shared_out + static_cast<size_t>(r) * H + h0);
     const int* idx = e2p_s + r * p.topk;
@@ -340,7 +349,8 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
         for (int j = 0; j < N; ++j) prefetch_l2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
       }
       if (FRONT == kPartials) {
-        for (int pp = 0; pp < p.P; ++pp) prefetch_l2(p.partials + pp * p.pstride + static_cast<size_t>(r) * H + h0);
+        if (!p.premote)
+          for (int pp = 0; pp < p.P; ++pp) prefetch_l2(p.pptr[pp] + static_cast<size_t>(r) * H + h0);
       } else if (FRONT == kMoe) {
         prefetch_l2(p.shared_out + static_cast<size_t>(r) * H + h0);
         for (int t = 0; t < p.topk; ++t) {
@@ -434,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
           }
           for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
             float2 f[4];
-            unpack8x2(ld_nc_v4(p.partials + u * p.pstride + static_cast<size_t>(r) * H + h0), f);
+            const __nv_bfloat16* src = p.pptr[u] + static_cast<size_t>(r) * H + h0;
+            unpack8x2(p.premote ? ld_v4(src) : ld_nc_v4(src), f);
 #pragma unroll
             for (int t = 0; t < 4; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
           }
@@ -512,6 +523,20 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
     if (p.write_res && valid) {
 #pragma unroll
       for (int i = 0; i < N; ++i) st_v4(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
+    }
+    if (p.aux_out != nullptr && valid) {  // mean over the streams, in stream order, rounded once
+      constexpr float kInvN = 1.f / N;    // exact: n is a power of two
+      uint4 ab;
+      unsigned* aw = reinterpret_cast<unsigned*>(&ab);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float2 m = nf[0][t];
+#pragma unroll
+        for (int j = 1; j < N; ++j) m = __fadd2_rn(m, nf[j][t]);
+        m = __fmul2_rn(m, make_float2(kInvN, kInvN));
+        aw[t] = pack_bf16x2(m.x, m.y);
+      }
+      st_v4(p.aux_out + static_cast<size_t>(r) * H + h0, ab);
     }
     if (p.do_layer) {  // collapse with the carried pre (identity pre-mix for the broadcast)
       float2 sq = make_float2(0.f, 0.f);
@@ -1270,27 +1295,30 @@ mhc_status mhc_workspace_init(void* workspace, size_t ws_bytes, mhc_stream strea
   return MHC_OK;
 }
 
-mhc_status mhc_boundary_post_pre(const mhc_bf16* partials, int num_partials, int64_t partial_stride,
-                                 const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
-                                 const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
-                                 mhc_bf16* residual_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
-                                 float* post_out, float* comb_out, float* pre_out, int rows, int hidden,
-                                 int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream) {
-  if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
-  if (num_partials < 1 || num_partials > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
-  if (!partials || !aligned(partials, 16) || partial_stride % 8 != 0) return MHC_ERR_INVALID_ARG;
-  if (num_partials > 1 && partial_stride == 0) return MHC_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// mhc_boundary_post_pre over a table of partial pointers (checked by the callers).
+mhc_status post_pre_impl(const __nv_bfloat16* const* pptr, int num_partials, bool remote, const mhc_bf16* residual,
+                         const float* post, const float* comb, const float* pre, const mhc_bf16* norm_weight,
+                         float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out, mhc_bf16* aux_out,
+                         mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out,
+                         float* pre_out, int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
+                         mhc_stream stream) {
   mhc_status st = check_mixes(residual, post, comb, residual_out);
   if (st != MHC_OK) return st;
   Params p{};
-  p.partials = reinterpret_cast<const __nv_bfloat16*>(partials);
-  p.pstride = partial_stride;
+  for (int u = 0; u < num_partials; ++u) p.pptr[u] = pptr[u];
+  p.premote = remote ? 1 : 0;
   p.P = num_partials;
   p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
   p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
   p.write_res = 1;
+  if (aux_out && !aligned(aux_out, 16)) return MHC_ERR_INVALID_ARG;
+  p.aux_out = reinterpret_cast<__nv_bfloat16*>(aux_out);
   p.R = rows;
   p.H = hidden;
   st = fill_tail(p, pre, norm_weight, norm_eps, coeffs, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
@@ -1299,12 +1327,56 @@ mhc_status mhc_boundary_post_pre(const mhc_bf16* partials, int num_partials, int
   return dispatch_n<kPartials>(p, hc_mult, stream);
 }
 
+}  // namespace
+
+extern "C" {
+
+mhc_status mhc_boundary_post_pre(const mhc_bf16* partials, int num_partials, int64_t partial_stride,
+                                 const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
+                                 const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+                                 mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input,
+                                 const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out, float* pre_out,
+                                 int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
+                                 mhc_stream stream) {
+  if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (num_partials < 1 || num_partials > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (!partials || !aligned(partials, 16) || partial_stride % 8 != 0) return MHC_ERR_INVALID_ARG;
+  if (num_partials > 1 && partial_stride == 0) return MHC_ERR_INVALID_ARG;
+  const __nv_bfloat16* pptr[kMaxPartials];
+  for (int u = 0; u < num_partials; ++u)
+    pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials) + static_cast<int64_t>(u) * partial_stride;
+  return post_pre_impl(pptr, num_partials, false, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                       residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult,
+                       workspace, ws_bytes, stream);
+}
+
+mhc_status mhc_boundary_post_pre_ptrs(const mhc_bf16* const* partials, int num_partials, const mhc_bf16* residual,
+                                      const float* post, const float* comb, const float* pre,
+                                      const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+                                      mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input,
+                                      const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out,
+                                      float* pre_out, int rows, int hidden, int hc_mult, void* workspace,
+                                      size_t ws_bytes, mhc_stream stream) {
+  if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (num_partials < 1 || num_partials > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (!partials) return MHC_ERR_INVALID_ARG;
+  const __nv_bfloat16* pptr[kMaxPartials];
+  for (int u = 0; u < num_partials; ++u) {
+    if (!partials[u] || !aligned(partials[u], 16)) return MHC_ERR_INVALID_ARG;
+    pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials[u]);
+  }
+  return post_pre_impl(pptr, num_partials, true, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                       residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult,
+                       workspace, ws_bytes, stream);
+}
+
 mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_permuted, const float* expert_weights,
                                      const int32_t* expanded_idx_to_permuted_idx, int top_k,
                                      const mhc_bf16* shared_output, const mhc_bf16* residual, const float* post,
                                      const float* comb, const float* pre, const mhc_bf16* norm_weight,
                                      float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out,
-                                     mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out,
+                                     mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+                                     float* post_out,
                                      float* comb_out, float* pre_out, int rows, int hidden, int hc_mult,
                                      void* workspace, size_t ws_bytes, mhc_stream stream) {
   if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
@@ -1328,6 +1400,8 @@ mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_per
   p.comb = comb;
   p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
   p.write_res = 1;
+  if (aux_out && !aligned(aux_out, 16)) return MHC_ERR_INVALID_ARG;
+  p.aux_out = reinterpret_cast<__nv_bfloat16*>(aux_out);
   p.R = rows;
   p.H = hidden;
   // the MoE routing of every row is staged in shared memory; the residual-only
@@ -1344,8 +1418,8 @@ mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_per
 
 mhc_status mhc_boundary_residual_only(const mhc_bf16* partials, int num_partials, int64_t partial_stride,
                                       const mhc_bf16* residual, const float* post, const float* comb,
-                                      mhc_bf16* residual_out, int rows, int hidden, int hc_mult,
-                                      mhc_stream stream) {
+                                      mhc_bf16* residual_out, mhc_bf16* aux_out, int rows, int hidden,
+                                      int hc_mult, mhc_stream stream) {
   if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (num_partials < 1 || num_partials > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!partials || !aligned(partials, 16) || partial_stride % 8 != 0) return MHC_ERR_INVALID_ARG;
@@ -1353,14 +1427,16 @@ mhc_status mhc_boundary_residual_only(const mhc_bf16* partials, int num_partials
   mhc_status st = check_mixes(residual, post, comb, residual_out);
   if (st != MHC_OK) return st;
   Params p{};
-  p.partials = reinterpret_cast<const __nv_bfloat16*>(partials);
-  p.pstride = partial_stride;
+  for (int u = 0; u < num_partials; ++u)
+    p.pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials) + static_cast<int64_t>(u) * partial_stride;
   p.P = num_partials;
   p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
   p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
   p.write_res = 1;
+  if (aux_out && !aligned(aux_out, 16)) return MHC_ERR_INVALID_ARG;
+  p.aux_out = reinterpret_cast<__nv_bfloat16*>(aux_out);
   p.R = rows;
   p.H = hidden;
   return dispatch_n<kPartials>(p, hc_mult, stream);
@@ -1476,6 +1552,92 @@ mhc_status mhc_projection_pack(const float* fn, void* packed, int hidden, int hc
   return MHC_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Exported handle: the CUDA IPC handle of the allocation that holds the
+// pointer, then the pointer's byte offset into it.
+struct IpcHandle {
+  cudaIpcMemHandle_t mem;
+  uint64_t offset;
+};
+
+// Base of the allocation holding p (the IPC handle covers a whole allocation),
+// through the driver's cuMemGetAddressRange, looked up once.
+bool allocation_base(const void* p, uintptr_t* base) {
+  typedef int (*GetRange)(uintptr_t*, size_t*, uintptr_t);
+  static GetRange fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetRange>(f);
+  });
+  if (fn == nullptr) return false;
+  size_t size = 0;
+  return fn(base, &size, reinterpret_cast<uintptr_t>(p)) == 0;
+}
+
+std::mutex g_ipc_mu;
+std::map<uintptr_t, uintptr_t> g_ipc_open;  // pointer handed out -> mapped base
+
+}  // namespace
+
+extern "C" {
+
+size_t mhc_ipc_handle_bytes(void) { return sizeof(IpcHandle); }
+
+mhc_status mhc_ipc_export(const void* dev_ptr, void* handle_out) {
+  if (!dev_ptr || !handle_out) return MHC_ERR_INVALID_ARG;
+  uintptr_t base = 0;
+  if (!allocation_base(dev_ptr, &base)) return MHC_ERR_CUDA;
+  IpcHandle h{};
+  if (cudaIpcGetMemHandle(&h.mem, reinterpret_cast<void*>(base)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MHC_ERR_CUDA;
+  }
+  h.offset = reinterpret_cast<uintptr_t>(dev_ptr) - base;
+  std::memcpy(handle_out, &h, sizeof(h));
+  return MHC_OK;
+}
+
+mhc_status mhc_ipc_import(const void* handle, void** dev_ptr_out) {
+  if (!handle || !dev_ptr_out) return MHC_ERR_INVALID_ARG;
+  IpcHandle h;
+  std::memcpy(&h, handle, sizeof(h));
+  void* base = nullptr;
+  if (cudaIpcOpenMemHandle(&base, h.mem, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MHC_ERR_CUDA;
+  }
+  const uintptr_t ptr = reinterpret_cast<uintptr_t>(base) + h.offset;
+  {
+    std::lock_guard<std::mutex> lock(g_ipc_mu);
+    g_ipc_open[ptr] = reinterpret_cast<uintptr_t>(base);
+  }
+  *dev_ptr_out = reinterpret_cast<void*>(ptr);
+  return MHC_OK;
+}
+
+mhc_status mhc_ipc_release(void* dev_ptr) {
+  uintptr_t base = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_ipc_mu);
+    auto it = g_ipc_open.find(reinterpret_cast<uintptr_t>(dev_ptr));
+    if (it == g_ipc_open.end()) return MHC_ERR_INVALID_ARG;
+    base = it->second;
+    g_ipc_open.erase(it);
+  }
+  if (cudaIpcCloseMemHandle(reinterpret_cast<void*>(base)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MHC_ERR_CUDA;
+  }
+  return MHC_OK;
+}
+
 mhc_status mhc_get_device_status(void* workspace, mhc_stream stream) {
   if (!workspace || !aligned(workspace, 256)) return MHC_ERR_WORKSPACE;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MHC_ERR_CUDA;
@@ -1558,9 +1720,9 @@ mhc_status mhc_boundary_post_pre_noalloc(const mhc_bf16* partials, int num_parti
                                          const mhc_bf16* residual, const float* post, const float* comb,
                                          const float* pre, const mhc_bf16* norm_weight, float norm_eps,
                                          const mhc_coeff_args* coeffs, mhc_bf16* residual_out,
-                                         mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out,
-                                         float* comb_out, float* pre_out, int rows, int hidden, int hc_mult,
-                                         mhc_stream stream) {
+                                         mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
+                                         float* post_out, float* comb_out, float* pre_out, int rows, int hidden,
+                                         int hc_mult, mhc_stream stream) {
   if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (rows > kNoAllocMaxRows || hidden > kNoAllocMaxHidden || hc_mult > kNoAllocMaxHc ||
       ws_layout(rows, hidden, hc_mult, nullptr, nullptr) > kNoAllocBytes)
@@ -1568,8 +1730,8 @@ mhc_status mhc_boundary_post_pre_noalloc(const mhc_bf16* partials, int num_parti
   void* ws = noalloc_scratch();
   if (ws == nullptr) return MHC_ERR_CUDA;
   return mhc_boundary_post_pre(partials, num_partials, partial_stride, residual, post, comb, pre, norm_weight,
-                               norm_eps, coeffs, residual_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
-                               hidden, hc_mult, ws, kNoAllocBytes, stream);
+                               norm_eps, coeffs, residual_out, aux_out, layer_input, mxfp8, post_out, comb_out,
+                               pre_out, rows, hidden, hc_mult, ws, kNoAllocBytes, stream);
 }
 
 }  // extern "C"

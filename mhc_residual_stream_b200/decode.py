@@ -5,9 +5,12 @@ SpecializedDecode.run, with the sublayers (attention, MoE) replaced by seeded
 synthetic outputs: per layer the attention entry (the first layer's broadcast,
 else the finalize of the previous MoE output with an MXFP8 layer input), the
 attention's TP-partial output, the FFN entry (the partial sum, bf16 layer
-input) and the MoE's unfinalized output; after the last layer the
-residual-only finalize that feeds the final collapse. The streams and the
-post / comb / pre mixes chain from boundary to boundary as in BoundaryState.
+input) and the MoE's unfinalized output; after the last layer the finalize
+that, fused with the step's head (SpecializedDecode._head: the final norm of the
+streams collapsed with the carried pre), gives the step's hidden state. Layers
+in `aux_layers` keep the mean of their new streams (capture_aux), the end layer
+after the last finalize. The streams and the post / comb / pre mixes chain from
+boundary to boundary as in BoundaryState.
 
 Every boundary has its own seeded fn, scale, base and norm_weight, so the
 weights a step reads exceed the L2 cache and come from HBM.
@@ -16,7 +19,7 @@ weights a step reads exceed the L2 cache and come from HBM.
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from typing import List, Optional
+from typing import Dict, List, Optional, Tuple
 
 import torch
 
@@ -63,6 +66,9 @@ class DecodeLoop:
     seed: int = 5000
     device: str = "cuda"
     pack_fn: bool = True  # fn packed once at weight load (mhc_projection_pack)
+    # layers whose hidden state (the stream mean) is kept; `layers` itself is the
+    # end layer, captured after the last finalize. None: layers 2, L/2, L-3 and L.
+    aux_layers: Optional[Tuple[int, ...]] = None
     steps: List[Step] = field(default_factory=list)
 
     def __post_init__(self):
@@ -79,6 +85,14 @@ class DecodeLoop:
         self.q_data = torch.empty(R, H, dtype=torch.uint8, device=dev)
         self.q_scale = torch.empty(M.mhc_mxfp8_scale_bytes(R, H, True), dtype=torch.uint8, device=dev)
         self.workspace = M.new_workspace(R, H, n, dev)
+        if self.aux_layers is None:
+            self.aux_layers = tuple(sorted({l for l in (2, self.layers // 2, self.layers - 3, self.layers)
+                                            if 1 <= l <= self.layers}))
+        self.aux: Dict[int, torch.Tensor] = {l: torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+                                             for l in self.aux_layers}
+        self.hidden_out = torch.empty(R, H, dtype=torch.bfloat16, device=dev)  # the step's output
+        g = S.gen(s0 + 7)
+        self.final_norm = (1.0 + torch.randn(H, generator=g) * 0.1).to(torch.bfloat16).to(dev)
 
         def weights(seed):
             g = S.gen(seed)
@@ -126,22 +140,36 @@ class DecodeLoop:
                          layer_input=self.layer_input, workspace=ws, stream=stream)
             return
         a, b = st.src, st.dst
-        final = st.kind == "final"
-        w = st.weights
+        aux = self.aux_of(st)
         q = (self.q_data, self.q_scale, True) if st.mxfp8 else None
+        if st.kind == "final":  # the last finalize fused with the head: no coefficients
+            pd = st.pending
+            M.mhc_boundary_moe_finalize(
+                pd.gemm2_permuted, pd.expert_weights, pd.e2p, pd.shared_output, self.res[a], self.post[a],
+                self.comb[a], self.pre[a], self.final_norm, 1e-6, None, self.res[b], layer_input=self.hidden_out,
+                workspace=ws, stream=stream, aux=aux)
+            return
+        w = st.weights
         if st.pending.kind == "partials":
             M.mhc_boundary_post_pre(st.pending.partials, self.res[a], self.post[a], self.comb[a], self.pre[a],
                                     w.norm_weight, 1e-6, w.coeffs, self.res[b], layer_input=self.layer_input,
                                     mxfp8=q, post_out=self.post[b], comb_out=self.comb[b], pre_out=self.pre[b],
-                                    workspace=ws, stream=stream)
+                                    workspace=ws, stream=stream, aux=aux)
         else:
             pd = st.pending
             M.mhc_boundary_moe_finalize(
                 pd.gemm2_permuted, pd.expert_weights, pd.e2p, pd.shared_output, self.res[a], self.post[a],
-                self.comb[a], None if final else self.pre[a], None if final else w.norm_weight, 1e-6,
-                None if final else w.coeffs, self.res[b], layer_input=None if final else self.layer_input,
-                mxfp8=q, post_out=None if final else self.post[b], comb_out=None if final else self.comb[b],
-                pre_out=None if final else self.pre[b], workspace=ws, stream=stream)
+                self.comb[a], self.pre[a], w.norm_weight, 1e-6, w.coeffs, self.res[b],
+                layer_input=self.layer_input, mxfp8=q, post_out=self.post[b], comb_out=self.comb[b],
+                pre_out=self.pre[b], workspace=ws, stream=stream, aux=aux)
+
+    def aux_of(self, st: Step) -> Optional[torch.Tensor]:
+        """The aux buffer a boundary writes: the attention entry of a captured layer
+        (its new streams, [boundary] Boundaries.sublayer with capture_aux) or the
+        final finalize for the end layer."""
+        if st.kind in ("attn", "final") and st.layer in self.aux:
+            return self.aux[st.layer]
+        return None
 
     def run(self, stream=None):
         """Enqueue every boundary of the step on `stream` (no host synchronisation)."""
@@ -149,7 +177,7 @@ class DecodeLoop:
             self.run_step(st, stream)
 
     def streams(self) -> torch.Tensor:
-        """The residual streams after the final residual-only boundary."""
+        """The residual streams after the final boundary."""
         return self.res[self.final_slot]
 
     def algorithmic_bytes(self) -> int:
@@ -170,9 +198,12 @@ class DecodeLoop:
                 else:
                     b += (R * self.top_k + R) * H * 2 + R * self.top_k * 8
                 b += 2 * R * n * H * 2 + mix_in
+                b += R * H * 2 + H * 2  # layer input (the hidden state at the end) and its norm weight
                 if st.kind != "final":
-                    b += R * H * 2 + H * 2 + fn_b + coeff_out
+                    b += fn_b + coeff_out
                     if st.mxfp8:
                         b += R * H + M.mhc_mxfp8_scale_bytes(R, H, True)
+                if self.aux_of(st) is not None:
+                    b += R * H * 2
             total += b
         return total

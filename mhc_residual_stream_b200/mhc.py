@@ -92,18 +92,24 @@ def lib() -> ctypes.CDLL:
         "mhc_workspace_bytes": (_sz, [_i, _i, _i]),
         "mhc_mxfp8_scale_bytes": (_sz, [_i, _i, _i]),
         "mhc_workspace_init": (_i, [_vp, _sz, _vp]),
-        "mhc_boundary_post_pre": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp,
+        "mhc_boundary_post_pre": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
-        "mhc_boundary_post_pre_noalloc": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+        "mhc_boundary_post_pre_noalloc": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp,
                                                _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
         "mhc_boundary_moe_finalize": (_i, [_vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _f, _vp,
-                                           _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
-        "mhc_boundary_residual_only": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+        "mhc_boundary_residual_only": (_i, [_vp, _i, _i64, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
         "mhc_coeffs": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
         "mxfp8_quantize_rows": (_i, [_vp, _i, _i, _vp, _vp]),
         "mhc_get_device_status": (_i, [_vp, _vp]),
         "mhc_status_string": (ctypes.c_char_p, [_i]),
         "mhc_debug_set_wait": (_i64, [_i64, _i]),
+        "mhc_boundary_post_pre_ptrs": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
+                                            _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+        "mhc_ipc_handle_bytes": (_sz, []),
+        "mhc_ipc_export": (_i, [_vp, _vp]),
+        "mhc_ipc_import": (_i, [_vp, ctypes.POINTER(ctypes.c_void_p)]),
+        "mhc_ipc_release": (_i, [_vp]),
         "mhc_projection_pack_bytes": (_sz, [_i, _i]),
         "mhc_projection_pack": (_i, [_vp, _vp, _i, _i, _vp]),
     }
@@ -268,24 +274,76 @@ def _tail_args(pre, norm_weight, layer_input, post_out, comb_out, pre_out, R, n,
         _contig(t, n_)
 
 
+def _aux_arg(aux, R, H):
+    _need(aux, torch.bfloat16, "aux", 2)
+    _contig(aux, "aux")
+    if aux is not None and tuple(aux.shape) != (R, H):
+        raise ValueError(f"aux must be [{R}, {H}]")
+
+
 def mhc_boundary_post_pre(partials, residual, post, comb, pre, norm_weight, norm_eps, coeffs: Optional[Coeffs],
                           residual_out, layer_input=None, mxfp8=None, post_out=None, comb_out=None,
-                          pre_out=None, workspace=None, stream=None):
-    """Boundary after a partial-output sublayer. mxfp8 = (data, scale, swizzled) or None."""
+                          pre_out=None, workspace=None, stream=None, aux=None):
+    """Boundary after a partial-output sublayer. mxfp8 = (data, scale, swizzled) or None;
+    aux (optional, bf16 [R, H]) receives the mean of the new streams."""
     R, n, H = _mix_args(residual, post, comb, residual_out)
     P, stride = _partials_args(partials, R, H)
     _tail_args(pre, norm_weight, layer_input, post_out, comb_out, pre_out, R, n, H)
+    _aux_arg(aux, R, H)
     cs, qs = _coeff_struct(coeffs), _mxfp8_struct(mxfp8)
     st = lib().mhc_boundary_post_pre(
         _p(partials), P, stride, _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight), float(norm_eps),
-        _ref(cs), _p(residual_out), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
+        _ref(cs), _p(residual_out), _p(aux), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
         R, H, n, _p(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "mhc_boundary_post_pre")
 
 
+def mhc_boundary_post_pre_ptrs(partial_ptrs, residual, post, comb, pre, norm_weight, norm_eps,
+                               coeffs: Optional[Coeffs], residual_out, layer_input=None, mxfp8=None, post_out=None,
+                               comb_out=None, pre_out=None, workspace=None, stream=None, aux=None):
+    """mhc_boundary_post_pre with the partials as a list of device addresses (ints),
+    each a [R, H] bf16 partial that may live in another GPU's memory (the
+    tensor-parallel boundary; see PeerPartials in tp.py)."""
+    R, n, H = _mix_args(residual, post, comb, residual_out)
+    ptrs = [int(a) for a in partial_ptrs]
+    if not 1 <= len(ptrs) <= 16:
+        raise MhcError(UNSUPPORTED_SHAPE, "mhc_boundary_post_pre_ptrs")
+    _tail_args(pre, norm_weight, layer_input, post_out, comb_out, pre_out, R, n, H)
+    _aux_arg(aux, R, H)
+    table = (ctypes.c_void_p * len(ptrs))(*ptrs)
+    cs, qs = _coeff_struct(coeffs), _mxfp8_struct(mxfp8)
+    st = lib().mhc_boundary_post_pre_ptrs(
+        ctypes.cast(table, ctypes.c_void_p), len(ptrs), _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight),
+        float(norm_eps), _ref(cs), _p(residual_out), _p(aux), _p(layer_input), _ref(qs), _p(post_out),
+        _p(comb_out), _p(pre_out), R, H, n, _p(workspace), 0 if workspace is None else workspace.numel(),
+        _stream(stream))
+    _check(st, "mhc_boundary_post_pre_ptrs")
+
+
+def ipc_export(t: torch.Tensor) -> bytes:
+    """The handle another process passes to ipc_import to map t's memory."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("ipc_export needs a CUDA tensor")
+    buf = ctypes.create_string_buffer(int(lib().mhc_ipc_handle_bytes()))
+    _check(lib().mhc_ipc_export(_p(t), buf), "mhc_ipc_export")
+    return buf.raw
+
+
+def ipc_import(handle: bytes) -> int:
+    """Device address of memory another process exported (release with ipc_release)."""
+    out = ctypes.c_void_p()
+    _check(lib().mhc_ipc_import(ctypes.create_string_buffer(handle, len(handle)), ctypes.byref(out)),
+           "mhc_ipc_import")
+    return int(out.value)
+
+
+def ipc_release(addr: int):
+    _check(lib().mhc_ipc_release(ctypes.c_void_p(addr)), "mhc_ipc_release")
+
+
 def mhc_boundary_post_pre_noalloc(partials, residual, post, comb, pre, norm_weight, norm_eps,
                                   coeffs: Optional[Coeffs], residual_out, layer_input=None, mxfp8=None,
-                                  post_out=None, comb_out=None, pre_out=None, stream=None):
+                                  post_out=None, comb_out=None, pre_out=None, stream=None, aux=None):
     """mhc_boundary_post_pre without a workspace, for callers that cannot allocate
     device memory (a runtime that owns all memory, graph capture, allocation-free
     serving loops): the scratch is a fixed array inside the library. Limits:
@@ -294,10 +352,11 @@ def mhc_boundary_post_pre_noalloc(partials, residual, post, comb, pre, norm_weig
     R, n, H = _mix_args(residual, post, comb, residual_out)
     P, stride = _partials_args(partials, R, H)
     _tail_args(pre, norm_weight, layer_input, post_out, comb_out, pre_out, R, n, H)
+    _aux_arg(aux, R, H)
     cs, qs = _coeff_struct(coeffs), _mxfp8_struct(mxfp8)
     st = lib().mhc_boundary_post_pre_noalloc(
         _p(partials), P, stride, _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight), float(norm_eps),
-        _ref(cs), _p(residual_out), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
+        _ref(cs), _p(residual_out), _p(aux), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
         R, H, n, _stream(stream))
     _check(st, "mhc_boundary_post_pre_noalloc")
 
@@ -305,8 +364,8 @@ def mhc_boundary_post_pre_noalloc(partials, residual, post, comb, pre, norm_weig
 def mhc_boundary_moe_finalize(gemm2_permuted, expert_weights, expanded_idx_to_permuted_idx, shared_output,
                               residual, post, comb, pre, norm_weight, norm_eps, coeffs: Optional[Coeffs],
                               residual_out, layer_input=None, mxfp8=None, post_out=None, comb_out=None,
-                              pre_out=None, workspace=None, stream=None):
-    """Boundary after a MoE sublayer left unfinalized."""
+                              pre_out=None, workspace=None, stream=None, aux=None):
+    """Boundary after a MoE sublayer left unfinalized; aux as in mhc_boundary_post_pre."""
     R, n, H = _mix_args(residual, post, comb, residual_out)
     _need(gemm2_permuted, torch.bfloat16, "gemm2_permuted", 2)
     _need(expert_weights, torch.float32, "expert_weights", 2)
@@ -320,20 +379,22 @@ def mhc_boundary_moe_finalize(gemm2_permuted, expert_weights, expanded_idx_to_pe
             or expanded_idx_to_permuted_idx.numel() != R * k:
         raise ValueError("MoE finalize shapes disagree")
     _tail_args(pre, norm_weight, layer_input, post_out, comb_out, pre_out, R, n, H)
+    _aux_arg(aux, R, H)
     cs, qs = _coeff_struct(coeffs), _mxfp8_struct(mxfp8)
     st = lib().mhc_boundary_moe_finalize(
         _p(gemm2_permuted), gemm2_permuted.shape[0], _p(expert_weights), _p(expanded_idx_to_permuted_idx), k,
         _p(shared_output), _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight), float(norm_eps), _ref(cs),
-        _p(residual_out), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out), R, H, n,
+        _p(residual_out), _p(aux), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out), R, H, n,
         _p(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "mhc_boundary_moe_finalize")
 
 
-def mhc_boundary_residual_only(partials, residual, post, comb, residual_out, stream=None):
+def mhc_boundary_residual_only(partials, residual, post, comb, residual_out, stream=None, aux=None):
     R, n, H = _mix_args(residual, post, comb, residual_out)
     P, stride = _partials_args(partials, R, H)
+    _aux_arg(aux, R, H)
     st = lib().mhc_boundary_residual_only(_p(partials), P, stride, _p(residual), _p(post), _p(comb),
-                                          _p(residual_out), R, H, n, _stream(stream))
+                                          _p(residual_out), _p(aux), R, H, n, _stream(stream))
     _check(st, "mhc_boundary_residual_only")
 
 

@@ -1,0 +1,80 @@
+"""Tensor-parallel boundary: every rank of a TP group sums all ranks' partials
+itself, reading the peers' buffers with plain loads over NVLink.
+
+On the pages the sublayers' outputs are TP partials and the boundary's fused
+kernel does the all-reduce ([boundary] Boundaries.post_only:
+tensor_model_parallel_all_reduce then mhc_post; [all_reduce]
+BoundaryAllReduce.__call__, through a multicast mailbox). Here each rank
+exports its partial buffer once (CUDA IPC), maps every peer's, and passes the
+table of the group's buffers, in rank order, to mhc_boundary_post_pre_ptrs:
+one launch per rank reads the R x H partial of every rank and computes the
+whole boundary for every row (the result is the same on every rank, as after
+an all-reduce). Ordering is the caller's: the group's partials must be
+complete before the boundaries read them and must not be overwritten until all
+have read them (``barrier`` below is the plain host form of both). Nothing
+here uses multicast.
+"""
+
+from __future__ import annotations
+
+from typing import List, Optional
+
+import torch
+import torch.distributed as dist
+
+from . import mhc as M
+
+
+def exchange(handle: bytes, shape, group=None) -> List:
+    """Every rank's (handle, shape), in rank order; the shapes must agree."""
+    gathered: List = [None] * dist.get_world_size(group)
+    dist.all_gather_object(gathered, (handle, tuple(shape)), group=group)
+    for _, sh in gathered:
+        if tuple(sh) != tuple(shape):
+            raise ValueError(f"partial shapes differ across the group: {sh} vs {tuple(shape)}")
+    return gathered
+
+
+def partial_table(rank: int, local_ptr: int, gathered: List, import_fn):
+    """Device addresses of the group's partials in rank order: this rank's own
+    buffer, the peers' mapped through import_fn. Returns (table, imported)."""
+    table, imported = [], []
+    for r, (h, _) in enumerate(gathered):
+        if r == rank:
+            table.append(int(local_ptr))
+        else:
+            a = import_fn(h)
+            imported.append(a)
+            table.append(a)
+    return table, imported
+
+
+class PeerPartials:
+    """The group's partial buffers [R, H] bf16, one per rank, mapped on every rank."""
+
+    def __init__(self, local: torch.Tensor, group: Optional[dist.ProcessGroup] = None):
+        if not local.is_cuda or local.dtype != torch.bfloat16 or local.dim() != 2 or not local.is_contiguous():
+            raise ValueError("the local partial must be a contiguous bf16 [R, H] CUDA tensor")
+        self.local = local
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        gathered = exchange(M.ipc_export(local), tuple(local.shape), group)
+        self.ptrs, self._imported = partial_table(self.rank, local.data_ptr(), gathered, M.ipc_import)
+
+    def barrier(self):
+        """Host-side ordering of the group: all work queued on this device so far
+        is complete and every rank has reached this point."""
+        torch.cuda.current_stream(self.local.device).synchronize()
+        dist.barrier(group=self.group)
+
+    def close(self):
+        for a in self._imported:
+            M.ipc_release(a)
+        self._imported = []
+        self.ptrs = []
+
+    def boundary(self, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out, **kw):
+        """mhc_boundary_post_pre over the group's partials (all ranks, rank order)."""
+        M.mhc_boundary_post_pre_ptrs(self.ptrs, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                                     residual_out, **kw)

@@ -1,8 +1,9 @@
 """GPU parity of the decode step's layer loop: 61 layers, 123 chained boundaries
 (first-layer broadcast, MoE finalize + MXFP8 attention entries, partial-sum FFN
-entries, the final residual-only finalize), each checked against the oracle on
-the inputs the GPU actually fed it (stage-wise), plus a CUDA-graph replay of the
-whole step that must equal the eager run bit for bit."""
+entries, the final finalize fused with the head), each checked against the
+oracle on the inputs the GPU actually fed it (stage-wise), with the stream means
+of the captured layers, plus a CUDA-graph replay of the whole step that must
+equal the eager run bit for bit."""
 
 import numpy as np
 import pytest
@@ -25,6 +26,7 @@ def _coeff_np(c: M.Coeffs):
 def test_decode_loop_every_boundary_stage_wise():
     loop = DecodeLoop(rows=4, layers=61, device="cuda:0")
     assert len(loop.steps) == 123
+    assert loop.aux_layers == (2, 30, 58, 61)
     for st in loop.steps:
         a = st.src
         inp = {k: f64(getattr(loop, k)[a]) for k in ("res", "post", "comb", "pre")} if st.kind != "first" else {}
@@ -52,11 +54,17 @@ def test_decode_loop_every_boundary_stage_wise():
             kw["moe"] = dict(gemm2_permuted=f64(pd.gemm2_permuted), expert_weights=f64(pd.expert_weights),
                              expanded_idx_to_permuted_idx=pd.e2p.cpu().numpy().astype(np.int64),
                              shared_output=f64(pd.shared_output))
-        if not final:
-            kw.update(pre=inp["pre"], norm_weight=f64(st.weights.norm_weight), norm_eps=1e-6, mxfp8=st.mxfp8)
+        nw = f64(loop.final_norm) if final else f64(st.weights.norm_weight)
+        kw.update(pre=inp["pre"], norm_weight=nw, norm_eps=1e-6, mxfp8=st.mxfp8)
         o = O.boundary(**kw)
         assert_bf16_close(g_res, o["residual"], what + " streams")
-        if final:
+        aux = loop.aux_of(st)
+        if aux is not None:  # the stream mean of the streams the GPU wrote: exact
+            assert np.array_equal(f64(aux), O.stream_mean(g_res)), what + " aux"
+        if final:  # the step's hidden state: final norm of the collapse with the carried pre
+            g_h = f64(loop.hidden_out)
+            assert_bf16_close(g_h, o["layer_input"], what + " hidden (end to end)")
+            assert_bf16_close(g_h, O.final_head(g_res, inp["pre"], nw, 1e-6), what + " hidden (stage-wise)")
             continue
         g_li = f64(loop.layer_input)
         assert_bf16_close(g_li, o["layer_input"], what + " layer input")
@@ -75,6 +83,8 @@ def test_decode_loop_graph_replay_equals_eager():
     torch.cuda.synchronize()
     eager = loop.streams().clone()
     eager_pre = loop.pre[loop.steps[-2].dst].clone()
+    eager_hidden = loop.hidden_out.clone()
+    eager_aux = {k: v.clone() for k, v in loop.aux.items()}
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
@@ -87,3 +97,6 @@ def test_decode_loop_graph_replay_equals_eager():
     assert M.mhc_get_device_status(loop.workspace) == M.OK
     assert torch.equal(loop.streams(), eager)
     assert torch.equal(loop.pre[loop.steps[-2].dst], eager_pre)
+    assert torch.equal(loop.hidden_out, eager_hidden)
+    for k, v in eager_aux.items():
+        assert torch.equal(loop.aux[k], v), k

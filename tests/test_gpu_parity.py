@@ -305,6 +305,59 @@ def test_mxfp8_nonfinite_block():
     assert np.array_equal(scale.cpu().numpy(), osc.reshape(-1))
 
 
+# ---------------------------------------------------------------- aux stream mean
+
+@pytest.mark.parametrize("R,H,n", [(32, 7168, 4), (5, 192, 2), (3, 64, 1), (128, 512, 4)])
+def test_aux_stream_mean_on_every_front(R, H, n):
+    d = S.draw_boundary(R, H, n=n, partials=4, seed=5100 + R + n)
+    g = to_dev({k: d[k] for k in ("partials", "residual", "post", "comb", "pre", "norm_weight")})
+    orc = oracle_post_pre(d, mxfp8=False, coeff=False)
+    o_aux = O.stream_mean(orc["residual"])
+    runs = {}
+    # full boundary (no coefficients), the residual-only form, and the no-workspace entry
+    out, aux = alloc_outputs(R, n, H, False, True, False), torch.empty(R, H, dtype=torch.bfloat16, device=DEV)
+    M.mhc_boundary_post_pre(g["partials"], g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"],
+                            d["norm_eps"], None, out["residual_out"], layer_input=out["layer_input"],
+                            workspace=M.new_workspace(R, H, n, DEV), aux=aux)
+    runs["post_pre"] = (out["residual_out"], aux)
+    res2, aux2 = torch.empty_like(g["residual"]), torch.empty(R, H, dtype=torch.bfloat16, device=DEV)
+    M.mhc_boundary_residual_only(g["partials"], g["residual"], g["post"], g["comb"], res2, aux=aux2)
+    runs["residual_only"] = (res2, aux2)
+    if R <= 128 and H <= 7168 and n <= 4:
+        out3, aux3 = alloc_outputs(R, n, H, False, True, True), torch.empty(R, H, dtype=torch.bfloat16, device=DEV)
+        M.mhc_boundary_post_pre_noalloc(g["partials"], g["residual"], g["post"], g["comb"], g["pre"],
+                                        g["norm_weight"], d["norm_eps"], M.Coeffs.from_weights(d["coeff"], DEV),
+                                        out3["residual_out"], layer_input=out3["layer_input"], post_out=out3["post"],
+                                        comb_out=out3["comb"], pre_out=out3["pre"], aux=aux3)
+        runs["noalloc"] = (out3["residual_out"], aux3)
+    torch.cuda.synchronize()
+    for name, (res, ax) in runs.items():
+        g_res = f64(res.cpu())
+        # stage-wise exact: the mean of the streams the GPU wrote, rounded once
+        assert np.array_equal(f64(ax.cpu()), O.stream_mean(g_res)), name
+        assert_bf16_close(f64(ax.cpu()), o_aux, name + " aux (end to end)")
+
+
+def test_aux_stream_mean_moe_front_and_null_aux_writes_nothing():
+    d = S.draw_moe(16, 7168, n=4, top_k=8, seed=5216)
+    g = to_dev(d)
+    out = alloc_outputs(16, 4, 7168, False, True, True)
+    aux = torch.empty(16, 7168, dtype=torch.bfloat16, device=DEV)
+    ws = M.new_workspace(16, 7168, 4, DEV)
+    M.mhc_boundary_moe_finalize(
+        g["gemm2_permuted"], g["expert_weights"], g["expanded_idx_to_permuted_idx"], g["shared_output"],
+        g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"], d["norm_eps"],
+        M.Coeffs.from_weights(d["coeff"], DEV), out["residual_out"], layer_input=out["layer_input"],
+        post_out=out["post"], comb_out=out["comb"], pre_out=out["pre"], workspace=ws, aux=aux)
+    torch.cuda.synchronize()
+    assert M.mhc_get_device_status(ws) == M.OK
+    assert np.array_equal(f64(aux.cpu()), O.stream_mean(f64(out["residual_out"].cpu())))
+    # the same call without aux gives the same streams, layer input and coefficients
+    b, _ = _moe_gpu(d)
+    for k in ("residual_out", "layer_input", "post", "comb", "pre"):
+        assert torch.equal(out[k].cpu(), b[k]), k
+
+
 # ---------------------------------------------------------------- packed projection weights
 
 @pytest.mark.parametrize("R,H,n,P", [(1, 7168, 4, 8), (5, 192, 4, 3), (13, 320, 2, 16), (7, 64, 1, 2),

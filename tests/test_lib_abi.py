@@ -76,7 +76,7 @@ def test_host_checks_reject_before_launch(L):
     f = L.mhc_boundary_post_pre
     a = _fake()
     args = dict(partials=a, P=8, stride=32 * 256, residual=a, post=a, comb=a, pre=None, nw=None, eps=0.0,
-                coeffs=None, res_out=a, li=None, q=None, po=None, co=None, pr=None, R=32, H=256, n=4,
+                coeffs=None, res_out=a, aux=None, li=None, q=None, po=None, co=None, pr=None, R=32, H=256, n=4,
                 ws=None, wsb=0, s=None)
 
     def call(**kw):
@@ -108,12 +108,14 @@ def test_host_checks_reject_before_launch(L):
     assert call(pre=a, nw=a, li=a, ws=a, wsb=1 << 20, coeffs=ctypes.byref(ok_coeff)) == M.INVALID_ARG
     q = M.Mxfp8Out(0x10004, 0x10000, 1)  # data not 8-byte aligned
     assert call(pre=a, nw=a, li=a, ws=a, wsb=1 << 20, q=ctypes.byref(q)) == M.INVALID_ARG
+    assert call(aux=_fake(0x10008)) == M.INVALID_ARG  # aux not 16-byte aligned
 
 
 def test_other_entry_points_host_checks(L):
     a = _fake()
-    assert L.mhc_boundary_residual_only(a, 8, 0, a, a, a, a, 4, 256, 4, None) == M.INVALID_ARG  # stride 0, P > 1
-    assert L.mhc_boundary_residual_only(a, 1, 0, a, a, a, a, 4, 256, 5, None) == M.UNSUPPORTED_SHAPE
+    assert L.mhc_boundary_residual_only(a, 8, 0, a, a, a, a, None, 4, 256, 4, None) == M.INVALID_ARG  # stride 0
+    assert L.mhc_boundary_residual_only(a, 1, 0, a, a, a, a, None, 4, 256, 5, None) == M.UNSUPPORTED_SHAPE
+    assert L.mhc_boundary_residual_only(a, 1, 0, a, a, a, a, _fake(0x10004), 4, 256, 4, None) == M.INVALID_ARG
     c = M.CoeffArgs(0x10000, 0x10000, 0x10000, 1e-6, 1e-6, 1e-6, 2.0, 20)
     # both residual and x, or neither
     assert L.mhc_coeffs(a, ctypes.byref(c), None, a, None, None, 0.0, None, a, a, a, 4, 256, 4, a, 1 << 20, None) \
@@ -125,7 +127,7 @@ def test_other_entry_points_host_checks(L):
         == M.INVALID_ARG
     # finalize: top_k out of range
     assert L.mhc_boundary_moe_finalize(a, 64, a, a, 17, a, a, a, a, None, None, 0.0, None, a, None, None, None,
-                                       None, None, 4, 256, 4, a, 1 << 20, None) == M.UNSUPPORTED_SHAPE
+                                       None, None, None, 4, 256, 4, a, 1 << 20, None) == M.UNSUPPORTED_SHAPE
     q = M.Mxfp8Out(0x10000, 0x10000, 1)
     assert L.mxfp8_quantize_rows(a, 4, 48, ctypes.byref(q), None) == M.UNSUPPORTED_SHAPE
     assert L.mxfp8_quantize_rows(None, 4, 64, ctypes.byref(q), None) == M.INVALID_ARG
@@ -138,5 +140,24 @@ def test_other_entry_points_host_checks(L):
                 M.CoeffArgs(None, 0x10000, 0x10000, 1e-6, 1e-6, 1e-6, 2.0, 20, 0x10008)):
         assert L.mhc_coeffs(a, ctypes.byref(bad), None, None, None, None, 0.0, None, a, a, a, 4, 256, 4, a,
                             1 << 20, None) == M.INVALID_ARG
+    # the partial table: bad table, entries and counts are refused before any launch
+    res = dict(residual=a, post=a, comb=a)
+
+    def ptrs(table, n_parts, R=4, H=256, n=4):
+        t = None if table is None else ctypes.cast((ctypes.c_void_p * len(table))(*table), ctypes.c_void_p)
+        return L.mhc_boundary_post_pre_ptrs(t, n_parts, res["residual"], res["post"], res["comb"], None, None, 0.0,
+                                            None, a, None, None, None, None, None, None, R, H, n, None, 0, None)
+    assert ptrs(None, 2) == M.INVALID_ARG
+    assert ptrs([0x10000, None], 2) == M.INVALID_ARG
+    assert ptrs([0x10000, 0x10008], 2) == M.INVALID_ARG  # a partial not 16-byte aligned
+    assert ptrs([0x10000], 0) == M.UNSUPPORTED_SHAPE
+    assert ptrs([0x10000] * 17, 17) == M.UNSUPPORTED_SHAPE
+    assert ptrs([0x10000], 1, H=100) == M.UNSUPPORTED_SHAPE
+    # IPC helpers: argument checks only (no GPU here)
+    assert M.lib().mhc_ipc_handle_bytes() == 72
+    assert L.mhc_ipc_export(None, a) == M.INVALID_ARG
+    assert L.mhc_ipc_export(a, None) == M.INVALID_ARG
+    assert L.mhc_ipc_import(None, None) == M.INVALID_ARG
+    assert L.mhc_ipc_release(ctypes.c_void_p(0x12340)) == M.INVALID_ARG  # never imported
     assert L.mhc_workspace_init(None, 4096, None) == M.WORKSPACE
     assert L.mhc_get_device_status(None, None) == M.WORKSPACE

@@ -59,6 +59,6 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     a = ctypes.c_void_p(0x10000)
     # host-side size check, before any CUDA call: rows 64, hidden 9472 needs more
     # scratch than the fixed array (sized for hidden 7168) holds
-    st = L.mhc_boundary_post_pre_noalloc(a, 8, 64 * 9472, a, a, a, a, a, 1e-6, None, a, a, None, None, None,
+    st = L.mhc_boundary_post_pre_noalloc(a, 8, 64 * 9472, a, a, a, a, a, 1e-6, None, a, None, a, None, None, None,
                                          None, 64, 9472, 4, None)
     assert st == M.WORKSPACE
