@@ -36,8 +36,7 @@
  *   - Errors are returned, never raised or aborted on. Errors found by a kernel
  *     (a wait that ran out, a gather index out of range) are recorded in the
  *     workspace and read with mhc_get_device_status.
- *   - Shapes: 1 <= R <= 128, H a multiple of 64 with H/64 no larger than the
- *     number of co-resident blocks of the GPU (148 on B200, so H <= 9472),
+ *   - Shapes: 1 <= R <= 128, H a multiple of 64 with H/64 <= 148 (H <= 9472),
  *     n in {1, 2, 4}, 1 <= P <= 16, 1 <= k <= 16.
  *   - Alignment: bf16 tensors and fn 16-byte aligned, MXFP8 data 8-byte aligned,
  *     fp32 vectors 4-byte aligned; partial_stride a multiple of 8 elements.

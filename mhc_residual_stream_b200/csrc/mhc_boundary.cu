@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -1149,35 +1150,40 @@ mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const 
   return MHC_OK;
 }
 
-// Number of SMs of the current device (cached per device).
+// Number of SMs of the current device (cached per device; safe to call from
+// several host threads).
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kMaxBlocks;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return kMaxBlocks;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
-// Raise a kernel's dynamic shared memory limit once per device.
+// Raise a kernel's dynamic shared memory limit to 200 KB, once per device
+// (idempotent, so concurrent first calls only repeat the same setting).
+constexpr int kSmemLimit = 200 * 1024;
 template <typename Kern>
-bool allow_smem(Kern kern, int bytes, int* configured) {
+bool allow_smem(Kern kern, int bytes, std::atomic<int>* configured) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (dev >= 64 || configured[dev] >= bytes) return dev < 64;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+  if (bytes > kSmemLimit || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (configured[dev].load(std::memory_order_acquire) != 0) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess) {
+    (void)cudaGetLastError();
     return false;
-  configured[dev] = 200 * 1024;
+  }
+  configured[dev].store(1, std::memory_order_release);
   return true;
 }
 
 template <int N, int FRONT>
 mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
-  static int configured[64] = {0};
+  static std::atomic<int> configured[64];
   if (!allow_smem(boundary_kernel<N, FRONT>, L.total, configured)) return MHC_ERR_CUDA;
   p.extra_tx = g_extra_tx;
   p.budget_ns = g_budget_ns;
