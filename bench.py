@@ -306,9 +306,21 @@ def cpu_baseline(budget_s=12.0):
         if time.perf_counter() > t_end or len(times) >= 200:
             break
     us = statistics.median(times) * 1e6
+    one = []  # the same on one thread
+    with threadpoolctl.threadpool_limits(limits=1):
+        t_end = time.perf_counter() + budget_s / 2
+        while True:
+            t0 = time.perf_counter()
+            O.boundary(partials=f["partials"], residual=f["residual"], post=f["post"], comb=f["comb"],
+                       pre=f["pre"], norm_weight=f["norm_weight"], norm_eps=1e-6, coeff=cw, mxfp8=True,
+                       swizzled=True)
+            one.append(time.perf_counter() - t0)
+            if time.perf_counter() > t_end or len(one) >= 100:
+                break
     return {"value": round(us, 1), "unit": "µs/boundary", "cores": cores, "kind": "oracle",
+            "single_thread_value": round(statistics.median(one) * 1e6, 1),
             "sample": f"{len(times)} full boundaries (rows 32, H 7168, n 4, P 8, MXFP8, coefficients), median; "
-                      f"numpy float64, BLAS threads {cores}"}
+                      f"numpy float64, BLAS threads {cores}; single_thread_value: {len(one)} more on 1 thread"}
 
 
 def dist_setup(args):

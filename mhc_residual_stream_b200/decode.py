@@ -18,6 +18,7 @@ weights a step reads exceed the L2 cache and come from HBM.
 
 from __future__ import annotations
 
+from contextlib import nullcontext as _nullcontext
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional, Tuple
 
@@ -35,18 +36,19 @@ class BoundaryWeights:
 
 @dataclass
 class Pending:
-    kind: str  # "partials" or "moe"
+    kind: str  # "partials", "moe" or "engram" (the injection's stand-in: a delta added to the streams)
     partials: Optional[torch.Tensor] = None
     gemm2_permuted: Optional[torch.Tensor] = None
     expert_weights: Optional[torch.Tensor] = None
     e2p: Optional[torch.Tensor] = None
     shared_output: Optional[torch.Tensor] = None
+    delta: Optional[torch.Tensor] = None
 
 
 @dataclass
 class Step:
     """One boundary of the schedule."""
-    kind: str            # "first", "attn", "ffn", "final"
+    kind: str            # "first", "attn", "ffn", "post_only", "engram", "final"
     layer: int
     weights: Optional[BoundaryWeights]
     pending: Optional[Pending]
@@ -69,6 +71,10 @@ class DecodeLoop:
     # layers whose hidden state (the stream mean) is kept; `layers` itself is the
     # end layer, captured after the last finalize. None: layers 2, L/2, L-3 and L.
     aux_layers: Optional[Tuple[int, ...]] = None
+    # layers whose attention entry goes through an Engram injection ([decode]
+    # SpecializedDecode.run: post_only, the injection, then Boundaries.pre on
+    # the injected streams); the injection is a seeded delta (it needs weights)
+    engram_layers: Tuple[int, ...] = ()
     steps: List[Step] = field(default_factory=list)
 
     def __post_init__(self):
@@ -112,6 +118,10 @@ class DecodeLoop:
                            e2p=d["expanded_idx_to_permuted_idx"].to(dev),
                            shared_output=d["shared_output"].to(dev))
 
+        def engram_delta(seed):
+            g = S.gen(seed)
+            return Pending("engram", delta=(torch.randn(R, n, H, generator=g) * 0.05).to(torch.bfloat16).to(dev))
+
         steps = []
         slot = 0
         prev_moe = None
@@ -119,6 +129,12 @@ class DecodeLoop:
             base = s0 + 10 * (layer + 1)
             if layer == 0:
                 steps.append(Step("first", 0, weights(base + 1), None, False, src=0, dst=0))
+            elif layer in self.engram_layers:
+                # streams only, then the coefficients and layer input of the injected streams
+                steps.append(Step("post_only", layer, None, prev_moe, False, src=slot, dst=1 - slot))
+                steps.append(Step("engram", layer, weights(base + 1), engram_delta(base + 5), False,
+                                  src=slot, dst=1 - slot))
+                slot = 1 - slot
             else:
                 steps.append(Step("attn", layer, weights(base + 1), prev_moe, True, src=slot, dst=1 - slot))
                 slot = 1 - slot
@@ -142,6 +158,19 @@ class DecodeLoop:
         a, b = st.src, st.dst
         aux = self.aux_of(st)
         q = (self.q_data, self.q_scale, True) if st.mxfp8 else None
+        if st.kind == "post_only":  # the finalize into the streams, no layer input
+            pd = st.pending
+            M.mhc_boundary_moe_finalize(
+                pd.gemm2_permuted, pd.expert_weights, pd.e2p, pd.shared_output, self.res[a], self.post[a],
+                self.comb[a], None, None, 0.0, None, self.res[b], workspace=ws, stream=stream, aux=aux)
+            return
+        if st.kind == "engram":  # injected = streams + delta (stand-in), then mhc pre with the carried pre
+            with torch.cuda.stream(stream) if stream is not None else _nullcontext():
+                self.res[b].add_(st.pending.delta)
+            M.mhc_coeffs(st.weights.coeffs, self.post[b], self.comb[b], self.pre[b], residual=self.res[b],
+                         pre_mix=self.pre[a], norm_weight=st.weights.norm_weight, norm_eps=1e-6,
+                         layer_input=self.layer_input, workspace=ws, stream=stream)
+            return
         if st.kind == "final":  # the last finalize fused with the head: no coefficients
             pd = st.pending
             M.mhc_boundary_moe_finalize(
@@ -165,9 +194,10 @@ class DecodeLoop:
 
     def aux_of(self, st: Step) -> Optional[torch.Tensor]:
         """The aux buffer a boundary writes: the attention entry of a captured layer
-        (its new streams, [boundary] Boundaries.sublayer with capture_aux) or the
-        final finalize for the end layer."""
-        if st.kind in ("attn", "final") and st.layer in self.aux:
+        (its new streams, [boundary] Boundaries.sublayer with capture_aux; for an
+        Engram layer the streams before the injection) or the final finalize for
+        the end layer."""
+        if st.kind in ("attn", "post_only", "final") and st.layer in self.aux:
             return self.aux[st.layer]
         return None
 
@@ -192,6 +222,12 @@ class DecodeLoop:
             coeff_out = R * (2 * n + n * n) * 4
             if st.kind == "first":
                 b = R * H * 2 + R * n * H * 2 + R * H * 2 + fn_b + H * 2 + coeff_out
+            elif st.kind == "engram":  # the injection's add is the stand-in's, not counted
+                b = R * n * H * 2 + R * n * 4 + fn_b + H * 2 + R * H * 2 + coeff_out
+            elif st.kind == "post_only":
+                b = (R * self.top_k + R) * H * 2 + R * self.top_k * 8 + 2 * R * n * H * 2 + R * (n + n * n) * 4
+                if self.aux_of(st) is not None:
+                    b += R * H * 2
             else:
                 if st.pending.kind == "partials":
                     b += self.partials * R * H * 2

@@ -50,3 +50,32 @@ def test_algorithmic_bytes_by_kind():
     assert loop.algorithmic_bytes() == first + ffn + 2 * (attn + ffn) + final
     with_aux = _loop(rows=R, layers=3, aux_layers=(2, 3))
     assert with_aux.algorithmic_bytes() == loop.algorithmic_bytes() + 2 * R * H * 2
+
+
+def test_engram_layers_split_the_attention_entry():
+    loop = _loop(layers=6, engram_layers=(2, 4), aux_layers=(2, 3))
+    kinds = [(st.kind, st.layer) for st in loop.steps]
+    assert kinds == [("first", 0), ("ffn", 0), ("attn", 1), ("ffn", 1), ("post_only", 2), ("engram", 2), ("ffn", 2),
+                     ("attn", 3), ("ffn", 3), ("post_only", 4), ("engram", 4), ("ffn", 4), ("attn", 5), ("ffn", 5),
+                     ("final", 6)]
+    # the finalize and the injected streams' coefficients share the slot pair of one boundary
+    po, en = loop.steps[4], loop.steps[5]
+    assert (po.src, po.dst) == (en.src, en.dst)
+    for a, b in zip(loop.steps, loop.steps[1:]):
+        if b.kind != "engram":
+            assert b.src == a.dst
+    # an Engram layer captures the streams before the injection
+    assert loop.aux_of(po) is loop.aux[2] and loop.aux_of(en) is None
+    R, H, n = 4, 7168, 4
+    C = 2 * n + n * n
+    fn_b = n * H * C * 4 + (3 + C) * 4
+    plain = _loop(layers=6, aux_layers=())
+    eng = _loop(layers=6, engram_layers=(2,), aux_layers=())
+    attn2 = [st for st in plain.steps if st.kind == "attn" and st.layer == 2][0]
+    scales = ((R + 127) // 128 * 128) * ((H // 32 + 3) // 4 * 4)
+    moe_in = (R * 8 + R) * H * 2 + R * 8 * 8
+    attn_b = moe_in + 2 * R * n * H * 2 + R * C * 4 + R * H * 2 + H * 2 + fn_b + R * C * 4 + R * H + scales
+    split_b = (moe_in + 2 * R * n * H * 2 + R * (n + n * n) * 4) + (R * n * H * 2 + R * n * 4 + fn_b + H * 2
+                                                                     + R * H * 2 + R * C * 4)
+    assert attn2.mxfp8
+    assert eng.algorithmic_bytes() - plain.algorithmic_bytes() == split_b - attn_b

@@ -24,9 +24,17 @@ def _coeff_np(c: M.Coeffs):
 
 
 def test_decode_loop_every_boundary_stage_wise():
-    loop = DecodeLoop(rows=4, layers=61, device="cuda:0")
-    assert len(loop.steps) == 123
-    assert loop.aux_layers == (2, 30, 58, 61)
+    _check_loop(DecodeLoop(rows=4, layers=61, device="cuda:0"), 123)
+
+
+def test_decode_loop_with_engram_entries_stage_wise():
+    # Engram layers: streams only (with the captured mean), then the coefficients
+    # and layer input of the injected streams with the carried pre
+    _check_loop(DecodeLoop(rows=8, layers=8, device="cuda:0", engram_layers=(2, 5), aux_layers=(2, 5, 8)), 19)
+
+
+def _check_loop(loop, n_steps):
+    assert len(loop.steps) == n_steps
     for st in loop.steps:
         a = st.src
         inp = {k: f64(getattr(loop, k)[a]) for k in ("res", "post", "comb", "pre")} if st.kind != "first" else {}
@@ -36,6 +44,13 @@ def test_decode_loop_every_boundary_stage_wise():
         b = st.dst
         g_res = f64(loop.res[b])
         what = f"{st.kind} layer {st.layer}"
+        if st.kind == "engram":  # stage-wise on the injected streams the GPU held
+            o = O.coeffs_entry(residual=g_res, pre_mix=inp["pre"], norm_weight=f64(st.weights.norm_weight),
+                               norm_eps=1e-6, coeff=_coeff_np(st.weights.coeffs))
+            assert_bf16_close(f64(loop.layer_input), o["layer_input"], what + " layer input")
+            assert_coeffs_close({"post": loop.post[b].cpu(), "comb": loop.comb[b].cpu(), "pre": loop.pre[b].cpu()},
+                                o["post"], o["comb"], o["pre"], what)
+            continue
         if st.kind == "first":
             x = f64(loop.x)
             o = O.coeffs_entry(x=x, hc_mult=4, norm_weight=f64(st.weights.norm_weight), norm_eps=1e-6,
@@ -54,13 +69,16 @@ def test_decode_loop_every_boundary_stage_wise():
             kw["moe"] = dict(gemm2_permuted=f64(pd.gemm2_permuted), expert_weights=f64(pd.expert_weights),
                              expanded_idx_to_permuted_idx=pd.e2p.cpu().numpy().astype(np.int64),
                              shared_output=f64(pd.shared_output))
-        nw = f64(loop.final_norm) if final else f64(st.weights.norm_weight)
-        kw.update(pre=inp["pre"], norm_weight=nw, norm_eps=1e-6, mxfp8=st.mxfp8)
+        if st.kind != "post_only":
+            nw = f64(loop.final_norm) if final else f64(st.weights.norm_weight)
+            kw.update(pre=inp["pre"], norm_weight=nw, norm_eps=1e-6, mxfp8=st.mxfp8)
         o = O.boundary(**kw)
         assert_bf16_close(g_res, o["residual"], what + " streams")
         aux = loop.aux_of(st)
         if aux is not None:  # the stream mean of the streams the GPU wrote: exact
             assert np.array_equal(f64(aux), O.stream_mean(g_res)), what + " aux"
+        if st.kind == "post_only":
+            continue
         if final:  # the step's hidden state: final norm of the collapse with the carried pre
             g_h = f64(loop.hidden_out)
             assert_bf16_close(g_h, o["layer_input"], what + " hidden (end to end)")
