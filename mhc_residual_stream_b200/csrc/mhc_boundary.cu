@@ -8,7 +8,7 @@
 //      bf16 terms, or fp32 that the block splits into bf16 terms) and the
 //      block's activations are prefetched into L2, both before the kernel waits
 //      for its predecessor on the stream;
-//   2. per (row, 8 columns) a lane sums the partials (or finalizes the MoE
+//   2. per (row, 4 columns) a lane sums the partials (or finalizes the MoE
 //      output), applies the mHC post-mix (vllm ...boundary.boundary,
 //      Boundaries.post_only: mhc_post(x, residual, post, comb)), rounds the new
 //      streams to bf16, stores them, sums the squares of their collapse with the
@@ -173,9 +173,9 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ float sum8_lanes(float v) {  // over the 8 lanes sharing lane bits 3-4
+__device__ __forceinline__ float sum16_lanes(float v) {  // over the 16 lanes sharing lane bit 4
 #pragma unroll
-  for (int m = 4; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  for (int m = 8; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
   return v;
 }
 
@@ -222,45 +222,50 @@ __device__ __forceinline__ float tree_sum(const float (&v)[N]) {
   }
 }
 
-// Registers of one row-quad step of a lane: the stream vectors and up to 8
-// partial (or gathered) vectors, plus the shared-output / embedding vector.
+// Registers of one row-pair step of a lane (4 columns of one row): the stream
+// vectors and up to 8 partial (or gathered) vectors, plus the shared-output /
+// embedding vector.
 template <int N>
-struct QuadLoads {
-  uint4 rv[N];
-  uint4 pv[8];
-  uint4 sv;
+struct PairLoads {
+  uint2 rv[N];
+  uint2 pv[8];
+  uint2 sv;
 };
+// The streaming kernel runs 16 warps; a warp covers a row pair x 64 columns,
+// a lane 4 columns of one row.
+constexpr int kT1 = 512;
+constexpr int kW1 = kT1 / 32;
 
 template <int N, int FRONT>
-__device__ __forceinline__ void load_quad(const Params& p, int r, int h0, const int* e2p_s, QuadLoads<N>& Q) {
+__device__ __forceinline__ void load_pair(const Params& p, int r, int h0, const int* e2p_s, PairLoads<N>& Q) {
   const int H = p.H;
   if (r >= p.R) return;
   if constexpr (FRONT == kBroadcast) {
-    Q.sv = ld_nc_v4(p.x + static_cast<size_t>(r) * H + h0);
+    Q.sv = ld_nc_v2(p.x + static_cast<size_t>(r) * H + h0);
   } else {
 #pragma unroll
-    for (int j = 0; j < N; ++j) Q.rv[j] = ld_v4(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
+    for (int j = 0; j < N; ++j) Q.rv[j] = ld_v2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
   }
   if (FRONT == kPartials) {
     const size_t off = static_cast<size_t>(r) * H + h0;
     if (p.premote) {
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (u < p.P) Q.pv[u] = ld_v4(p.pptr[u] + off);
+        if (u < p.P) Q.pv[u] = ld_v2(p.pptr[u] + off);
     } else {
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (u < p.P) Q.pv[u] = ld_nc_v4(p.pptr[u] + off);
+        if (u < p.P) Q.pv[u] = ld_nc_v2(p.pptr[u] + off);
     }
   } else if (FRONT == kMoe) {
-    Q.sv = ld_nc_v4(p.shared_out + static_cast<size_t>(r) * H + h0);
+    Q.sv = ld_nc_v2(p.shared_out + static_cast<size_t>(r) * H + h0);
     const int* idx = e2p_s + r * p.topk;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (u < p.topk) {
         const int e = idx[u];
-        Q.pv[u] = (e >= 0 && e < p.num_perm) ? ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0)
-                                             : make_uint4(0, 0, 0, 0);
+        Q.pv[u] = (e >= 0 && e < p.num_perm) ? ld_nc_v2(p.gemm2 + static_cast<size_t>(e) * H + h0)
+                                             : make_uint2(0, 0);
       }
     }
   }
@@ -283,7 +288,9 @@ static_assert(packed_slice_bytes(1) % 16 == 0 && packed_slice_bytes(2) % 16 == 0
               "a bulk copy moves a multiple of 16 bytes");
 
 template <int N, int FRONT>
-__global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
+// 80 registers a thread: 512 threads leave room on the SM for the tail kernel's
+// blocks, which launch early (programmatic dependent launch).
+__global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   constexpr int C = logits_of(N);
   constexpr int KC = N * kCols;       // stream values per row in this block
   constexpr int KS = kstride_of(N);   // staged row stride (bf16)
@@ -308,11 +315,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   const int H = p.H;
   const int R = p.R;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rq = lane >> 3, vec = lane & 7;
-  const int h0 = g * kCols + vec * 8;  // this lane's 8 columns in the row-quad phase
+  const int rq = lane >> 4, vec = lane & 15;
+  const int h0 = g * kCols + vec * 4;  // this lane's 4 columns in the row-pair phase
   const long long deadline = wait_deadline(p.budget_ns);
   unsigned* status = p.ctl + kStatusWord;
-  const int nquads = (R + 3) >> 2;
+  const int npairs = (R + 1) >> 1;
 
   // ---- 1. the block's fn slice by TMA bulk copies. Weights are never written by
   // the kernel that precedes this one on the stream, so this runs before the
@@ -340,9 +347,9 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   // ---- 2. bring this block's activations into L2 while the preceding kernel may
   // still run: a prefetch is only a hint and L2 is the point of coherence, so
   // it is safe before the wait; gather indices read now only steer prefetches.
-  if (vec == 0 || vec == 7) {
-    for (int q = warp; q < nquads; q += kWarps) {
-      const int r = q * 4 + rq;
+  if (vec == 0 || vec == 15) {
+    for (int q = warp; q < npairs; q += kW1) {
+      const int r = q * 2 + rq;
       if (r >= R) break;
       if constexpr (FRONT == kBroadcast) {
         prefetch_l2(p.x + static_cast<size_t>(r) * H + h0);
@@ -369,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
     const bool ok = mbar_wait_bounded(bar, 0, deadline);
     if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
     if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
-    for (int e = tid; e < CP8 * KC; e += kThreads) {
+    for (int e = tid; e < CP8 * KC; e += kT1) {
       const int c = e / KC, k = e - c * KC;
       const float f = c < C ? reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4)[c] : 0.f;
       __nv_bfloat16 hi, mid, lo;
@@ -386,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
   // ---- 3. wait for the preceding kernel, let the next one launch, and read
   griddep_wait();
   griddep_launch_dependents();
-  for (int k = tid; k < R * MIX; k += kThreads) {  // [R][post n | comb n*n | pre n]
+  for (int k = tid; k < R * MIX; k += kT1) {  // [R][post n | comb n*n | pre n]
     const int r = k / MIX, c = k - r * MIX;
     if (c < N + N * N) {
       if (FRONT == kStreams || FRONT == kBroadcast) {
@@ -403,55 +410,55 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
     }
   }
   if (FRONT == kMoe) {
-    for (int k = tid; k < R * p.topk; k += kThreads) {
+    for (int k = tid; k < R * p.topk; k += kT1) {
       cp_async4(e2p_s + k, p.e2p + k);
       cp_async4(ew_s + k, p.ew + k);
     }
   }
-  QuadLoads<N> cur;
-  if (FRONT != kMoe && warp < nquads) load_quad<N, FRONT>(p, warp * 4 + rq, h0, e2p_s, cur);
+  PairLoads<N> cur;
+  if (FRONT != kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
   cp_async_wait_all();
   __syncthreads();
-  if (FRONT == kMoe && warp < nquads) load_quad<N, FRONT>(p, warp * 4 + rq, h0, e2p_s, cur);
+  if (FRONT == kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
 
-  // ---- 4. row quads: sum / finalize, post-mix, store the streams, sum c^2
-  for (int q = warp; q < nquads; q += kWarps) {
-    QuadLoads<N> nxt;
-    if (q + kWarps < nquads) load_quad<N, FRONT>(p, (q + kWarps) * 4 + rq, h0, e2p_s, nxt);
-    const int r = q * 4 + rq;
+  // ---- 4. row pairs: sum / finalize, post-mix, store the streams, sum c^2
+  for (int q = warp; q < npairs; q += kW1) {
+    PairLoads<N> nxt;
+    if (q + kW1 < npairs) load_pair<N, FRONT>(p, (q + kW1) * 2 + rq, h0, e2p_s, nxt);
+    const int r = q * 2 + rq;
     const bool valid = r < R;
     const float* mix = mix_s + (valid ? r : 0) * MIX;
     // Pairs of columns in packed f32x2 arithmetic (each element the same fp32
     // operations, in the same order, as one at a time).
-    float2 nf[N][4];  // the new streams, as rounded to bf16
-    uint4 nb[N];
-    float2 xs[4];
+    float2 nf[N][2];  // the new streams, as rounded to bf16
+    uint2 nb[N];
+    float2 xs[2];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) xs[t] = make_float2(0.f, 0.f);
+    for (int t = 0; t < 2; ++t) xs[t] = make_float2(0.f, 0.f);
     if (FRONT == kPartials || FRONT == kMoe) {
-      float2 rf[N][4];
+      float2 rf[N][2];
       if (valid) {
 #pragma unroll
-        for (int j = 0; j < N; ++j) unpack8x2(cur.rv[j], rf[j]);
+        for (int j = 0; j < N; ++j) unpack4x2(cur.rv[j], rf[j]);
         if (FRONT == kPartials) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             if (u < p.P) {
-              float2 f[4];
-              unpack8x2(cur.pv[u], f);
+              float2 f[2];
+              unpack4x2(cur.pv[u], f);
 #pragma unroll
-              for (int t = 0; t < 4; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
+              for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
             }
           }
           for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
-            float2 f[4];
+            float2 f[2];
             const __nv_bfloat16* src = p.pptr[u] + static_cast<size_t>(r) * H + h0;
-            unpack8x2(p.premote ? ld_v4(src) : ld_nc_v4(src), f);
+            unpack4x2(p.premote ? ld_v2(src) : ld_nc_v2(src), f);
 #pragma unroll
-            for (int t = 0; t < 4; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
+            for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
           }
         } else {
-          unpack8x2(cur.sv, xs);
+          unpack4x2(cur.sv, xs);
           const int* idx = e2p_s + r * p.topk;
           const float* wt = ew_s + r * p.topk;
 #pragma unroll
@@ -461,11 +468,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
               if (e >= p.num_perm) {
                 if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
               } else if (e >= 0) {
-                float2 f[4];
-                unpack8x2(cur.pv[u], f);
+                float2 f[2];
+                unpack4x2(cur.pv[u], f);
                 const float2 w2 = make_float2(wt[u], wt[u]);
 #pragma unroll
-                for (int t = 0; t < 4; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
+                for (int t = 0; t < 2; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
               }
             }
           }
@@ -474,11 +481,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
             if (e >= p.num_perm) {
               if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
             } else if (e >= 0) {
-              float2 f[4];
-              unpack8x2(ld_nc_v4(p.gemm2 + static_cast<size_t>(e) * H + h0), f);
+              float2 f[2];
+              unpack4x2(ld_nc_v2(p.gemm2 + static_cast<size_t>(e) * H + h0), f);
               const float2 w2 = make_float2(wt[u], wt[u]);
 #pragma unroll
-              for (int t = 0; t < 4; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
+              for (int t = 0; t < 2; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
             }
           }
         }
@@ -486,15 +493,15 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
 #pragma unroll
         for (int j = 0; j < N; ++j)
 #pragma unroll
-          for (int t = 0; t < 4; ++t) rf[j][t] = make_float2(0.f, 0.f);
+          for (int t = 0; t < 2; ++t) rf[j][t] = make_float2(0.f, 0.f);
       }
       // mHC post: new[i] = bf16(post[i] * x + sum_j comb[j][i] * res[j])
 #pragma unroll
       for (int i = 0; i < N; ++i) {
-        float2 a[4];
+        float2 a[2];
         const float2 po = make_float2(mix[i], mix[i]);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
+        for (int t = 0; t < 2; ++t) {
           float2 s2 = __fmul2_rn(po, xs[t]);
 #pragma unroll
           for (int j = 0; j < N; ++j) {
@@ -503,46 +510,47 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
           }
           a[t] = s2;
         }
-        nb[i] = round8x2(a, nf[i]);
+        nb[i] = make_uint2(pack_bf16x2(a[0].x, a[0].y), pack_bf16x2(a[1].x, a[1].y));
+        unpack4x2(nb[i], nf[i]);
       }
     } else if (FRONT == kStreams) {
 #pragma unroll
       for (int j = 0; j < N; ++j) {
-        nb[j] = valid ? cur.rv[j] : make_uint4(0, 0, 0, 0);
-        unpack8x2(nb[j], nf[j]);
+        nb[j] = valid ? cur.rv[j] : make_uint2(0, 0);
+        unpack4x2(nb[j], nf[j]);
       }
     } else {  // kBroadcast: every stream is the embedding row
-      const uint4 xv = valid ? cur.sv : make_uint4(0, 0, 0, 0);
-      unpack8x2(xv, xs);
+      const uint2 xv = valid ? cur.sv : make_uint2(0, 0);
+      unpack4x2(xv, xs);
 #pragma unroll
       for (int j = 0; j < N; ++j) {
         nb[j] = xv;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) nf[j][t] = xs[t];
+        for (int t = 0; t < 2; ++t) nf[j][t] = xs[t];
       }
     }
     if (p.write_res && valid) {
 #pragma unroll
-      for (int i = 0; i < N; ++i) st_v4(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
+      for (int i = 0; i < N; ++i) st_v2(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
     }
     if (p.aux_out != nullptr && valid) {  // mean over the streams, in stream order, rounded once
       constexpr float kInvN = 1.f / N;    // exact: n is a power of two
-      uint4 ab;
+      uint2 ab;
       unsigned* aw = reinterpret_cast<unsigned*>(&ab);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
+      for (int t = 0; t < 2; ++t) {
         float2 m = nf[0][t];
 #pragma unroll
         for (int j = 1; j < N; ++j) m = __fadd2_rn(m, nf[j][t]);
         m = __fmul2_rn(m, make_float2(kInvN, kInvN));
         aw[t] = pack_bf16x2(m.x, m.y);
       }
-      st_v4(p.aux_out + static_cast<size_t>(r) * H + h0, ab);
+      st_v2(p.aux_out + static_cast<size_t>(r) * H + h0, ab);
     }
     if (p.do_layer) {  // collapse with the carried pre (identity pre-mix for the broadcast)
       float2 sq = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
+      for (int t = 0; t < 2; ++t) {
         float2 c;
         if (FRONT == kBroadcast) {
           c = xs[t];
@@ -556,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
         }
         sq = __ffma2_rn(c, c, sq);
       }
-      const float sc2 = sum8_lanes(sq.x + sq.y);
+      const float sc2 = sum16_lanes(sq.x + sq.y);
       if (valid && vec == 0) p.sc2_part[r * G + g] = sc2;
     }
     if (p.do_coeff) {  // stage the streams for the projection; sum v^2 of the row
@@ -564,11 +572,11 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
 #pragma unroll
       for (int i = 0; i < N; ++i)
 #pragma unroll
-        for (int t = 0; t < 4; ++t) sv = __ffma2_rn(nf[i][t], nf[i][t], sv);
-      const float sv2 = sum8_lanes(sv.x + sv.y);
+        for (int t = 0; t < 2; ++t) sv = __ffma2_rn(nf[i][t], nf[i][t], sv);
+      const float sv2 = sum16_lanes(sv.x + sv.y);
       if (valid) {
 #pragma unroll
-        for (int i = 0; i < N; ++i) *reinterpret_cast<uint4*>(v_s + r * KS + i * kCols + vec * 8) = nb[i];
+        for (int i = 0; i < N; ++i) *reinterpret_cast<uint2*>(v_s + r * KS + i * kCols + vec * 4) = nb[i];
         if (vec == 0) p.dot_part[(static_cast<size_t>(r) * G + g) * RED + C] = sv2;
       }
     }
@@ -597,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.f;
     const bool two = rb + 16 < R;  // second 16-row tile of the chunk in use
-    for (int kstep = warp; kstep < KC / 16; kstep += kWarps) {
+    for (int kstep = warp; warp < kWarps && kstep < KC / 16; kstep += kWarps) {  // warps 0-7
       const int k0 = kstep * 16;
       unsigned a[2][4];
       ldmatrix_x4(a[0], v_s + (rb + (lane & 15)) * KS + k0 + (lane >> 4) * 8);
@@ -615,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
     }
     // C fragment: lane holds rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < 2 && warp < kWarps; ++mt)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int row = mt * 16 + (lane >> 2), col = nt * 8 + 2 * (lane & 3);
@@ -626,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_kernel(const Params p) {
         dst[8 * CP8 + 1] = acc[mt][nt][3];
       }
     __syncthreads();
-    for (int e = tid; e < 32 * C; e += kThreads) {
+    for (int e = tid; e < 32 * C; e += kT1) {
       const int row = e / C, col = e - row * C, r = rb + row;
       if (r < R) {
         float sum = 0.f;
@@ -1132,10 +1140,10 @@ mhc_status check_mxfp8(const mhc_mxfp8_out* q) {
 // preceding kernel on the stream finishes, and waits for it (griddepcontrol.wait)
 // before reading anything that kernel may have written.
 template <typename Kern>
-mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const Params& p) {
+mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const Params& p, int threads = kThreads) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1188,7 +1196,7 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   p.extra_tx = g_extra_tx;
   p.budget_ns = g_budget_ns;
   const int G = p.H / kCols;
-  mhc_status st = launch_pdl(boundary_kernel<N, FRONT>, G, L.total, stream, p);
+  mhc_status st = launch_pdl(boundary_kernel<N, FRONT>, G, L.total, stream, p, kT1);
   if (st != MHC_OK || !(p.do_layer || p.do_coeff)) return st;
   if (FRONT == kBroadcast) {
     p.tail_streams = p.x;

@@ -106,6 +106,25 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {  // read-only, stream
   return v;
 }
 
+// 8-byte forms (4 bf16): the streaming kernel's lanes own 4 columns.
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint2 ld_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void st_v2(void* p, uint2 v) {
+  asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+// 4 bf16 as two column pairs: f[m] = (element 2m, element 2m + 1).
+__device__ __forceinline__ void unpack4x2(const uint2 v, float2 (&f)[2]) {
+  f[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
+  f[1] = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+}
 __device__ __forceinline__ uint4 ld_v4(const void* p) {  // coherent (may alias an output)
   uint4 v;
   asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -157,13 +176,6 @@ __device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8]) {
   }
 }
 
-// The same as column pairs: f[m] = (element 2m, element 2m + 1).
-__device__ __forceinline__ void unpack8x2(const uint4 v, float2 (&f)[4]) {
-  const unsigned w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int m = 0; m < 4; ++m) f[m] = make_float2(__uint_as_float(w[m] << 16), __uint_as_float(w[m] & 0xffff0000u));
-}
-
 __device__ __forceinline__ unsigned pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<unsigned*>(&b);
@@ -177,16 +189,6 @@ __device__ __forceinline__ uint4 round8(const float (&f)[8], float (&r)[8]) {
   v.z = pack_bf16x2(f[4], f[5]);
   v.w = pack_bf16x2(f[6], f[7]);
   unpack8(v, r);
-  return v;
-}
-
-__device__ __forceinline__ uint4 round8x2(const float2 (&f)[4], float2 (&r)[4]) {
-  uint4 v;
-  v.x = pack_bf16x2(f[0].x, f[0].y);
-  v.y = pack_bf16x2(f[1].x, f[1].y);
-  v.z = pack_bf16x2(f[2].x, f[2].y);
-  v.w = pack_bf16x2(f[3].x, f[3].y);
-  unpack8x2(v, r);
   return v;
 }
 
