@@ -115,7 +115,7 @@ struct Params {
 };
 
 struct SmemLayout {
-  int fn_off, bs_off, v_off, mix_off, moe_off, red_off, misc_off, total;
+  int fn_off, bs_off, v_off, mix_off, moe_off, misc_off, total;
 };
 
 // Projection operands: n-tiles of 8 logit columns; staged stream rows and fn
@@ -123,14 +123,15 @@ struct SmemLayout {
 __host__ __device__ constexpr int ntiles_of(int n) { return (logits_of(n) + 7) / 8; }
 __host__ __device__ constexpr int kstride_of(int n) { return n * kCols + 8; }
 
-// Shared memory of the streaming kernel.
+// Shared memory of the streaming kernel (packed: fn arrives already split, so
+// the fp32 staging area is not needed).
 template <int N>
-__host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe) {
+__host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe, bool packed) {
   constexpr int CP8 = ntiles_of(N) * 8;
   SmemLayout L{};
   int o = 0;
   L.fn_off = o;  // fn slice as the bulk copies land it
-  o += N * 8 * fn_piece_bytes(N);
+  if (!packed) o += N * 8 * fn_piece_bytes(N);
   L.bs_off = o;  // fn slice as three bf16 terms, [3][CP8][n*64 + 8]
   o += 3 * CP8 * kstride_of(N) * 2;
   L.v_off = o;  // new streams, bf16 [roundup(R, 16)][n*64 + 8]
@@ -141,8 +142,6 @@ __host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe) {
   L.moe_off = o;
   if (moe) o += R * topk * 8;
   o = (o + 15) & ~15;
-  L.red_off = o;  // per-warp projection sums of a 32-row chunk, [8][32][CP8]
-  o += kWarps * 32 * CP8 * 4;
   L.misc_off = o;  // mbarrier
   o += 16;
   L.total = o;
@@ -300,14 +299,13 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   constexpr int MIX = 2 * N + N * N;
   constexpr int PIECE = fn_piece_bytes(N);
   extern __shared__ __align__(128) unsigned char smem[];
-  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
+  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe, p.fn_packed != nullptr);
   unsigned char* fn_s = smem + L.fn_off;
   __nv_bfloat16* bs_s = reinterpret_cast<__nv_bfloat16*>(smem + L.bs_off);
   __nv_bfloat16* v_s = reinterpret_cast<__nv_bfloat16*>(smem + L.v_off);
   float* mix_s = reinterpret_cast<float*>(smem + L.mix_off);
   int* e2p_s = reinterpret_cast<int*>(smem + L.moe_off);
   float* ew_s = reinterpret_cast<float*>(smem + L.moe_off) + p.R * p.topk;
-  float* red_s = reinterpret_cast<float*>(smem + L.red_off);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.misc_off);
 
   const int g = blockIdx.x;
@@ -586,9 +584,7 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
 
   // ---- 5. projection of this block's n*64 stream values per row onto the C fn
   // columns on the tensor cores: [rows x n*64] bf16 x [n*64 x C] as three bf16
-  // terms, fp32 accumulation (mma.sync m16n8k16). Warp w takes the k-steps
-  // w, w+8, ... of every 16-row tile and 8-column tile of a 32-row chunk; the
-  // warps' sums are added in warp order.
+  // terms, fp32 accumulation (mma.sync m16n8k16).
   if (packed) {  // the packed slice, copied before the wait, has surely landed by now
     const bool ok = mbar_wait_bounded(bar, 0, deadline);
     if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
@@ -596,54 +592,40 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   } else {
     __syncthreads();  // staged streams
   }
-  for (int rb = 0; rb < R; rb += 32) {
-    float acc[2][NT][4];
+  // Work items: (16-row tile, 8-column tile) of the block's rows x C logits. A
+  // warp takes items w, w + 16, ...; for its item it runs every k-step, with
+  // one accumulator per bf16 term of fn (three independent MMA chains), adds
+  // the terms and stores its rows' dot products itself: no cross-warp sums.
+  const int mtiles = (R + 15) >> 4;
+  for (int item = warp; item < mtiles * NT; item += kW1) {
+    const int mt = item / NT, nt = item - mt * NT;
+    float acc[3][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int sp = 0; sp < 3; ++sp)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int q = 0; q < 4; ++q) acc[sp][q] = 0.f;
+    const __nv_bfloat16* arow = v_s + (mt * 16 + (lane & 15)) * KS + (lane >> 4) * 8;
+    const __nv_bfloat16* brow = bs_s + (nt * 8 + (lane & 7)) * KS + ((lane >> 3) & 1) * 8;
+#pragma unroll 4
+    for (int k0 = 0; k0 < KC; k0 += 16) {
+      unsigned a[4], b[3][2];
+      ldmatrix_x4(a, arow + k0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.f;
-    const bool two = rb + 16 < R;  // second 16-row tile of the chunk in use
-    for (int kstep = warp; warp < kWarps && kstep < KC / 16; kstep += kWarps) {  // warps 0-7
-      const int k0 = kstep * 16;
-      unsigned a[2][4];
-      ldmatrix_x4(a[0], v_s + (rb + (lane & 15)) * KS + k0 + (lane >> 4) * 8);
-      if (two) ldmatrix_x4(a[1], v_s + (rb + 16 + (lane & 15)) * KS + k0 + (lane >> 4) * 8);
+      for (int sp = 0; sp < 3; ++sp) ldmatrix_x2(b[sp], brow + sp * CP8 * KS + k0);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int sp = 0; sp < 3; ++sp) {
-          unsigned b[2];
-          ldmatrix_x2(b, bs_s + (sp * CP8 + nt * 8 + (lane & 7)) * KS + k0 + ((lane >> 3) & 1) * 8);
-          mma_bf16_16816(acc[0][nt], a[0], b);
-          if (two) mma_bf16_16816(acc[1][nt], a[1], b);
-        }
-      }
+      for (int sp = 0; sp < 3; ++sp) mma_bf16_16816(acc[sp], a, b[sp]);
     }
     // C fragment: lane holds rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
+    const int col = nt * 8 + 2 * (lane & 3);
 #pragma unroll
-    for (int mt = 0; mt < 2 && warp < kWarps; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int row = mt * 16 + (lane >> 2), col = nt * 8 + 2 * (lane & 3);
-        float* dst = red_s + (warp * 32 + row) * CP8 + col;
-        dst[0] = acc[mt][nt][0];
-        dst[1] = acc[mt][nt][1];
-        dst[8 * CP8] = acc[mt][nt][2];
-        dst[8 * CP8 + 1] = acc[mt][nt][3];
-      }
-    __syncthreads();
-    for (int e = tid; e < 32 * C; e += kT1) {
-      const int row = e / C, col = e - row * C, r = rb + row;
-      if (r < R) {
-        float sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) sum += red_s[(w * 32 + row) * CP8 + col];
-        p.dot_part[(static_cast<size_t>(r) * G + g) * RED + col] = sum;
+    for (int h = 0; h < 2; ++h) {
+      const int r = mt * 16 + (lane >> 2) + 8 * h;
+      if (r < R && col < C) {
+        float* dst = p.dot_part + (static_cast<size_t>(r) * G + g) * RED + col;
+        dst[0] = (acc[0][2 * h] + acc[1][2 * h]) + acc[2][2 * h];
+        if (col + 1 < C) dst[1] = (acc[0][2 * h + 1] + acc[1][2 * h + 1]) + acc[2][2 * h + 1];
       }
     }
-    __syncthreads();
   }
 }
 
@@ -1190,7 +1172,7 @@ bool allow_smem(Kern kern, int bytes, std::atomic<int>* configured) {
 
 template <int N, int FRONT>
 mhc_status launch_boundary(Params& p, cudaStream_t stream) {
-  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe);
+  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe, p.fn_packed != nullptr);
   static std::atomic<int> configured[64];
   if (!allow_smem(boundary_kernel<N, FRONT>, L.total, configured)) return MHC_ERR_CUDA;
   p.extra_tx = g_extra_tx;
