@@ -19,7 +19,7 @@
 // The tail kernel (boundary_tail_kernel), once the streaming kernel is done:
 //   4. layer-input blocks normalise 256-column tasks of the rows into the layer
 //      input (and MXFP8); beside them, coefficient blocks finish the rows'
-//      coefficients (logits, sigmoid, Sinkhorn with one matrix entry per lane).
+//      coefficients (logits, sigmoid, Sinkhorn in one thread per row).
 // The residual-only variant is the streaming kernel alone. All reductions run
 // in a fixed order, so results are bitwise reproducible.
 
@@ -52,16 +52,16 @@ constexpr int kStatusWord = 0;
 enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3 };
 
 __host__ __device__ constexpr int logits_of(int n) { return 2 * n + n * n; }
-// logit columns padded to a multiple of 4: the projection's four column groups
+// logit count padded to a multiple of 4 (the tail's base array in shared memory)
 __host__ __device__ constexpr int cpad_of(int n) { return (logits_of(n) + 3) & ~3; }
 // Per-block record of a row in the workspace: C dot products, then sum v^2,
 // padded to a power of two >= 8 floats.
 __host__ __device__ constexpr int red_of(int n) {
   return logits_of(n) + 1 <= 8 ? 8 : (logits_of(n) + 1 <= 16 ? 16 : 32);
 }
-// fn slice in shared memory as the bulk copies land it: pieces of 8 rows of C
-// floats followed by a 16-byte gap (the gap puts the rows that a half-warp of
-// the projection reads into distinct banks).
+// fp32 fn slice in shared memory as the bulk copies land it (unpacked fn): pieces
+// of 8 rows of C floats followed by a 16-byte gap, which spreads the split
+// loop's reads over the banks.
 __host__ __device__ constexpr int fn_piece_bytes(int n) { return 8 * logits_of(n) * 4 + 16; }
 
 struct Params {
@@ -184,43 +184,6 @@ __device__ __forceinline__ int swizzled_scale_offset(int r, int c, int col_tiles
   return tile * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (c & 3);
 }
 
-// Sum over blocks of row r's per-block records ([r][g][RED] floats): thread t
-// loads the float4 number t % (RED/4) of records g = t/(RED/4) + k*kThreads/(RED/4)
-// (all loads issued before any add) and adds them in k order.
-template <int RED, int MAXK>
-__device__ __forceinline__ float4 sum_row_partials(const float* part, int r, int G, int tid) {
-  constexpr int V4 = RED / 4;
-  const float4* base = reinterpret_cast<const float4*>(part + static_cast<size_t>(r) * G * RED);
-  const int F = G * V4;
-  float4 v[MAXK];
-#pragma unroll
-  for (int k = 0; k < MAXK; ++k) {
-    const int f = tid + k * kThreads;
-    v[k] = f < F ? __ldcg(base + f) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  float4 a = v[0];
-#pragma unroll
-  for (int k = 1; k < MAXK; ++k) {
-    a.x += v[k].x;
-    a.y += v[k].y;
-    a.z += v[k].z;
-    a.w += v[k].w;
-  }
-  return a;
-}
-
-template <int N>
-__device__ __forceinline__ float tree_sum(const float (&v)[N]) {
-  if constexpr (N == 4) {
-    return (v[0] + v[1]) + (v[2] + v[3]);
-  } else {
-    float s = v[0];
-#pragma unroll
-    for (int i = 1; i < N; ++i) s += v[i];
-    return s;
-  }
-}
-
 // Registers of one row-pair step of a lane (4 columns of one row): the stream
 // vectors and up to 8 partial (or gathered) vectors, plus the shared-output /
 // embedding vector.
@@ -286,9 +249,9 @@ __host__ __device__ constexpr int packed_slice_bytes(int n) { return 3 * ntiles_
 static_assert(packed_slice_bytes(1) % 16 == 0 && packed_slice_bytes(2) % 16 == 0 && packed_slice_bytes(4) % 16 == 0,
               "a bulk copy moves a multiple of 16 bytes");
 
-template <int N, int FRONT>
 // 80 registers a thread: 512 threads leave room on the SM for the tail kernel's
 // blocks, which launch early (programmatic dependent launch).
+template <int N, int FRONT>
 __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   constexpr int C = logits_of(N);
   constexpr int KC = N * kCols;       // stream values per row in this block
@@ -391,6 +354,8 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   // ---- 3. wait for the preceding kernel, let the next one launch, and read
   griddep_wait();
   griddep_launch_dependents();
+  PairLoads<N> cur;  // the row data first: the longest round trip goes out first
+  if (FRONT != kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
   for (int k = tid; k < R * MIX; k += kT1) {  // [R][post n | comb n*n | pre n]
     const int r = k / MIX, c = k - r * MIX;
     if (c < N + N * N) {
@@ -413,8 +378,6 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
       cp_async4(ew_s + k, p.ew + k);
     }
   }
-  PairLoads<N> cur;
-  if (FRONT != kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
   cp_async_wait_all();
   __syncthreads();
   if (FRONT == kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
@@ -942,23 +905,21 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
         const int grp = lane < N ? 0 : (lane < 2 * N ? 1 : 2);
         const float l = lane < C ? scale_s[grp] * inv * s + base_s[lane] : 0.f;
         if (s_comb >= 0) {
-          // Sinkhorn in one thread: M = exp(L - max L); rows then columns, iters times
+          // M = exp(L - max L) with one exp per lane, then Sinkhorn in one thread
+          float lk = __shfl_sync(kFull, l, (lane + 2 * N) & 31);  // lane k < n*n: comb logit k
+          float mx = lk;
+#pragma unroll
+          for (int b = 1; b < NN; b <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, b));
+          const float ek = expf(lk - mx);
           float lc[NN];
 #pragma unroll
-          for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, l, 2 * N + k);
+          for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, ek, k);
           if (lane == 0) {
-            float t[NN];
-#pragma unroll
-            for (int k = 0; k < NN; ++k) t[k] = lc[k];
-#pragma unroll
-            for (int w = NN / 2; w >= 1; w >>= 1)
-#pragma unroll
-              for (int k = 0; k < w; ++k) t[k] = fmaxf(t[k], t[k + w]);
             float M[N][N];
 #pragma unroll
             for (int j = 0; j < N; ++j)
 #pragma unroll
-              for (int i = 0; i < N; ++i) M[j][i] = expf(lc[j * N + i] - t[0]);
+              for (int i = 0; i < N; ++i) M[j][i] = lc[j * N + i];
             sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
 #pragma unroll
             for (int j = 0; j < N; ++j)
