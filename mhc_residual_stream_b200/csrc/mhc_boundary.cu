@@ -67,8 +67,11 @@ __host__ __device__ constexpr int fn_piece_bytes(int n) { return 8 * logits_of(n
 struct Params {
   // front ends
   const __nv_bfloat16* pptr[kMaxPartials];  // partial u: [R, H] at pptr[u]
-  int premote;  // partials may be other GPUs' memory: plain loads, no L2 prefetch
+  int premote;  // partials may be other GPUs' memory or a mailbox: L2-only loads, no prefetch
   int P;
+  // mailbox collect: partial u's row r is complete once cflags[u * R + r] == cround
+  const unsigned* cflags;
+  unsigned cround;
   const __nv_bfloat16* gemm2;
   int num_perm;
   const float* ew;
@@ -213,7 +216,7 @@ __device__ __forceinline__ void load_pair(const Params& p, int r, int h0, const 
     if (p.premote) {
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (u < p.P) Q.pv[u] = ld_v2(p.pptr[u] + off);
+        if (u < p.P) Q.pv[u] = ld_cg_v2(p.pptr[u] + off);
     } else {
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -354,6 +357,15 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   // ---- 3. wait for the preceding kernel, let the next one launch, and read
   griddep_wait();
   griddep_launch_dependents();
+  if (FRONT == kPartials && p.cflags != nullptr) {
+    // mailbox collect: every producer's rows of this round published (bounded wait;
+    // an acquire per flag, then the block barrier orders every thread's reads)
+    bool ok = true;
+    for (int k = tid; k < p.P * R; k += kT1)
+      while (ok && ld_acquire_sys(p.cflags + k) != p.cround) ok = clock64() <= deadline;
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    __syncthreads();
+  }
   PairLoads<N> cur;  // the row data first: the longest round trip goes out first
   if (FRONT != kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
   for (int k = tid; k < R * MIX; k += kT1) {  // [R][post n | comb n*n | pre n]
@@ -414,7 +426,7 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
           for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
             float2 f[2];
             const __nv_bfloat16* src = p.pptr[u] + static_cast<size_t>(r) * H + h0;
-            unpack4x2(p.premote ? ld_v2(src) : ld_nc_v2(src), f);
+            unpack4x2(p.premote ? ld_cg_v2(src) : ld_nc_v2(src), f);
 #pragma unroll
             for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
           }
@@ -941,6 +953,66 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
 }
 
 
+// Mailbox of a consumer (one per rank of a TP group, in that rank's memory):
+// a 256-byte header (the status word at byte 0, the consumed round per parity
+// at bytes 8 and 12), the flags [2 parities][W producers][R rows] u32 (round + 1
+// of the last publish of that row), then the slots [2][W][R][H] bf16.
+struct MailboxLayout {
+  size_t flags_off, slots_off, total;
+};
+
+inline MailboxLayout mailbox_layout(int W, int R, int H) {
+  MailboxLayout L{};
+  L.flags_off = 256;
+  L.slots_off = (L.flags_off + static_cast<size_t>(2) * W * R * 4 + 255) & ~static_cast<size_t>(255);
+  L.total = L.slots_off + static_cast<size_t>(2) * W * R * H * 2;
+  return L;
+}
+
+struct PublishParams {
+  unsigned char* mb[kMaxPartials];  // every consumer's mailbox (this GPU's or a peer's)
+  const __nv_bfloat16* x;           // this producer's partial [R, H]
+  unsigned* status;                 // this producer's own mailbox header
+  int rank, W, R, H;
+  unsigned round;
+  size_t flags_off, slots_off;
+  int64_t budget_ns;
+};
+
+// Producer side of the mailbox: block (r, c) stores row r of x into slot
+// [parity][rank][r] of consumer c's mailbox, once c has consumed the round that
+// last used this parity (bounded wait), then raises the row's flag to round + 1
+// after a system-scope fence (the stores may cross NVLink).
+__global__ void __launch_bounds__(256) mailbox_publish_kernel(const PublishParams q) {
+  const int r = blockIdx.x, c = blockIdx.y;
+  const unsigned par = q.round & 1u;
+  unsigned char* mb = q.mb[c];
+  const unsigned* done = reinterpret_cast<const unsigned*>(mb + 8);
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    const long long deadline = wait_deadline(q.budget_ns);
+    while (ok && ld_acquire_sys(done + par) + 1u < q.round) ok = clock64() <= deadline;
+    if (!ok) record_error(q.status, MHC_ERR_DEVICE_TIMEOUT);
+  }
+  if (__syncthreads_or(!ok)) return;  // nothing written for a consumer that is behind
+  __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(mb + q.slots_off) +
+                        ((static_cast<size_t>(par) * q.W + q.rank) * q.R + r) * q.H;
+  const __nv_bfloat16* src = q.x + static_cast<size_t>(r) * q.H;
+  for (int k = threadIdx.x * 8; k < q.H; k += blockDim.x * 8) st_v4(slot + k, ld_nc_v4(src + k));
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence_system();
+    unsigned* flags = reinterpret_cast<unsigned*>(mb + q.flags_off);
+    st_release_sys(flags + (static_cast<size_t>(par) * q.W + q.rank) * q.R + r, q.round + 1u);
+  }
+}
+
+// After a collect: the round is consumed, its parity's slots may be reused.
+__global__ void mailbox_done_kernel(unsigned* done, unsigned par, unsigned value) {
+  __threadfence_system();
+  st_release_sys(done + par, value);
+}
+
 // fn [n*H, C] fp32 -> per block g the B operand of its projection as three bf16
 // terms, [G][3][CP8][n*64 + 8]: entry (t, c, k) is term t of fn[(k/64)*H + 64g + k%64][c];
 // columns c >= C and the 8-entry gap after each column are zero.
@@ -1262,13 +1334,15 @@ mhc_status post_pre_impl(const __nv_bfloat16* const* pptr, int num_partials, boo
                          float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out, mhc_bf16* aux_out,
                          mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out,
                          float* pre_out, int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
-                         mhc_stream stream) {
+                         mhc_stream stream, const unsigned* cflags = nullptr, unsigned cround = 0) {
   mhc_status st = check_mixes(residual, post, comb, residual_out);
   if (st != MHC_OK) return st;
   Params p{};
   for (int u = 0; u < num_partials; ++u) p.pptr[u] = pptr[u];
   p.premote = remote ? 1 : 0;
   p.P = num_partials;
+  p.cflags = cflags;
+  p.cround = cround;
   p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
@@ -1281,6 +1355,10 @@ mhc_status post_pre_impl(const __nv_bfloat16* const* pptr, int num_partials, boo
   st = fill_tail(p, pre, norm_weight, norm_eps, coeffs, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
                  hidden, hc_mult, workspace, ws_bytes);
   if (st != MHC_OK) return st;
+  if (cflags != nullptr && p.ctl == nullptr) {  // the flag wait reports through the workspace header
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return MHC_ERR_WORKSPACE;
+    p.ctl = static_cast<unsigned*>(workspace);
+  }
   return dispatch_n<kPartials>(p, hc_mult, stream);
 }
 
@@ -1325,6 +1403,73 @@ mhc_status mhc_boundary_post_pre_ptrs(const mhc_bf16* const* partials, int num_p
   return post_pre_impl(pptr, num_partials, true, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
                        residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult,
                        workspace, ws_bytes, stream);
+}
+
+size_t mhc_mailbox_bytes(int world, int rows, int hidden) {
+  if (world < 1 || world > kMaxPartials || !shape_ok(rows, hidden, 1)) return 0;
+  return mailbox_layout(world, rows, hidden).total;
+}
+
+mhc_status mhc_mailbox_init(void* mailbox, size_t bytes, mhc_stream stream) {
+  if (!mailbox || !aligned(mailbox, 256) || bytes < 256) return MHC_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(mailbox, 0, bytes, stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MHC_ERR_CUDA;
+  }
+  return MHC_OK;
+}
+
+mhc_status mhc_mailbox_publish(const mhc_bf16* x, int rank, uint32_t round, void* const* mailboxes, int world,
+                               int rows, int hidden, mhc_stream stream) {
+  if (world < 1 || world > kMaxPartials || !shape_ok(rows, hidden, 1)) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (!x || !aligned(x, 16) || !mailboxes || rank < 0 || rank >= world || round == 0xffffffffu)
+    return MHC_ERR_INVALID_ARG;
+  const MailboxLayout ml = mailbox_layout(world, rows, hidden);
+  PublishParams q{};
+  for (int c = 0; c < world; ++c) {
+    if (!mailboxes[c] || !aligned(mailboxes[c], 256)) return MHC_ERR_INVALID_ARG;
+    q.mb[c] = static_cast<unsigned char*>(mailboxes[c]);
+  }
+  q.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  q.status = static_cast<unsigned*>(mailboxes[rank]);
+  q.rank = rank;
+  q.W = world;
+  q.R = rows;
+  q.H = hidden;
+  q.round = round;
+  q.flags_off = ml.flags_off;
+  q.slots_off = ml.slots_off;
+  q.budget_ns = g_budget_ns;
+  mailbox_publish_kernel<<<dim3(rows, world), 256, 0, stream>>>(q);
+  if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
+  return MHC_OK;
+}
+
+mhc_status mhc_boundary_collect(void* mailbox, int world, uint32_t round, const mhc_bf16* residual,
+                                const float* post, const float* comb, const float* pre,
+                                const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
+                                mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input,
+                                const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out, float* pre_out,
+                                int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
+                                mhc_stream stream) {
+  if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (world < 1 || world > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (!mailbox || !aligned(mailbox, 256) || round == 0xffffffffu) return MHC_ERR_INVALID_ARG;
+  const MailboxLayout ml = mailbox_layout(world, rows, hidden);
+  const unsigned par = round & 1u;
+  unsigned char* mb = static_cast<unsigned char*>(mailbox);
+  const __nv_bfloat16* slots = reinterpret_cast<const __nv_bfloat16*>(mb + ml.slots_off);
+  const __nv_bfloat16* pptr[kMaxPartials];
+  for (int u = 0; u < world; ++u) pptr[u] = slots + (static_cast<size_t>(par) * world + u) * rows * hidden;
+  const unsigned* flags = reinterpret_cast<const unsigned*>(mb + ml.flags_off) + static_cast<size_t>(par) * world * rows;
+  mhc_status st = post_pre_impl(pptr, world, true, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                                residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden,
+                                hc_mult, workspace, ws_bytes, stream, flags, round + 1u);
+  if (st != MHC_OK) return st;
+  // an ordinary launch: it runs once the boundary has read every slot of this round
+  mailbox_done_kernel<<<1, 1, 0, stream>>>(reinterpret_cast<unsigned*>(mb + 8), par, round + 1u);
+  if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
+  return MHC_OK;
 }
 
 mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_permuted, const float* expert_weights,

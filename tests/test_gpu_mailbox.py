@@ -1,0 +1,213 @@
+"""The publish/collect mailbox of the tensor-parallel boundary on one GPU.
+
+* One process plays every producer and every consumer of a group on one stream:
+  each round every producer publishes, then every consumer collects. Each
+  collect must give bitwise the results of the strided entry over the same
+  partials (the same sum order), over four rounds, so both parities are used
+  twice and the flow control of round t + 2 sees round t consumed.
+* The header words: after round t every flag of parity t & 1 reads t + 1 and the
+  parity's consumed word reads t + 1.
+* A collect of a round nobody published runs out of its (shortened) wait and
+  records MHC_ERR_DEVICE_TIMEOUT in the workspace; a publish two rounds ahead of
+  a consumer runs out of its wait, writes nothing and records the timeout in the
+  producer's own mailbox. Both are waits on words that nothing sets.
+* Two processes on the same GPU form a gloo group of 2 and exchange mailboxes
+  through CUDA IPC (PeerMailbox). Each round both publish, a host barrier
+  follows, then both collect: every wait is satisfied when its kernel starts, so
+  no kernel waits on another that runs at the same time.
+"""
+
+import datetime
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from mhc_residual_stream_b200 import mhc as M
+from mhc_residual_stream_b200 import synthetic as S
+
+from _parity import DEV, alloc_outputs, assert_bf16_close, check_tail, f64, gpu_post_pre, oracle_post_pre, to_dev
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = 256  # status word at byte 0, consumed words at bytes 8 and 12, then the flags
+
+
+def _header(mb: torch.Tensor, W: int, R: int):
+    """(consumed words [2], flags [2][W][R]) of a mailbox, read on the host."""
+    words = mb[:HEADER].cpu().view(torch.int32).numpy().view(np.uint32)
+    flags = mb[HEADER:HEADER + 2 * W * R * 4].cpu().view(torch.int32).numpy().view(np.uint32)
+    return words[2:4].copy(), flags.reshape(2, W, R).copy()
+
+
+def _collect(mb, W, t, d, g, packed=False):
+    R, n, H = g["residual"].shape
+    out = alloc_outputs(R, n, H)
+    ws = M.new_workspace(R, H, n, DEV)
+    M.mhc_boundary_collect(mb, W, t, g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"],
+                           d["norm_eps"], M.Coeffs.from_weights(d["coeff"], DEV, packed=packed),
+                           out["residual_out"], layer_input=out["layer_input"],
+                           mxfp8=(out["q_data"], out["q_scale"], True), post_out=out["post"], comb_out=out["comb"],
+                           pre_out=out["pre"], workspace=ws)
+    return out, ws
+
+
+@pytest.mark.parametrize("R,H,n,W,packed", [(32, 7168, 4, 2, True), (7, 192, 2, 3, False),
+                                            (128, 512, 4, 16, False), (1, 64, 1, 1, False)])
+def test_rounds_match_strided_bitwise(R, H, n, W, packed):
+    from mhc_residual_stream_b200 import build
+    build.build()
+    mbs = [M.new_mailbox(W, R, H, DEV) for _ in range(W)]
+    ptrs = [m.data_ptr() for m in mbs]
+    for t in range(4):
+        d = S.draw_boundary(R, H, n=n, partials=W, seed=7100 + 10 * t + W)
+        ref = gpu_post_pre(d, packed=packed)
+        g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
+        xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
+        for u in range(W):
+            M.mhc_mailbox_publish(xs[u], u, t, ptrs)
+        outs = [_collect(mbs[c], W, t, d, g, packed) for c in range(W)]
+        torch.cuda.synchronize()
+        for c, (out, ws) in enumerate(outs):
+            assert M.mhc_get_device_status(ws) == M.OK, (t, c)
+            for k, v in out.items():
+                assert torch.equal(v.cpu(), ref[k]), (t, c, k)
+        for c in range(W):
+            assert M.mhc_get_device_status(mbs[c]) == M.OK  # no producer timed out
+            done, flags = _header(mbs[c], W, R)
+            assert done[t & 1] == t + 1 and (t == 0 or done[(t - 1) & 1] == t), (t, c, done)
+            assert (flags[t & 1] == t + 1).all(), (t, c)
+
+
+def test_collect_of_unpublished_round_times_out_and_recovers():
+    R, H, n, W = 4, 256, 4, 2
+    d = S.draw_boundary(R, H, n=n, partials=W, seed=7201)
+    g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
+    mb, other = M.new_mailbox(W, R, H, DEV), M.new_mailbox(W, R, H, DEV)
+    old = M.mhc_debug_set_wait(20_000_000, 0)  # 20 ms
+    try:
+        out, ws = _collect(mb, W, 0, d, g)
+        assert M.mhc_get_device_status(ws) == M.DEVICE_TIMEOUT
+    finally:
+        M.mhc_debug_set_wait(old, 0)
+    assert M.mhc_get_device_status(ws) == M.OK  # reading cleared it
+    # round 1 (the other parity) published and collected as usual
+    xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
+    for u in range(W):
+        M.mhc_mailbox_publish(xs[u], u, 1, [mb.data_ptr(), other.data_ptr()])
+    out, ws = _collect(mb, W, 1, d, g)
+    torch.cuda.synchronize()
+    assert M.mhc_get_device_status(ws) == M.OK
+    ref = gpu_post_pre(d)
+    for k, v in out.items():
+        assert torch.equal(v.cpu(), ref[k]), k
+
+
+def test_publish_ahead_of_consumer_times_out_and_writes_nothing():
+    R, H, W = 3, 128, 2
+    mbs = [M.new_mailbox(W, R, H, DEV) for _ in range(W)]
+    x = torch.randn(R, H, device=DEV).to(torch.bfloat16)
+    old = M.mhc_debug_set_wait(20_000_000, 0)
+    try:
+        M.mhc_mailbox_publish(x, 0, 2, [m.data_ptr() for m in mbs])  # nobody consumed round 0
+        torch.cuda.synchronize()
+    finally:
+        M.mhc_debug_set_wait(old, 0)
+    assert M.mhc_get_device_status(mbs[0]) == M.DEVICE_TIMEOUT  # the producer's own mailbox
+    assert M.mhc_get_device_status(mbs[1]) == M.OK
+    for m in mbs:
+        assert int(m.count_nonzero()) == 0  # no slot, flag or consumed word written
+    # once round 0 is consumed (here: published and collected), round 2 goes through
+    d = S.draw_boundary(R, H, n=1, partials=W, seed=7301)
+    d["partials"][0] = x.cpu()
+    g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
+    xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
+    for t in (0, 2):
+        for u in range(W):
+            M.mhc_mailbox_publish(xs[u], u, t, [m.data_ptr() for m in mbs])
+        outs = [_collect(mbs[c], W, t, d, g) for c in range(W)]
+        torch.cuda.synchronize()
+        ref = gpu_post_pre(d)
+        for out, ws in outs:
+            assert M.mhc_get_device_status(ws) == M.OK
+            for k, v in out.items():
+                assert torch.equal(v.cpu(), ref[k]), (t, k)
+    assert M.mhc_get_device_status(mbs[0]) == M.OK
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+ROUNDS = 3
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from mhc_residual_stream_b200 import mhc as M
+    from mhc_residual_stream_b200 import synthetic as S
+    from mhc_residual_stream_b200.tp import PeerMailbox
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    box = None
+    try:
+        torch.cuda.set_device(0)
+        R, H, n = 16, 7168, 4
+        box = PeerMailbox(R, H, device="cuda:0")
+        for t in range(ROUNDS):
+            d = S.draw_boundary(R, H, n=n, partials=world, seed=7400 + t)  # the same draw on both ranks
+            x = d["partials"][rank].to("cuda:0").contiguous()  # this rank's sublayer output
+            box.publish(x, t)
+            torch.cuda.synchronize()
+            dist.barrier()  # every rank's rows of round t are in every mailbox
+            g = {k: d[k].to("cuda:0") for k in ("residual", "post", "comb", "pre", "norm_weight")}
+            res_out = torch.empty_like(g["residual"])
+            li = torch.empty(R, H, dtype=torch.bfloat16, device="cuda:0")
+            post, comb, pre = (torch.empty(R, n, device="cuda:0"), torch.empty(R, n, n, device="cuda:0"),
+                               torch.empty(R, n, device="cuda:0"))
+            ws = M.new_workspace(R, H, n, "cuda:0")
+            box.collect(t, g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"], d["norm_eps"],
+                        M.Coeffs.from_weights(d["coeff"], "cuda:0"), res_out, layer_input=li, post_out=post,
+                        comb_out=comb, pre_out=pre, workspace=ws)
+            torch.cuda.synchronize()
+            st, pst = M.mhc_get_device_status(ws), M.mhc_get_device_status(box.local)
+            dist.barrier()  # round t consumed everywhere before anyone publishes round t + 1
+            q.put((rank, t, st, pst, {k: v.cpu() for k, v in dict(residual_out=res_out, layer_input=li, post=post,
+                                                                   comb=comb, pre=pre).items()}))
+    finally:
+        if box is not None:
+            box.close()      # unmap the peer's mailbox ...
+            dist.barrier()   # ... on every rank before any rank frees its own
+        dist.destroy_process_group()
+
+
+def test_two_processes_publish_and_collect_through_ipc():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=240) for _ in range(2 * ROUNDS)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    by_round = {}
+    for rank, t, st, pst, res in got:
+        assert st == M.OK and pst == M.OK, (rank, t, st, pst)
+        by_round.setdefault(t, {})[rank] = res
+    for t in range(ROUNDS):
+        d = S.draw_boundary(16, 7168, n=4, partials=2, seed=7400 + t)
+        orc = oracle_post_pre(d, mxfp8=False)
+        for rank, res in sorted(by_round[t].items()):
+            assert_bf16_close(f64(res["residual_out"]), orc["residual"], f"round {t} rank {rank} streams")
+            check_tail(d, dict(res), orc, mxfp8=False, what=f"round {t} rank {rank}")
+        for k in by_round[t][0]:  # both ranks computed the same boundary
+            assert torch.equal(by_round[t][0][k], by_round[t][1][k]), (t, k)
