@@ -205,39 +205,46 @@ MHC_API mhc_status mhc_boundary_post_pre_ptrs(
 
 /* Publish/collect mailbox of a tensor-parallel group, without multicast
  * ([all_reduce] BoundaryAllReduce.publish_target / mark_published: a producer
- * stores its contribution into slot [rank][token] of the mailbox and raises a
- * generation; here each rank's mailbox is its own device memory and the
- * producers store into every rank's mailbox, over NVLink for the peers').
- * Layout of a mailbox (mhc_mailbox_bytes(W, R, H) bytes, 256-byte aligned):
- * a 256-byte header (status word at byte 0; at bytes 8 and 12 the round + 1 last
- * consumed for each parity), flags uint32 [2][W][R] (round + 1 of the last
- * publish of row r by producer u), slots bf16 [2][W][R][H]. Round t uses parity
- * t & 1, so a producer may run one round ahead of a consumer.
- *   mhc_mailbox_init: zero a mailbox (before first use, on its own stream).
- *   mhc_mailbox_publish: producer `rank` of a group of `world` stores x [R, H]
- *     bf16 (16-byte aligned) into slot [t & 1][rank] of every consumer's
- *     mailbox (mailboxes: HOST array of `world` device pointers, this GPU's or
- *     peers' via mhc_ipc_import), then raises each row's flag to t + 1 after a
- *     system-scope fence. Before writing into a consumer's mailbox it waits
- *     (bounded, mhc_debug_set_wait) until that consumer has consumed round
- *     t - 2; on timeout it writes nothing there and records
+ * stores its bf16 contribution, negative zero cleared, into slot [rank][token]
+ * of the mailbox; the consumer's reduction waits for it. Here each rank's
+ * mailbox is its own device memory and producers store into every rank's
+ * mailbox, over NVLink for the peers'.)
+ * Layout of a mailbox (mhc_mailbox_bytes(W, M, H) bytes, 256-byte aligned, M
+ * the row capacity): a 256-byte header (status word at byte 0; at bytes 8 and
+ * 12 the round + 1 last consumed for each parity), then slots bf16
+ * [2][W][M][H]. A slot element holding negative zero (0x8000) is "not yet
+ * written": producers never store it, the consumer writes it back into every
+ * element it has read. Round t uses parity t & 1, so a producer may run one
+ * round ahead of a consumer.
+ *   mhc_mailbox_bytes: 0 for world outside [1, 16] or an unsupported (M, H).
+ *   mhc_mailbox_init: header zero, every slot element negative zero (a kernel
+ *     on `stream`; bytes = mhc_mailbox_bytes(...), a multiple of 16).
+ *   mhc_mailbox_publish: producer `rank` of a group of `world` stores x
+ *     [rows, H] bf16 (16-byte aligned, rows <= M) into slot [t & 1][rank] of
+ *     every consumer's mailbox (mailboxes: HOST array of `world` device
+ *     pointers, this GPU's or peers' via mhc_ipc_import), with each negative
+ *     zero stored as positive zero. Before writing into a consumer's mailbox it
+ *     waits (bounded, mhc_debug_set_wait) until that consumer has consumed
+ *     round t - 2; on timeout it writes nothing there and records
  *     MHC_ERR_DEVICE_TIMEOUT in its OWN mailbox's status word (read it with
  *     mhc_get_device_status(mailboxes[rank])).
- *   mhc_boundary_collect: the consumer's boundary of round t: as
- *     mhc_boundary_post_pre with the W slots of parity t & 1 as the partials
- *     (summed in producer order). Its streaming kernel waits (bounded) until
- *     every flag of the round reads t + 1; a timeout records
- *     MHC_ERR_DEVICE_TIMEOUT in the workspace (required, also for the
- *     residual-only form). After the boundary a one-thread kernel marks round
- *     t consumed. round must be below 0xffffffff.
+ *   mhc_boundary_collect: the consumer's boundary of round t over `rows`
+ *     (<= M) tokens: as mhc_boundary_post_pre with the W slots of parity t & 1
+ *     as the partials (summed in producer order). Its streaming kernel re-reads
+ *     each slot element until it is not negative zero (bounded; a timeout
+ *     records MHC_ERR_DEVICE_TIMEOUT in the workspace, which is required, also
+ *     for the residual-only form) and marks it negative zero again once read.
+ *     A one-thread kernel then marks round t consumed. round must be below
+ *     0xffffffff.
  * Producers and consumers on different GPUs run concurrently; the waits are
- * the only ordering between them. */
-MHC_API size_t mhc_mailbox_bytes(int world, int rows, int hidden);
+ * the only ordering between them. A published value of negative zero arrives
+ * as positive zero (the sum then differs at most in the sign of a zero). */
+MHC_API size_t mhc_mailbox_bytes(int world, int max_rows, int hidden);
 MHC_API mhc_status mhc_mailbox_init(void* mailbox, size_t bytes, mhc_stream stream);
-MHC_API mhc_status mhc_mailbox_publish(const mhc_bf16* x, int rank, uint32_t round, void* const* mailboxes,
-                                       int world, int rows, int hidden, mhc_stream stream);
+MHC_API mhc_status mhc_mailbox_publish(const mhc_bf16* x, int rows, int hidden, int rank, uint32_t round,
+                                       void* const* mailboxes, int world, int max_rows, mhc_stream stream);
 MHC_API mhc_status mhc_boundary_collect(
-    void* mailbox, int world, uint32_t round,
+    void* mailbox, int world, int max_rows, uint32_t round,
     const mhc_bf16* residual, const float* post, const float* comb, const float* pre,
     const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
     mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
@@ -343,7 +350,7 @@ MHC_API mhc_status mhc_get_device_status(void* workspace, mhc_stream stream);
 MHC_API const char* mhc_status_string(mhc_status status);
 
 /* Test hook for the bounded waits. A kernel waits on the TMA copies of its fn
- * slice (and the mailbox kernels on their flags) with a time limit: `budget_ns`
+ * slice (and the mailbox kernels on their slots and consumed words) with a time limit: `budget_ns`
  * > 0 sets it (default 1e9 ns, counted as
  * 2 SM cycles per ns); `extra_units` makes that wait expect that many 16-byte
  * units more than are copied, so that it can never complete and runs out

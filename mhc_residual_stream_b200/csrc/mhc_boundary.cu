@@ -49,7 +49,10 @@ constexpr int kMaxBlocks = 148;  // most H/64 blocks: the tail's per-lane loads 
 constexpr size_t kWsHeader = 1024;
 constexpr int kStatusWord = 0;
 
-enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3 };
+enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3, kMailbox = 4 };
+// Fronts whose x is a sum of P bf16 partials (kMailbox: slots of a mailbox that
+// producers fill concurrently, each element valid once it is not negative zero).
+__host__ __device__ constexpr bool sums_partials(int front) { return front == kPartials || front == kMailbox; }
 
 __host__ __device__ constexpr int logits_of(int n) { return 2 * n + n * n; }
 // logit count padded to a multiple of 4 (the tail's base array in shared memory)
@@ -67,11 +70,8 @@ __host__ __device__ constexpr int fn_piece_bytes(int n) { return 8 * logits_of(n
 struct Params {
   // front ends
   const __nv_bfloat16* pptr[kMaxPartials];  // partial u: [R, H] at pptr[u]
-  int premote;  // partials may be other GPUs' memory or a mailbox: L2-only loads, no prefetch
+  int premote;  // partials may be other GPUs' memory: L2-only loads, no prefetch
   int P;
-  // mailbox collect: partial u's row r is complete once cflags[u * R + r] == cround
-  const unsigned* cflags;
-  unsigned cround;
   const __nv_bfloat16* gemm2;
   int num_perm;
   const float* ew;
@@ -211,9 +211,9 @@ __device__ __forceinline__ void load_pair(const Params& p, int r, int h0, const 
 #pragma unroll
     for (int j = 0; j < N; ++j) Q.rv[j] = ld_v2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
   }
-  if (FRONT == kPartials) {
+  if (sums_partials(FRONT)) {
     const size_t off = static_cast<size_t>(r) * H + h0;
-    if (p.premote) {
+    if (FRONT == kMailbox || p.premote) {
 #pragma unroll
       for (int u = 0; u < 8; ++u)
         if (u < p.P) Q.pv[u] = ld_cg_v2(p.pptr[u] + off);
@@ -234,6 +234,20 @@ __device__ __forceinline__ void load_pair(const Params& p, int r, int h0, const 
       }
     }
   }
+}
+
+// A mailbox slot's 4 elements as loaded, re-read until none is negative zero
+// (bounded: on timeout the status records it and the values are used as they are).
+__device__ __forceinline__ uint2 settle_slot(const __nv_bfloat16* src, uint2 v, long long deadline,
+                                             unsigned* status) {
+  while (has_neg_zero(v)) {
+    if (clock64() > deadline) {
+      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+      break;
+    }
+    v = ld_volatile_v2(src);
+  }
+  return v;
 }
 
 // fn as three bf16 terms, f = hi + mid + lo to 2^-24: each bf16 x bf16 product is
@@ -320,8 +334,8 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
       } else {
         for (int j = 0; j < N; ++j) prefetch_l2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
       }
-      if (FRONT == kPartials) {
-        if (!p.premote)
+      if (sums_partials(FRONT)) {  // (a mailbox's slots are this GPU's memory)
+        if (FRONT == kMailbox || !p.premote)
           for (int pp = 0; pp < p.P; ++pp) prefetch_l2(p.pptr[pp] + static_cast<size_t>(r) * H + h0);
       } else if (FRONT == kMoe) {
         prefetch_l2(p.shared_out + static_cast<size_t>(r) * H + h0);
@@ -357,15 +371,6 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   // ---- 3. wait for the preceding kernel, let the next one launch, and read
   griddep_wait();
   griddep_launch_dependents();
-  if (FRONT == kPartials && p.cflags != nullptr) {
-    // mailbox collect: every producer's rows of this round published (bounded wait;
-    // an acquire per flag, then the block barrier orders every thread's reads)
-    bool ok = true;
-    for (int k = tid; k < p.P * R; k += kT1)
-      while (ok && ld_acquire_sys(p.cflags + k) != p.cround) ok = clock64() <= deadline;
-    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-    __syncthreads();
-  }
   PairLoads<N> cur;  // the row data first: the longest round trip goes out first
   if (FRONT != kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
   for (int k = tid; k < R * MIX; k += kT1) {  // [R][post n | comb n*n | pre n]
@@ -408,15 +413,17 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
     float2 xs[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) xs[t] = make_float2(0.f, 0.f);
-    if (FRONT == kPartials || FRONT == kMoe) {
+    if (sums_partials(FRONT) || FRONT == kMoe) {
       float2 rf[N][2];
       if (valid) {
 #pragma unroll
         for (int j = 0; j < N; ++j) unpack4x2(cur.rv[j], rf[j]);
-        if (FRONT == kPartials) {
+        if (sums_partials(FRONT)) {
+          const size_t off = static_cast<size_t>(r) * H + h0;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             if (u < p.P) {
+              if (FRONT == kMailbox) cur.pv[u] = settle_slot(p.pptr[u] + off, cur.pv[u], deadline, status);
               float2 f[2];
               unpack4x2(cur.pv[u], f);
 #pragma unroll
@@ -425,10 +432,16 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
           }
           for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
             float2 f[2];
-            const __nv_bfloat16* src = p.pptr[u] + static_cast<size_t>(r) * H + h0;
-            unpack4x2(p.premote ? ld_cg_v2(src) : ld_nc_v2(src), f);
+            const __nv_bfloat16* src = p.pptr[u] + off;
+            uint2 v = (FRONT == kMailbox || p.premote) ? ld_cg_v2(src) : ld_nc_v2(src);
+            if (FRONT == kMailbox) v = settle_slot(src, v, deadline, status);
+            unpack4x2(v, f);
 #pragma unroll
             for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
+          }
+          if (FRONT == kMailbox) {  // consumed: back to "not written" for the round after next
+            for (int u = 0; u < p.P; ++u)
+              st_v2(const_cast<__nv_bfloat16*>(p.pptr[u]) + off, make_uint2(kNegZero2, kNegZero2));
           }
         } else {
           unpack4x2(cur.sv, xs);
@@ -954,35 +967,30 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
 
 
 // Mailbox of a consumer (one per rank of a TP group, in that rank's memory):
-// a 256-byte header (the status word at byte 0, the consumed round per parity
-// at bytes 8 and 12), the flags [2 parities][W producers][R rows] u32 (round + 1
-// of the last publish of that row), then the slots [2][W][R][H] bf16.
-struct MailboxLayout {
-  size_t flags_off, slots_off, total;
-};
+// a 256-byte header (the status word at byte 0, the consumed round + 1 per parity
+// at bytes 8 and 12), then the slots [2 parities][W producers][M rows][H] bf16,
+// M the mailbox's row capacity. A slot element that holds negative zero has not
+// been written yet: the consumer turns every element it reads back into that
+// mark, and a producer never stores it.
+constexpr size_t kMailboxHeader = 256;
 
-inline MailboxLayout mailbox_layout(int W, int R, int H) {
-  MailboxLayout L{};
-  L.flags_off = 256;
-  L.slots_off = (L.flags_off + static_cast<size_t>(2) * W * R * 4 + 255) & ~static_cast<size_t>(255);
-  L.total = L.slots_off + static_cast<size_t>(2) * W * R * H * 2;
-  return L;
+inline size_t mailbox_total(int W, int M, int H) {
+  return kMailboxHeader + static_cast<size_t>(2) * W * M * H * 2;
 }
 
 struct PublishParams {
   unsigned char* mb[kMaxPartials];  // every consumer's mailbox (this GPU's or a peer's)
-  const __nv_bfloat16* x;           // this producer's partial [R, H]
+  const __nv_bfloat16* x;           // this producer's contribution [R, H]
   unsigned* status;                 // this producer's own mailbox header
-  int rank, W, R, H;
+  int rank, W, M, H;
   unsigned round;
-  size_t flags_off, slots_off;
   int64_t budget_ns;
 };
 
-// Producer side of the mailbox: block (r, c) stores row r of x into slot
-// [parity][rank][r] of consumer c's mailbox, once c has consumed the round that
-// last used this parity (bounded wait), then raises the row's flag to round + 1
-// after a system-scope fence (the stores may cross NVLink).
+// Producer side: block (r, c) stores row r of x, negative zeros made positive,
+// into slot [parity][rank][r] of consumer c's mailbox once c has consumed the
+// round that last used this parity (bounded wait). No flag follows: each element
+// is its own mark, so nothing waits for the stores to be acknowledged.
 __global__ void __launch_bounds__(256) mailbox_publish_kernel(const PublishParams q) {
   const int r = blockIdx.x, c = blockIdx.y;
   const unsigned par = q.round & 1u;
@@ -994,16 +1002,18 @@ __global__ void __launch_bounds__(256) mailbox_publish_kernel(const PublishParam
     while (ok && ld_acquire_sys(done + par) + 1u < q.round) ok = clock64() <= deadline;
     if (!ok) record_error(q.status, MHC_ERR_DEVICE_TIMEOUT);
   }
+  // the barrier carries thread 0's acquire to every thread's stores
   if (__syncthreads_or(!ok)) return;  // nothing written for a consumer that is behind
-  __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(mb + q.slots_off) +
-                        ((static_cast<size_t>(par) * q.W + q.rank) * q.R + r) * q.H;
+  __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(mb + kMailboxHeader) +
+                        ((static_cast<size_t>(par) * q.W + q.rank) * q.M + r) * q.H;
   const __nv_bfloat16* src = q.x + static_cast<size_t>(r) * q.H;
-  for (int k = threadIdx.x * 8; k < q.H; k += blockDim.x * 8) st_v4(slot + k, ld_nc_v4(src + k));
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence_system();
-    unsigned* flags = reinterpret_cast<unsigned*>(mb + q.flags_off);
-    st_release_sys(flags + (static_cast<size_t>(par) * q.W + q.rank) * q.R + r, q.round + 1u);
+  for (int k = threadIdx.x * 8; k < q.H; k += blockDim.x * 8) {
+    uint4 v = ld_nc_v4(src + k);
+    v.x = clear_neg_zero2(v.x);
+    v.y = clear_neg_zero2(v.y);
+    v.z = clear_neg_zero2(v.z);
+    v.w = clear_neg_zero2(v.w);
+    st_v4(slot + k, v);
   }
 }
 
@@ -1011,6 +1021,15 @@ __global__ void __launch_bounds__(256) mailbox_publish_kernel(const PublishParam
 __global__ void mailbox_done_kernel(unsigned* done, unsigned par, unsigned value) {
   __threadfence_system();
   st_release_sys(done + par, value);
+}
+
+// A fresh mailbox: header zero, every slot element negative zero.
+__global__ void mailbox_init_kernel(unsigned char* mb, size_t units) {
+  const size_t i0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i0 < kMailboxHeader / 16) st_v4(mb + i0 * 16, make_uint4(0, 0, 0, 0));
+  const uint4 z = make_uint4(kNegZero2, kNegZero2, kNegZero2, kNegZero2);
+  for (size_t i = i0; i < units; i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    st_v4(mb + kMailboxHeader + i * 16, z);
 }
 
 // fn [n*H, C] fp32 -> per block g the B operand of its projection as three bf16
@@ -1334,15 +1353,13 @@ mhc_status post_pre_impl(const __nv_bfloat16* const* pptr, int num_partials, boo
                          float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out, mhc_bf16* aux_out,
                          mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out,
                          float* pre_out, int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
-                         mhc_stream stream, const unsigned* cflags = nullptr, unsigned cround = 0) {
+                         mhc_stream stream, bool mailbox = false) {
   mhc_status st = check_mixes(residual, post, comb, residual_out);
   if (st != MHC_OK) return st;
   Params p{};
   for (int u = 0; u < num_partials; ++u) p.pptr[u] = pptr[u];
   p.premote = remote ? 1 : 0;
   p.P = num_partials;
-  p.cflags = cflags;
-  p.cround = cround;
   p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
@@ -1355,11 +1372,11 @@ mhc_status post_pre_impl(const __nv_bfloat16* const* pptr, int num_partials, boo
   st = fill_tail(p, pre, norm_weight, norm_eps, coeffs, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
                  hidden, hc_mult, workspace, ws_bytes);
   if (st != MHC_OK) return st;
-  if (cflags != nullptr && p.ctl == nullptr) {  // the flag wait reports through the workspace header
+  if (mailbox && p.ctl == nullptr) {  // the slot wait reports through the workspace header
     if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return MHC_ERR_WORKSPACE;
     p.ctl = static_cast<unsigned*>(workspace);
   }
-  return dispatch_n<kPartials>(p, hc_mult, stream);
+  return mailbox ? dispatch_n<kMailbox>(p, hc_mult, stream) : dispatch_n<kPartials>(p, hc_mult, stream);
 }
 
 }  // namespace
@@ -1405,26 +1422,31 @@ mhc_status mhc_boundary_post_pre_ptrs(const mhc_bf16* const* partials, int num_p
                        workspace, ws_bytes, stream);
 }
 
-size_t mhc_mailbox_bytes(int world, int rows, int hidden) {
-  if (world < 1 || world > kMaxPartials || !shape_ok(rows, hidden, 1)) return 0;
-  return mailbox_layout(world, rows, hidden).total;
+size_t mhc_mailbox_bytes(int world, int max_rows, int hidden) {
+  if (world < 1 || world > kMaxPartials || !shape_ok(max_rows, hidden, 1)) return 0;
+  return mailbox_total(world, max_rows, hidden);
 }
 
 mhc_status mhc_mailbox_init(void* mailbox, size_t bytes, mhc_stream stream) {
-  if (!mailbox || !aligned(mailbox, 256) || bytes < 256) return MHC_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(mailbox, 0, bytes, stream) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MHC_ERR_CUDA;
-  }
+  if (!mailbox || !aligned(mailbox, 256) || bytes < kMailboxHeader || bytes % 16 != 0) return MHC_ERR_INVALID_ARG;
+  const size_t units = (bytes - kMailboxHeader) / 16;
+  const int sms = sm_count();
+  size_t blocks = (units + 255) / 256;
+  const size_t cap = static_cast<size_t>(sms > 0 ? sms : 1) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  mailbox_init_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<unsigned char*>(mailbox),
+                                                                         units);
+  if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
   return MHC_OK;
 }
 
-mhc_status mhc_mailbox_publish(const mhc_bf16* x, int rank, uint32_t round, void* const* mailboxes, int world,
-                               int rows, int hidden, mhc_stream stream) {
-  if (world < 1 || world > kMaxPartials || !shape_ok(rows, hidden, 1)) return MHC_ERR_UNSUPPORTED_SHAPE;
+mhc_status mhc_mailbox_publish(const mhc_bf16* x, int rows, int hidden, int rank, uint32_t round,
+                               void* const* mailboxes, int world, int max_rows, mhc_stream stream) {
+  if (world < 1 || world > kMaxPartials || !shape_ok(max_rows, hidden, 1) || rows < 1 || rows > max_rows)
+    return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!x || !aligned(x, 16) || !mailboxes || rank < 0 || rank >= world || round == 0xffffffffu)
     return MHC_ERR_INVALID_ARG;
-  const MailboxLayout ml = mailbox_layout(world, rows, hidden);
   PublishParams q{};
   for (int c = 0; c < world; ++c) {
     if (!mailboxes[c] || !aligned(mailboxes[c], 256)) return MHC_ERR_INVALID_ARG;
@@ -1434,18 +1456,16 @@ mhc_status mhc_mailbox_publish(const mhc_bf16* x, int rank, uint32_t round, void
   q.status = static_cast<unsigned*>(mailboxes[rank]);
   q.rank = rank;
   q.W = world;
-  q.R = rows;
+  q.M = max_rows;
   q.H = hidden;
   q.round = round;
-  q.flags_off = ml.flags_off;
-  q.slots_off = ml.slots_off;
   q.budget_ns = g_budget_ns;
   mailbox_publish_kernel<<<dim3(rows, world), 256, 0, stream>>>(q);
   if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
   return MHC_OK;
 }
 
-mhc_status mhc_boundary_collect(void* mailbox, int world, uint32_t round, const mhc_bf16* residual,
+mhc_status mhc_boundary_collect(void* mailbox, int world, int max_rows, uint32_t round, const mhc_bf16* residual,
                                 const float* post, const float* comb, const float* pre,
                                 const mhc_bf16* norm_weight, float norm_eps, const mhc_coeff_args* coeffs,
                                 mhc_bf16* residual_out, mhc_bf16* aux_out, mhc_bf16* layer_input,
@@ -1453,20 +1473,19 @@ mhc_status mhc_boundary_collect(void* mailbox, int world, uint32_t round, const 
                                 int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
                                 mhc_stream stream) {
   if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
-  if (world < 1 || world > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
+  if (world < 1 || world > kMaxPartials || max_rows < rows || max_rows > kMaxRows) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!mailbox || !aligned(mailbox, 256) || round == 0xffffffffu) return MHC_ERR_INVALID_ARG;
-  const MailboxLayout ml = mailbox_layout(world, rows, hidden);
   const unsigned par = round & 1u;
   unsigned char* mb = static_cast<unsigned char*>(mailbox);
-  const __nv_bfloat16* slots = reinterpret_cast<const __nv_bfloat16*>(mb + ml.slots_off);
+  const __nv_bfloat16* slots = reinterpret_cast<const __nv_bfloat16*>(mb + kMailboxHeader);
   const __nv_bfloat16* pptr[kMaxPartials];
-  for (int u = 0; u < world; ++u) pptr[u] = slots + (static_cast<size_t>(par) * world + u) * rows * hidden;
-  const unsigned* flags = reinterpret_cast<const unsigned*>(mb + ml.flags_off) + static_cast<size_t>(par) * world * rows;
+  for (int u = 0; u < world; ++u)
+    pptr[u] = slots + (static_cast<size_t>(par) * world + u) * max_rows * static_cast<size_t>(hidden);
   mhc_status st = post_pre_impl(pptr, world, true, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
                                 residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden,
-                                hc_mult, workspace, ws_bytes, stream, flags, round + 1u);
+                                hc_mult, workspace, ws_bytes, stream, true);
   if (st != MHC_OK) return st;
-  // an ordinary launch: it runs once the boundary has read every slot of this round
+  // an ordinary launch: it runs once the boundary has read (and re-marked) every slot of this round
   mailbox_done_kernel<<<1, 1, 0, stream>>>(reinterpret_cast<unsigned*>(mb + 8), par, round + 1u);
   if (cudaGetLastError() != cudaSuccess) return MHC_ERR_CUDA;
   return MHC_OK;

@@ -122,6 +122,19 @@ __device__ __forceinline__ uint2 ld_cg_v2(const void* p) {  // L2 only: data oth
   asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
 }
+__device__ __forceinline__ uint2 ld_volatile_v2(const void* p) {  // re-read on every call
+  uint2 v;
+  asm volatile("ld.volatile.global.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
+  return v;
+}
+// bf16 negative zero in both halves: the mark of a mailbox slot element that its
+// producer has not written yet (a producer never stores negative zero).
+constexpr unsigned kNegZero2 = 0x80008000u;
+__device__ __forceinline__ bool has_neg_zero(const uint2 v) {
+  return (__vcmpeq2(v.x, kNegZero2) | __vcmpeq2(v.y, kNegZero2)) != 0u;
+}
+// Negative zero halves of a bf16 pair replaced by positive zero.
+__device__ __forceinline__ unsigned clear_neg_zero2(unsigned w) { return w & __vcmpne2(w, kNegZero2); }
 __device__ __forceinline__ void st_v2(void* p, uint2 v) {
   asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
@@ -237,7 +250,7 @@ __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// System scope: flags that other GPUs write (peer stores over NVLink) or read.
+// System scope: words that other GPUs write (peer stores over NVLink) or read.
 __device__ __forceinline__ unsigned ld_acquire_sys(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -108,8 +108,8 @@ def lib() -> ctypes.CDLL:
                                             _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
         "mhc_mailbox_bytes": (_sz, [_i, _i, _i]),
         "mhc_mailbox_init": (_i, [_vp, _sz, _vp]),
-        "mhc_mailbox_publish": (_i, [_vp, _i, ctypes.c_uint32, _vp, _i, _i, _i, _vp]),
-        "mhc_boundary_collect": (_i, [_vp, _i, ctypes.c_uint32, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
+        "mhc_mailbox_publish": (_i, [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _i, _i, _vp]),
+        "mhc_boundary_collect": (_i, [_vp, _i, _i, ctypes.c_uint32, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
                                       _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
         "mhc_ipc_handle_bytes": (_sz, []),
         "mhc_ipc_export": (_i, [_vp, _vp]),
@@ -325,32 +325,40 @@ def mhc_boundary_post_pre_ptrs(partial_ptrs, residual, post, comb, pre, norm_wei
     _check(st, "mhc_boundary_post_pre_ptrs")
 
 
-def mhc_mailbox_bytes(world: int, rows: int, hidden: int) -> int:
-    return int(lib().mhc_mailbox_bytes(world, rows, hidden))
+def mhc_mailbox_bytes(world: int, max_rows: int, hidden: int) -> int:
+    return int(lib().mhc_mailbox_bytes(world, max_rows, hidden))
 
 
-def new_mailbox(world: int, rows: int, hidden: int, device=None) -> torch.Tensor:
-    """A zeroed mailbox (uint8 device tensor) for a group of `world` producers."""
-    n = mhc_mailbox_bytes(world, rows, hidden)
+def mhc_mailbox_init(mailbox: torch.Tensor, stream=None):
+    """Header zero, every slot element negative zero ("not yet written")."""
+    _check(lib().mhc_mailbox_init(_p(mailbox), mailbox.numel(), _stream(stream)), "mhc_mailbox_init")
+
+
+def new_mailbox(world: int, max_rows: int, hidden: int, device=None, stream=None) -> torch.Tensor:
+    """An initialised mailbox (uint8 device tensor) for a group of `world`
+    producers and up to `max_rows` tokens a round."""
+    n = mhc_mailbox_bytes(world, max_rows, hidden)
     if n == 0:
         raise MhcError(UNSUPPORTED_SHAPE, "mhc_mailbox_bytes")
-    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+    mb = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    mhc_mailbox_init(mb, stream)
+    return mb
 
 
-def mhc_mailbox_publish(x: torch.Tensor, rank: int, round_: int, mailbox_ptrs, stream=None):
-    """Producer `rank`: store x [R, H] bf16 into slot [round & 1][rank] of every
-    consumer's mailbox (device addresses, rank order) and raise its row flags."""
+def mhc_mailbox_publish(x: torch.Tensor, rank: int, round_: int, mailbox_ptrs, max_rows: int, stream=None):
+    """Producer `rank`: store x [R, H] bf16 (R <= max_rows) into slot
+    [round & 1][rank] of every consumer's mailbox (device addresses, rank order)."""
     _need(x, torch.bfloat16, "x", 2)
     _contig(x, "x")
     ptrs = [int(a) for a in mailbox_ptrs]
     table = (ctypes.c_void_p * len(ptrs))(*ptrs)
     R, H = x.shape
-    _check(lib().mhc_mailbox_publish(_p(x), int(rank), int(round_), ctypes.cast(table, ctypes.c_void_p), len(ptrs),
-                                     R, H, _stream(stream)), "mhc_mailbox_publish")
+    _check(lib().mhc_mailbox_publish(_p(x), R, H, int(rank), int(round_), ctypes.cast(table, ctypes.c_void_p),
+                                     len(ptrs), int(max_rows), _stream(stream)), "mhc_mailbox_publish")
 
 
-def mhc_boundary_collect(mailbox, world: int, round_: int, residual, post, comb, pre, norm_weight, norm_eps,
-                         coeffs: Optional[Coeffs], residual_out, layer_input=None, mxfp8=None, post_out=None,
+def mhc_boundary_collect(mailbox, world: int, max_rows: int, round_: int, residual, post, comb, pre, norm_weight,
+                         norm_eps, coeffs: Optional[Coeffs], residual_out, layer_input=None, mxfp8=None, post_out=None,
                          comb_out=None, pre_out=None, workspace=None, stream=None, aux=None):
     """The consumer's boundary of round `round_` over the `world` slots of its mailbox
     (a tensor from new_mailbox, or a device address)."""
@@ -360,7 +368,7 @@ def mhc_boundary_collect(mailbox, world: int, round_: int, residual, post, comb,
     mb = mailbox.data_ptr() if isinstance(mailbox, torch.Tensor) else int(mailbox)
     cs, qs = _coeff_struct(coeffs), _mxfp8_struct(mxfp8)
     st = lib().mhc_boundary_collect(
-        mb, int(world), int(round_), _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight), float(norm_eps),
+        mb, int(world), int(max_rows), int(round_), _p(residual), _p(post), _p(comb), _p(pre), _p(norm_weight), float(norm_eps),
         _ref(cs), _p(residual_out), _p(aux), _p(layer_input), _ref(qs), _p(post_out), _p(comb_out), _p(pre_out),
         R, H, n, _p(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "mhc_boundary_collect")

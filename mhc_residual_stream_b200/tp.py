@@ -15,9 +15,10 @@ have read them (``barrier`` below is the plain host form of both). Nothing
 here uses multicast.
 
 PeerMailbox is the publish/collect form ([all_reduce] publish_target /
-mark_published): producers store their rows into every rank's mailbox and
-raise per-row generation flags; the boundary waits on its own mailbox's flags,
-so the group needs no barrier between a sublayer and the boundary.
+mark_published): producers store their rows, negative zero cleared, into every
+rank's mailbox, whose unwritten elements hold negative zero; each rank's
+boundary re-reads its own mailbox's elements until they are written, so the
+group needs no barrier between a sublayer and the boundary.
 """
 
 from __future__ import annotations
@@ -88,26 +89,28 @@ class PeerPartials:
 class PeerMailbox:
     """Publish/collect over the group: each rank's mailbox lives in its own memory
     and is mapped by every other rank; producers store their rows into every
-    mailbox and raise per-row flags, each rank's boundary waits on the flags of
-    its own mailbox (no host barrier between the sublayer and the boundary)."""
+    mailbox, and each rank's boundary reads the slots of its own mailbox as they
+    fill (an element is written once it is not negative zero), so no host barrier
+    sits between the sublayer and the boundary."""
 
-    def __init__(self, rows: int, hidden: int, group: Optional[dist.ProcessGroup] = None, device=None):
+    def __init__(self, max_rows: int, hidden: int, group: Optional[dist.ProcessGroup] = None, device=None):
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
-        self.local = M.new_mailbox(self.world, rows, hidden, device)
-        torch.cuda.current_stream(self.local.device).synchronize()  # zeroed before anyone maps it
+        self.max_rows = max_rows
+        self.local = M.new_mailbox(self.world, max_rows, hidden, device)
+        torch.cuda.current_stream(self.local.device).synchronize()  # initialised before anyone maps it
         gathered = exchange(M.ipc_export(self.local), tuple(self.local.shape), group)
         self.ptrs, self._imported = partial_table(self.rank, self.local.data_ptr(), gathered, M.ipc_import)
 
     def publish(self, x: torch.Tensor, round_: int, stream=None):
         """This rank's contribution of round `round_` into every rank's mailbox."""
-        M.mhc_mailbox_publish(x, self.rank, round_, self.ptrs, stream)
+        M.mhc_mailbox_publish(x, self.rank, round_, self.ptrs, self.max_rows, stream)
 
     def collect(self, round_: int, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out, **kw):
         """This rank's boundary of round `round_` over the group's contributions."""
-        M.mhc_boundary_collect(self.local, self.world, round_, residual, post, comb, pre, norm_weight, norm_eps,
-                               coeffs, residual_out, **kw)
+        M.mhc_boundary_collect(self.local, self.world, self.max_rows, round_, residual, post, comb, pre, norm_weight,
+                               norm_eps, coeffs, residual_out, **kw)
 
     def close(self):
         for a in self._imported:

@@ -4,13 +4,15 @@
   each round every producer publishes, then every consumer collects. Each
   collect must give bitwise the results of the strided entry over the same
   partials (the same sum order), over four rounds, so both parities are used
-  twice and the flow control of round t + 2 sees round t consumed.
-* The header words: after round t every flag of parity t & 1 reads t + 1 and the
-  parity's consumed word reads t + 1.
+  twice and the flow control of round t + 2 sees round t consumed; the row
+  count varies from round to round below the mailbox's capacity.
+* The mailbox words: after round t the consumed word of parity t & 1 reads
+  t + 1, and every slot element of both parities is back to negative zero.
+* A published negative zero arrives as positive zero.
 * A collect of a round nobody published runs out of its (shortened) wait and
   records MHC_ERR_DEVICE_TIMEOUT in the workspace; a publish two rounds ahead of
   a consumer runs out of its wait, writes nothing and records the timeout in the
-  producer's own mailbox. Both are waits on words that nothing sets.
+  producer's own mailbox. Both are waits on words that nothing writes.
 * Two processes on the same GPU form a gloo group of 2 and exchange mailboxes
   through CUDA IPC (PeerMailbox). Each round both publish, a host barrier
   follows, then both collect: every wait is satisfied when its kernel starts, so
@@ -33,21 +35,25 @@ from _parity import DEV, alloc_outputs, assert_bf16_close, check_tail, f64, gpu_
 
 pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = 256  # status word at byte 0, consumed words at bytes 8 and 12, then the flags
+HEADER = 256  # status word at byte 0, consumed words at bytes 8 and 12, then the slots
+NEG_ZERO = 0x8000
 
 
-def _header(mb: torch.Tensor, W: int, R: int):
-    """(consumed words [2], flags [2][W][R]) of a mailbox, read on the host."""
+def _consumed(mb: torch.Tensor):
     words = mb[:HEADER].cpu().view(torch.int32).numpy().view(np.uint32)
-    flags = mb[HEADER:HEADER + 2 * W * R * 4].cpu().view(torch.int32).numpy().view(np.uint32)
-    return words[2:4].copy(), flags.reshape(2, W, R).copy()
+    return words[2:4].copy()
 
 
-def _collect(mb, W, t, d, g, packed=False):
+def _slots(mb: torch.Tensor, W: int, M_: int, H: int) -> np.ndarray:
+    """The slot elements' bit patterns, [2][W][M][H] uint16."""
+    return mb[HEADER:].cpu().view(torch.int16).numpy().view(np.uint16).reshape(2, W, M_, H).copy()
+
+
+def _collect(mb, W, M_, t, d, g, packed=False):
     R, n, H = g["residual"].shape
     out = alloc_outputs(R, n, H)
     ws = M.new_workspace(R, H, n, DEV)
-    M.mhc_boundary_collect(mb, W, t, g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"],
+    M.mhc_boundary_collect(mb, W, M_, t, g["residual"], g["post"], g["comb"], g["pre"], g["norm_weight"],
                            d["norm_eps"], M.Coeffs.from_weights(d["coeff"], DEV, packed=packed),
                            out["residual_out"], layer_input=out["layer_input"],
                            mxfp8=(out["q_data"], out["q_scale"], True), post_out=out["post"], comb_out=out["comb"],
@@ -55,86 +61,112 @@ def _collect(mb, W, t, d, g, packed=False):
     return out, ws
 
 
-@pytest.mark.parametrize("R,H,n,W,packed", [(32, 7168, 4, 2, True), (7, 192, 2, 3, False),
-                                            (128, 512, 4, 16, False), (1, 64, 1, 1, False)])
-def test_rounds_match_strided_bitwise(R, H, n, W, packed):
+def _round_trip(mbs, W, M_, t, d, packed=False):
+    """Every producer publishes d's partials as round t, every consumer collects;
+    each consumer's results, compared bitwise with the strided entry."""
+    g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
+    xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
+    ptrs = [m.data_ptr() for m in mbs]
+    for u in range(W):
+        M.mhc_mailbox_publish(xs[u], u, t, ptrs, M_)
+    outs = [_collect(mbs[c], W, M_, t, d, g, packed) for c in range(W)]
+    torch.cuda.synchronize()
+    ref = gpu_post_pre(d, packed=packed)
+    for c, (out, ws) in enumerate(outs):
+        assert M.mhc_get_device_status(ws) == M.OK, (t, c)
+        for k, v in out.items():
+            assert torch.equal(v.cpu(), ref[k]), (t, c, k)
+
+
+@pytest.mark.parametrize("M_,H,n,W,packed,rows", [(32, 7168, 4, 2, True, (32, 32, 32, 32)),
+                                                  (8, 192, 2, 3, False, (7, 3, 8, 1)),
+                                                  (128, 512, 4, 16, False, (128, 5, 77, 128)),
+                                                  (1, 64, 1, 1, False, (1, 1, 1, 1))])
+def test_rounds_match_strided_bitwise(M_, H, n, W, packed, rows):
     from mhc_residual_stream_b200 import build
     build.build()
-    mbs = [M.new_mailbox(W, R, H, DEV) for _ in range(W)]
-    ptrs = [m.data_ptr() for m in mbs]
-    for t in range(4):
+    mbs = [M.new_mailbox(W, M_, H, DEV) for _ in range(W)]
+    torch.cuda.synchronize()
+    for c in range(W):
+        assert (_slots(mbs[c], W, M_, H) == NEG_ZERO).all() and (_consumed(mbs[c]) == 0).all()
+    for t, R in enumerate(rows):
         d = S.draw_boundary(R, H, n=n, partials=W, seed=7100 + 10 * t + W)
-        ref = gpu_post_pre(d, packed=packed)
-        g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
-        xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
-        for u in range(W):
-            M.mhc_mailbox_publish(xs[u], u, t, ptrs)
-        outs = [_collect(mbs[c], W, t, d, g, packed) for c in range(W)]
-        torch.cuda.synchronize()
-        for c, (out, ws) in enumerate(outs):
-            assert M.mhc_get_device_status(ws) == M.OK, (t, c)
-            for k, v in out.items():
-                assert torch.equal(v.cpu(), ref[k]), (t, c, k)
+        _round_trip(mbs, W, M_, t, d, packed)
         for c in range(W):
             assert M.mhc_get_device_status(mbs[c]) == M.OK  # no producer timed out
-            done, flags = _header(mbs[c], W, R)
+            done = _consumed(mbs[c])
             assert done[t & 1] == t + 1 and (t == 0 or done[(t - 1) & 1] == t), (t, c, done)
-            assert (flags[t & 1] == t + 1).all(), (t, c)
+            assert (_slots(mbs[c], W, M_, H) == NEG_ZERO).all(), (t, c)  # every read element re-marked
+
+
+def test_published_negative_zero_arrives_as_positive_zero():
+    R, H, n, W = 4, 128, 2, 2
+    d = S.draw_boundary(R, H, n=n, partials=W, seed=7150)
+    mbs = [M.new_mailbox(W, R, H, DEV) for _ in range(W)]
+    x = d["partials"][0].clone()
+    x[1, 5] = -0.0
+    x[2, :] = -0.0
+    # publish only producer 0; then inspect consumer 1's slot before anyone collects
+    M.mhc_mailbox_publish(x.to(DEV), 0, 0, [m.data_ptr() for m in mbs], R)
+    torch.cuda.synchronize()
+    slot = _slots(mbs[1], W, R, H)[0, 0]
+    want = x.view(torch.int16).numpy().view(np.uint16).copy()
+    want[want == NEG_ZERO] = 0
+    assert np.array_equal(slot, want)
+    assert (_slots(mbs[1], W, R, H)[0, 1] == NEG_ZERO).all()  # producer 1's slot untouched
+    # the round completes as the strided entry on the cleared partials
+    M.mhc_mailbox_publish(d["partials"][1].to(DEV).contiguous(), 1, 0, [m.data_ptr() for m in mbs], R)
+    d["partials"][0] = torch.from_numpy(want.view(np.int16)).view(torch.bfloat16)
+    g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
+    outs = [_collect(mbs[c], W, R, 0, d, g) for c in range(W)]
+    torch.cuda.synchronize()
+    ref = gpu_post_pre(d)
+    for out, ws in outs:
+        assert M.mhc_get_device_status(ws) == M.OK
+        for k, v in out.items():
+            assert torch.equal(v.cpu(), ref[k]), k
 
 
 def test_collect_of_unpublished_round_times_out_and_recovers():
     R, H, n, W = 4, 256, 4, 2
     d = S.draw_boundary(R, H, n=n, partials=W, seed=7201)
     g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
-    mb, other = M.new_mailbox(W, R, H, DEV), M.new_mailbox(W, R, H, DEV)
+    mbs = [M.new_mailbox(W, R, H, DEV) for _ in range(W)]
     old = M.mhc_debug_set_wait(20_000_000, 0)  # 20 ms
     try:
-        out, ws = _collect(mb, W, 0, d, g)
-        assert M.mhc_get_device_status(ws) == M.DEVICE_TIMEOUT
+        outs = [_collect(mbs[c], W, R, 0, d, g) for c in range(W)]
+        for out, ws in outs:
+            assert M.mhc_get_device_status(ws) == M.DEVICE_TIMEOUT
     finally:
         M.mhc_debug_set_wait(old, 0)
-    assert M.mhc_get_device_status(ws) == M.OK  # reading cleared it
-    # round 1 (the other parity) published and collected as usual
-    xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
-    for u in range(W):
-        M.mhc_mailbox_publish(xs[u], u, 1, [mb.data_ptr(), other.data_ptr()])
-    out, ws = _collect(mb, W, 1, d, g)
-    torch.cuda.synchronize()
-    assert M.mhc_get_device_status(ws) == M.OK
-    ref = gpu_post_pre(d)
-    for k, v in out.items():
-        assert torch.equal(v.cpu(), ref[k]), k
+    for c, (out, ws) in enumerate(outs):
+        assert M.mhc_get_device_status(ws) == M.OK  # reading cleared it
+        assert _consumed(mbs[c])[0] == 1 and (_slots(mbs[c], W, R, H) == NEG_ZERO).all()
+    # round 1 (the other parity), then round 2 (parity 0 again), go through as usual
+    for t in (1, 2):
+        _round_trip(mbs, W, R, t, d)
 
 
 def test_publish_ahead_of_consumer_times_out_and_writes_nothing():
     R, H, W = 3, 128, 2
     mbs = [M.new_mailbox(W, R, H, DEV) for _ in range(W)]
+    fresh = [m.clone() for m in mbs]
     x = torch.randn(R, H, device=DEV).to(torch.bfloat16)
     old = M.mhc_debug_set_wait(20_000_000, 0)
     try:
-        M.mhc_mailbox_publish(x, 0, 2, [m.data_ptr() for m in mbs])  # nobody consumed round 0
+        M.mhc_mailbox_publish(x, 0, 2, [m.data_ptr() for m in mbs], R)  # nobody consumed round 0
         torch.cuda.synchronize()
     finally:
         M.mhc_debug_set_wait(old, 0)
     assert M.mhc_get_device_status(mbs[0]) == M.DEVICE_TIMEOUT  # the producer's own mailbox
     assert M.mhc_get_device_status(mbs[1]) == M.OK
-    for m in mbs:
-        assert int(m.count_nonzero()) == 0  # no slot, flag or consumed word written
+    for m, f in zip(mbs, fresh):
+        assert torch.equal(m, f)  # no slot or consumed word written
     # once round 0 is consumed (here: published and collected), round 2 goes through
     d = S.draw_boundary(R, H, n=1, partials=W, seed=7301)
     d["partials"][0] = x.cpu()
-    g = to_dev({k: d[k] for k in ("residual", "post", "comb", "pre", "norm_weight")})
-    xs = [d["partials"][u].to(DEV).contiguous() for u in range(W)]
     for t in (0, 2):
-        for u in range(W):
-            M.mhc_mailbox_publish(xs[u], u, t, [m.data_ptr() for m in mbs])
-        outs = [_collect(mbs[c], W, t, d, g) for c in range(W)]
-        torch.cuda.synchronize()
-        ref = gpu_post_pre(d)
-        for out, ws in outs:
-            assert M.mhc_get_device_status(ws) == M.OK
-            for k, v in out.items():
-                assert torch.equal(v.cpu(), ref[k]), (t, k)
+        _round_trip(mbs, W, R, t, d)
     assert M.mhc_get_device_status(mbs[0]) == M.OK
 
 
@@ -160,7 +192,7 @@ def _rank(rank, world, port, q):
     try:
         torch.cuda.set_device(0)
         R, H, n = 16, 7168, 4
-        box = PeerMailbox(R, H, device="cuda:0")
+        box = PeerMailbox(R, H, device="cuda:0")  # capacity R
         for t in range(ROUNDS):
             d = S.draw_boundary(R, H, n=n, partials=world, seed=7400 + t)  # the same draw on both ranks
             x = d["partials"][rank].to("cuda:0").contiguous()  # this rank's sublayer output

@@ -159,27 +159,31 @@ def test_other_entry_points_host_checks(L):
     assert L.mhc_ipc_export(a, None) == M.INVALID_ARG
     assert L.mhc_ipc_import(None, None) == M.INVALID_ARG
     assert L.mhc_ipc_release(ctypes.c_void_p(0x12340)) == M.INVALID_ARG  # never imported
-    # mailbox: sizes (header 256, flags [2][W][R] rounded to 256, slots [2][W][R][H] bf16) and refusals
-    assert M.mhc_mailbox_bytes(2, 32, 7168) == 256 + 512 + 2 * 2 * 32 * 7168 * 2
-    assert M.mhc_mailbox_bytes(8, 128, 64) == 256 + 8192 + 2 * 8 * 128 * 64 * 2
+    # mailbox: sizes (header 256, slots [2][W][max_rows][H] bf16) and refusals
+    assert M.mhc_mailbox_bytes(2, 32, 7168) == 256 + 2 * 2 * 32 * 7168 * 2
+    assert M.mhc_mailbox_bytes(8, 128, 64) == 256 + 2 * 8 * 128 * 64 * 2
     for bad in ((0, 32, 7168), (17, 32, 7168), (2, 0, 7168), (2, 129, 7168), (2, 32, 100)):
         assert M.mhc_mailbox_bytes(*bad) == 0
     mbs = (ctypes.c_void_p * 2)(0x10000, 0x20000)
-    pub = L.mhc_mailbox_publish
-    assert pub(a, 2, 0, ctypes.cast(mbs, ctypes.c_void_p), 2, 4, 256, None) == M.INVALID_ARG  # rank >= world
-    assert pub(a, 0, 0xFFFFFFFF, ctypes.cast(mbs, ctypes.c_void_p), 2, 4, 256, None) == M.INVALID_ARG
-    assert pub(_fake(0x10008), 0, 0, ctypes.cast(mbs, ctypes.c_void_p), 2, 4, 256, None) == M.INVALID_ARG
-    assert pub(a, 0, 0, None, 2, 4, 256, None) == M.INVALID_ARG
-    assert pub(a, 0, 0, ctypes.cast(mbs, ctypes.c_void_p), 17, 4, 256, None) == M.UNSUPPORTED_SHAPE
+    tbl = ctypes.cast(mbs, ctypes.c_void_p)
+    pub = L.mhc_mailbox_publish  # (x, rows, hidden, rank, round, mailboxes, world, max_rows, stream)
+    assert pub(a, 4, 256, 2, 0, tbl, 2, 4, None) == M.INVALID_ARG  # rank >= world
+    assert pub(a, 4, 256, 0, 0xFFFFFFFF, tbl, 2, 4, None) == M.INVALID_ARG
+    assert pub(_fake(0x10008), 4, 256, 0, 0, tbl, 2, 4, None) == M.INVALID_ARG
+    assert pub(a, 4, 256, 0, 0, None, 2, 4, None) == M.INVALID_ARG
+    assert pub(a, 4, 256, 0, 0, tbl, 17, 4, None) == M.UNSUPPORTED_SHAPE
+    assert pub(a, 5, 256, 0, 0, tbl, 2, 4, None) == M.UNSUPPORTED_SHAPE  # rows > capacity
+    assert pub(a, 4, 100, 0, 0, tbl, 2, 4, None) == M.UNSUPPORTED_SHAPE
     bad_mbs = (ctypes.c_void_p * 2)(0x10000, 0x20080)  # a mailbox not 256-byte aligned
-    assert pub(a, 0, 0, ctypes.cast(bad_mbs, ctypes.c_void_p), 2, 4, 256, None) == M.INVALID_ARG
-    col = L.mhc_boundary_collect
-    assert col(_fake(0x10080), 2, 0, a, a, a, None, None, 0.0, None, a, None, None, None, None, None, None,
-               4, 256, 4, a, 1 << 20, None) == M.INVALID_ARG  # mailbox not 256-byte aligned
-    assert col(a, 0, 0, a, a, a, None, None, 0.0, None, a, None, None, None, None, None, None,
-               4, 256, 4, a, 1 << 20, None) == M.UNSUPPORTED_SHAPE
-    assert col(a, 2, 0, a, a, a, None, None, 0.0, None, a, None, None, None, None, None, None,
-               4, 256, 4, None, 0, None) == M.WORKSPACE  # the flag wait needs the status word
+    assert pub(a, 4, 256, 0, 0, ctypes.cast(bad_mbs, ctypes.c_void_p), 2, 4, None) == M.INVALID_ARG
+    col = L.mhc_boundary_collect  # (mailbox, world, max_rows, round, ... as post_pre_ptrs from residual on)
+    tail = (a, a, a, None, None, 0.0, None, a, None, None, None, None, None, None, 4, 256, 4)
+    assert col(_fake(0x10080), 2, 4, 0, *tail, a, 1 << 20, None) == M.INVALID_ARG  # not 256-byte aligned
+    assert col(a, 0, 4, 0, *tail, a, 1 << 20, None) == M.UNSUPPORTED_SHAPE
+    assert col(a, 2, 3, 0, *tail, a, 1 << 20, None) == M.UNSUPPORTED_SHAPE  # rows 4 > capacity 3
+    assert col(a, 2, 4, 0xFFFFFFFF, *tail, a, 1 << 20, None) == M.INVALID_ARG
+    assert col(a, 2, 4, 0, *tail, None, 0, None) == M.WORKSPACE  # the slot wait needs the status word
     assert L.mhc_mailbox_init(_fake(0x10010), 4096, None) == M.INVALID_ARG
+    assert L.mhc_mailbox_init(a, 4100, None) == M.INVALID_ARG  # not whole 16-byte units
     assert L.mhc_workspace_init(None, 4096, None) == M.WORKSPACE
     assert L.mhc_get_device_status(None, None) == M.WORKSPACE
