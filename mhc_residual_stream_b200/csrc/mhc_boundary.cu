@@ -111,8 +111,9 @@ struct Params {
   // embedding of the first layer (whose identity pre-mix selects it)
   const __nv_bfloat16* tail_streams;
   int tail_broadcast;
-  int tail_layer_blocks;  // tail blocks [0, this) write the layer input (at most G, or 0)
-  int tail_coeff_blocks;  // the next ones finish the coefficients of rows j, j + this, ...
+  int tail_layer_blocks;  // tail blocks that write the layer input (at most G, or 0)
+  int tail_coeff_blocks;  // tail blocks that finish the coefficients of rows j, j + this, ...
+  int tail_coeff_first;   // coefficient blocks take the tail's first block indices
   int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
   int64_t budget_ns;
 };
@@ -619,12 +620,16 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
 
 // Sinkhorn normalisation of an n x n matrix in one thread's registers: `iters`
 // times, each row divided by (its sum + eps), then each column by (its sum +
-// eps). For n = 4, eps rides in copies of column 0 (row sums) and row 0 (column
-// sums) made by a fused multiply-add from the previous step's scaling, instead
-// of an add on the dependency chain. Measured on this part, scalar code beats
-// packed f32x2 pairs, and neither sharing the matrix between lanes (a shuffle
-// costs about 27 cycles) nor taking a step's four reciprocals from one (batch
-// inversion) is faster.
+// eps). For n = 4 the matrix stays as it came, K, and the steps update scale
+// vectors, M = diag(a) K diag(b): a row step's denominator is a_j (K b)_j + eps,
+// so with al_j = 1 / a_j it becomes al_j <- (K b)_j + eps al_j and a_j = 1 / al_j
+// (columns likewise with be = 1 / b). eps rides in the first fused multiply-add
+// of each dot product, so a step is three dependent additions and a
+// reciprocal, with 28 instructions against 36 for scaling the matrix in place
+// (2,400 against 2,761 cycles for 20 iterations, measured on this part alone).
+// Scalar code beats packed f32x2 pairs here, and neither sharing the matrix
+// between lanes (a shuffle costs about 27 cycles) nor taking a step's four
+// reciprocals from one (batch inversion) is faster.
 template <int N>
 __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, float eps) {
   if constexpr (N == 1) {
@@ -653,28 +658,34 @@ __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, fl
     }
   } else {
     static_assert(N == 4, "hc_mult 1, 2 or 4");
-    float e0[4];  // column 0 plus eps: the row sums' eps
+    float a[4], b[4], al[4], be[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) e0[j] = M[j][0] + eps;
-    for (int it = 0; it < iters; ++it) {
-      float r[4], c0[4], c[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) r[j] = rcp_approx((e0[j] + M[j][1]) + (M[j][2] + M[j][3]));
-#pragma unroll
-      for (int i = 0; i < 4; ++i) c0[i] = fmaf(M[0][i], r[0], eps);  // row 0 plus eps: the column sums' eps
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) M[j][i] *= r[j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) c[i] = rcp_approx((c0[i] + M[1][i]) + (M[2][i] + M[3][i]));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) e0[j] = fmaf(M[j][0], c[0], eps);
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) M[j][i] *= c[i];
+    for (int k = 0; k < 4; ++k) {
+      a[k] = 1.f;
+      b[k] = 1.f;
+      al[k] = 1.f;
+      be[k] = 1.f;
     }
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // rows: al_j <- (K b)_j + eps al_j
+        const float q0 = fmaf(M[j][1], b[1], fmaf(M[j][0], b[0], eps * al[j]));
+        const float q1 = fmaf(M[j][3], b[3], M[j][2] * b[2]);
+        al[j] = q0 + q1;
+        a[j] = rcp_approx(al[j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // columns: be_i <- (K^T a)_i + eps be_i
+        const float q0 = fmaf(M[1][i], a[1], fmaf(M[0][i], a[0], eps * be[i]));
+        const float q1 = fmaf(M[3][i], a[3], M[2][i] * a[2]);
+        be[i] = q0 + q1;
+        b[i] = rcp_approx(be[i]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) M[j][i] = (a[j] * M[j][i]) * b[i];
   }
 }
 
@@ -734,11 +745,15 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rq = lane >> 3, vec = lane & 7;
 
-  if (static_cast<int>(blockIdx.x) < p.tail_layer_blocks) {
+  // block roles: coefficient blocks first or last in the grid (the first blocks
+  // are placed first, on the SMs the streaming kernel leaves free)
+  const int bid = blockIdx.x;
+  const int lbid = p.tail_coeff_first ? bid - p.tail_coeff_blocks : bid;
+  if (lbid >= 0 && lbid < p.tail_layer_blocks) {
     const int GT = (G + 3) >> 2;  // tasks per row
     const int T = R * GT;
     const int W = p.tail_layer_blocks * kWarps;
-    const int w0 = blockIdx.x * kWarps + warp;
+    const int w0 = lbid * kWarps + warp;
     LayerLoads<N> cur;
     if (w0 < T) {  // norm weights of the first task: weights, so before the wait
       const int g = (w0 % GT) * 4 + rq;
@@ -856,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
     // Coefficient rows jb, jb + CB, ...: in batches of up to kWarps rows, every
     // warp adds a share of each row's per-block records (fixed order) into a
     // slot, then warp s finishes row s of the batch: logits, sigmoid, Sinkhorn.
-    const int jb = blockIdx.x - p.tail_layer_blocks;
+    const int jb = p.tail_coeff_first ? bid : bid - p.tail_layer_blocks;
     const int CB = p.tail_coeff_blocks;
     if (tid < 3) cp_async4(scale_s + tid, p.scale + tid);  // weights: before the wait
     if (tid >= 32 && tid < 32 + C) cp_async4(base_s + tid - 32, p.base + (tid - 32));
@@ -932,9 +947,7 @@ __global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params
         if (s_comb >= 0) {
           // M = exp(L - max L) with one exp per lane, then Sinkhorn in one thread
           float lk = __shfl_sync(kFull, l, (lane + 2 * N) & 31);  // lane k < n*n: comb logit k
-          float mx = lk;
-#pragma unroll
-          for (int b = 1; b < NN; b <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, b));
+          const float mx = warp_max(lane < NN ? lk : -INFINITY);
           const float ek = expf(lk - mx);
           float lc[NN];
 #pragma unroll
@@ -1173,18 +1186,25 @@ mhc_status check_mxfp8(const mhc_mxfp8_out* q) {
 // Launch with programmatic stream serialization: the kernel may start while the
 // preceding kernel on the stream finishes, and waits for it (griddepcontrol.wait)
 // before reading anything that kernel may have written.
+// A carveout >= 0 sets this launch's preferred shared-memory share (percent).
 template <typename Kern>
-mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const Params& p, int threads = kThreads) {
+mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const Params& p, int threads = kThreads,
+                      int carveout = -1) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (carveout >= 0) {
+    attr[1].id = cudaLaunchAttributePreferredSharedMemoryCarveout;
+    attr[1].val.sharedMemCarveout = static_cast<unsigned>(carveout);
+    cfg.numAttrs = 2;
+  }
   if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return MHC_ERR_CUDA;
@@ -1209,6 +1229,20 @@ int sm_count() {
 // Raise a kernel's dynamic shared memory limit to 200 KB, once per device
 // (idempotent, so concurrent first calls only repeat the same setting).
 constexpr int kSmemLimit = 200 * 1024;
+
+// Placement of the tail's blocks. An SM changes its L1 / shared-memory split only
+// when it is empty, and the split the driver picks for the streaming kernel alone
+// (just above its shared memory) leaves no room for a tail block beside it. Up to
+// kCoexistRows rows the streaming kernel asks for the largest shared-memory split,
+// so tail blocks launch early on its SMs too, and from kCoeffFirstRows rows the
+// coefficient blocks take the first block indices, which land on the SMs the
+// streaming kernel leaves free. Measured on B200 (whole boundaries in CUDA graphs,
+// us per boundary): 7.84 against 8.26 at 32 rows, 6.84 against 7.05 at 16, 5.85
+// against 5.94 at 4; the largest split is slower from 48 rows on (10.23 against
+// 9.95 at 48, 11.6 against 10.9 at 64, 22.2 against 19.9 at 128), and at 2 rows
+// the coefficient blocks first are (6.20 against 6.07).
+constexpr int kCoexistRows = 32;
+constexpr int kCoeffFirstRows = 4;
 template <typename Kern>
 bool allow_smem(Kern kern, int bytes, std::atomic<int>* configured) {
   int dev = 0;
@@ -1230,7 +1264,9 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   p.extra_tx = g_extra_tx;
   p.budget_ns = g_budget_ns;
   const int G = p.H / kCols;
-  mhc_status st = launch_pdl(boundary_kernel<N, FRONT>, G, L.total, stream, p, kT1);
+  const bool few_rows = p.R <= kCoexistRows;
+  mhc_status st = launch_pdl(boundary_kernel<N, FRONT>, G, L.total, stream, p, kT1,
+                             few_rows ? static_cast<int>(cudaSharedmemCarveoutMaxShared) : -1);
   if (st != MHC_OK || !(p.do_layer || p.do_coeff)) return st;
   if (FRONT == kBroadcast) {
     p.tail_streams = p.x;
@@ -1246,6 +1282,7 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   p.tail_layer_blocks = p.do_layer ? (lb < G ? lb : G) : 0;
   const int spare = sm_count() - p.tail_layer_blocks;
   p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
+  p.tail_coeff_first = few_rows && p.R >= kCoeffFirstRows;
   return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>().total,
                     stream, p);
 }

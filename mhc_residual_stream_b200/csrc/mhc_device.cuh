@@ -122,6 +122,12 @@ __device__ __forceinline__ uint2 ld_cg_v2(const void* p) {  // L2 only: data oth
   asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
 }
+// Maximum over the warp in one instruction (sm_100a); NaN inputs are skipped, as by fmaxf.
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 __device__ __forceinline__ uint2 ld_volatile_v2(const void* p) {  // re-read on every call
   uint2 v;
   asm volatile("ld.volatile.global.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
