@@ -630,6 +630,12 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
 // Scalar code beats packed f32x2 pairs here, and neither sharing the matrix
 // between lanes (a shuffle costs about 27 cycles) nor taking a step's four
 // reciprocals from one (batch inversion) is faster.
+// Each denominator also gets the smallest normal float, added off the chain: a
+// row (or column) of K that is exactly zero (its logits some 100 or more below the
+// largest) would otherwise shrink its denominator by eps every step until it
+// underflows, and 1/0 times 0 is NaN where scaling in place gives 0. In fp32 the
+// term changes nothing unless the denominator is already below ~2e-31.
+constexpr float kTinyNormal = 1.17549435e-38f;  // 2^-126
 template <int N>
 __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, float eps) {
   if constexpr (N == 1) {
@@ -669,14 +675,14 @@ __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, fl
     for (int it = 0; it < iters; ++it) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {  // rows: al_j <- (K b)_j + eps al_j
-        const float q0 = fmaf(M[j][1], b[1], fmaf(M[j][0], b[0], eps * al[j]));
+        const float q0 = fmaf(M[j][1], b[1], fmaf(M[j][0], b[0], fmaf(eps, al[j], kTinyNormal)));
         const float q1 = fmaf(M[j][3], b[3], M[j][2] * b[2]);
         al[j] = q0 + q1;
         a[j] = rcp_approx(al[j]);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {  // columns: be_i <- (K^T a)_i + eps be_i
-        const float q0 = fmaf(M[1][i], a[1], fmaf(M[0][i], a[0], eps * be[i]));
+        const float q0 = fmaf(M[1][i], a[1], fmaf(M[0][i], a[0], fmaf(eps, be[i], kTinyNormal)));
         const float q1 = fmaf(M[3][i], a[3], M[2][i] * a[2]);
         be[i] = q0 + q1;
         b[i] = rcp_approx(be[i]);

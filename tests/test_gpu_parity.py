@@ -122,6 +122,27 @@ def test_sinkhorn_iteration_counts_and_eps():
         assert_coeffs_close(gpu, post, comb, pre, f"iters={iters}")
 
 
+@pytest.mark.parametrize("n", [4, 2])
+def test_sinkhorn_extreme_comb_logits(n):
+    # comb logits far apart, 50 iterations: one dominant entry, a row whose
+    # exp(L - max L) is exactly zero in fp32 (logits ~280 below the largest; in
+    # float64 it is ~1e-122), and an entry near e^-90 (a denormal in fp32)
+    d = S.draw_boundary(6, 256, n=n, partials=2, seed=4100 + n)
+    c = d["coeff"]
+    base = c.base.clone()
+    c0 = 2 * n
+    base[c0 + 0] = 30.0
+    base[c0 + 1 * n: c0 + 2 * n] = -250.0
+    base[c0 + n - 1] = -60.0
+    c.base = base
+    c.sinkhorn_iters = 50
+    gpu = gpu_post_pre(d)
+    assert np.isfinite(f64(gpu["comb"])).all()
+    post, comb, pre = O.mhc_coefficients(f64(gpu["residual_out"]), **coeff_np(c))
+    assert_coeffs_close(gpu, post, comb, pre, f"extreme comb logits, n={n}")
+    assert np.abs(f64(gpu["comb"])[:, 1, :]).max() <= 1e-5  # the vanishing row stays (near) zero
+
+
 # ---------------------------------------------------------------- MoE finalize
 
 def _moe_gpu(d, pre=True, mxfp8=False, coeff=True, ws=None, check_status=True, packed=False):
