@@ -23,6 +23,7 @@ group needs no barrier between a sublayer and the boundary.
 
 from __future__ import annotations
 
+import time
 from typing import List, Optional
 
 import torch
@@ -53,6 +54,55 @@ def partial_table(rank: int, local_ptr: int, gathered: List, import_fn):
             imported.append(a)
             table.append(a)
     return table, imported
+
+
+class PeerLost(RuntimeError):
+    """Peers of the group that did not reach a round in time (host-side check)."""
+
+    def __init__(self, ranks, round_):
+        super().__init__(f"ranks {sorted(ranks)} did not reach round {round_}")
+        self.ranks = sorted(ranks)
+        self.round = round_
+
+
+class Heartbeat:
+    """Host-side liveness of a group through a c10d store (the process group's by
+    default): each rank posts the last round it reached, and before work that
+    reads peers' memory a rank checks, with a time limit, that every peer has
+    reached a given round, raising PeerLost otherwise. A rank that died or left
+    is thus noticed on the host before the next launch instead of by a device
+    wait running out; nothing here touches the GPU."""
+
+    def __init__(self, rank: int, world: int, store=None, prefix: str = "mhc/heartbeat"):
+        self.store = store if store is not None else dist.distributed_c10d._get_default_store()
+        self.rank, self.world, self.prefix = rank, world, prefix
+
+    def _key(self, r: int) -> str:
+        return f"{self.prefix}/{r}"
+
+    def beat(self, round_: int):
+        """This rank has reached `round_`."""
+        self.store.set(self._key(self.rank), str(int(round_)))
+
+    def reached(self) -> List[int]:
+        """The last round every rank posted (-1 where none yet)."""
+        out = []
+        for r in range(self.world):
+            k = self._key(r)
+            out.append(int(self.store.get(k).decode()) if self.store.check([k]) else -1)
+        return out
+
+    def require(self, round_: int, timeout_s: float = 5.0, poll_s: float = 0.01):
+        """Wait until every peer has reached `round_`; PeerLost after `timeout_s`."""
+        deadline = time.monotonic() + timeout_s
+        while True:
+            seen = self.reached()
+            missing = [r for r in range(self.world) if r != self.rank and seen[r] < round_]
+            if not missing:
+                return
+            if time.monotonic() >= deadline:
+                raise PeerLost(missing, round_)
+            time.sleep(poll_s)
 
 
 class PeerPartials:
@@ -93,8 +143,10 @@ class PeerMailbox:
     fill (an element is written once it is not negative zero), so no host barrier
     sits between the sublayer and the boundary."""
 
-    def __init__(self, max_rows: int, hidden: int, group: Optional[dist.ProcessGroup] = None, device=None):
+    def __init__(self, max_rows: int, hidden: int, group: Optional[dist.ProcessGroup] = None, device=None,
+                 heartbeat: Optional[Heartbeat] = None):
         self.group = group
+        self.heartbeat = heartbeat
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.max_rows = max_rows
@@ -104,8 +156,14 @@ class PeerMailbox:
         self.ptrs, self._imported = partial_table(self.rank, self.local.data_ptr(), gathered, M.ipc_import)
 
     def publish(self, x: torch.Tensor, round_: int, stream=None):
-        """This rank's contribution of round `round_` into every rank's mailbox."""
+        """This rank's contribution of round `round_` into every rank's mailbox.
+        With a heartbeat: every peer must have reached the previous round (its
+        mailbox is still served), then this rank posts this one."""
+        if self.heartbeat is not None and round_ > 0:
+            self.heartbeat.require(round_ - 1)
         M.mhc_mailbox_publish(x, self.rank, round_, self.ptrs, self.max_rows, stream)
+        if self.heartbeat is not None:
+            self.heartbeat.beat(round_)
 
     def collect(self, round_: int, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out, **kw):
         """This rank's boundary of round `round_` over the group's contributions."""

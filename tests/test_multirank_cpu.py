@@ -113,3 +113,93 @@ def test_tp_partial_table_gloo(bad_shape):
         assert table == [0xABC0 if r == rank else 0x10000 * (r + 1) for r in range(world)]
         assert sorted(imported) == [r for r in range(world) if r != rank]
         assert mapped == [0x10000 * (r + 1) for r in range(world) if r != rank]
+
+
+# ---------------------------------------------------------------- failure detection on the host
+
+def _hb_worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from mhc_residual_stream_b200 import tp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    hb = tp.Heartbeat(rank, world)
+    try:
+        for t in range(3):
+            if t > 0:
+                hb.require(t - 1, timeout_s=10.0)
+            if rank == world - 1 and t == 2:
+                q.put((rank, "left", None))  # this rank stops between rounds
+                return
+            hb.beat(t)
+        try:
+            hb.require(2, timeout_s=1.0)
+            q.put((rank, "all reached", None))
+        except tp.PeerLost as e:
+            q.put((rank, "lost", (e.ranks, e.round)))
+        # the survivors end together (rank 0 hosts the store): a count on the store
+        import time
+        store = dist.distributed_c10d._get_default_store()
+        store.add("mhc/test/done", 1)
+        deadline = time.monotonic() + 30
+        while store.add("mhc/test/done", 0) < world - 1 and time.monotonic() < deadline:
+            time.sleep(0.01)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_heartbeat_names_a_rank_that_stopped():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_hb_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted((q.get(timeout=120) for _ in range(world)), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got[world - 1][1] == "left"
+    for rank, what, info in got[:world - 1]:
+        assert what == "lost" and info == ([world - 1], 2), (rank, what, info)
+
+
+def _late_worker(rank, world, port, q):
+    import datetime
+    import time
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from mhc_residual_stream_b200 import tp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=3))
+    try:
+        if rank == 1:
+            time.sleep(8)  # never joins the handle exchange
+            q.put((rank, "absent", 0.0))
+            return
+        t0 = time.monotonic()
+        try:
+            tp.exchange(bytes(72), (4, 64))
+            q.put((rank, "no error", time.monotonic() - t0))
+        except Exception as e:  # the group's timeout ends the collective with an error
+            q.put((rank, type(e).__name__, time.monotonic() - t0))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_exchange_errors_when_a_rank_never_joins():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_late_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted((q.get(timeout=120) for _ in range(2)), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+    rank0 = got[0]
+    assert rank0[1] != "no error" and rank0[2] < 30.0, rank0
