@@ -14,9 +14,10 @@
   a consumer runs out of its wait, writes nothing and records the timeout in the
   producer's own mailbox. Both are waits on words that nothing writes.
 * Two processes on the same GPU form a gloo group of 2 and exchange mailboxes
-  through CUDA IPC (PeerMailbox). Each round both publish, a host barrier
-  follows, then both collect: every wait is satisfied when its kernel starts, so
-  no kernel waits on another that runs at the same time.
+  through CUDA IPC (PeerMailbox, with a host heartbeat). Each round both
+  publish, a host barrier follows, then both collect: every wait is satisfied
+  when its kernel starts, so no kernel waits on another that runs at the same
+  time.
 """
 
 import datetime
@@ -185,14 +186,15 @@ def _rank(rank, world, port, q):
     sys.path.insert(0, ROOT)
     from mhc_residual_stream_b200 import mhc as M
     from mhc_residual_stream_b200 import synthetic as S
-    from mhc_residual_stream_b200.tp import PeerMailbox
+    from mhc_residual_stream_b200.tp import Heartbeat, PeerMailbox
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     box = None
     try:
         torch.cuda.set_device(0)
         R, H, n = 16, 7168, 4
-        box = PeerMailbox(R, H, device="cuda:0")  # capacity R
+        hb = Heartbeat(rank, world)  # each publish first requires the peer's previous round
+        box = PeerMailbox(R, H, device="cuda:0", heartbeat=hb)  # capacity R
         for t in range(ROUNDS):
             d = S.draw_boundary(R, H, n=n, partials=world, seed=7400 + t)  # the same draw on both ranks
             x = d["partials"][rank].to("cuda:0").contiguous()  # this rank's sublayer output
@@ -213,6 +215,7 @@ def _rank(rank, world, port, q):
             dist.barrier()  # round t consumed everywhere before anyone publishes round t + 1
             q.put((rank, t, st, pst, {k: v.cpu() for k, v in dict(residual_out=res_out, layer_input=li, post=post,
                                                                    comb=comb, pre=pre).items()}))
+        hb.require(ROUNDS - 1, timeout_s=10.0)  # every rank published every round
     finally:
         if box is not None:
             box.close()      # unmap the peer's mailbox ...
