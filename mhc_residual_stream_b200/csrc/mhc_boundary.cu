@@ -8,18 +8,22 @@
 //      bf16 terms, or fp32 that the block splits into bf16 terms) and the
 //      block's activations are prefetched into L2, both before the kernel waits
 //      for its predecessor on the stream;
-//   2. per (row, 4 columns) a lane sums the partials (or finalizes the MoE
-//      output), applies the mHC post-mix (vllm ...boundary.boundary,
-//      Boundaries.post_only: mhc_post(x, residual, post, comb)), rounds the new
-//      streams to bf16, stores them, sums the squares of their collapse with the
-//      carried pre (BoundaryState.pre) and of the streams;
+//   2. per (row, 4 columns) a lane sums the partials (local buffers, peers'
+//      buffers, or the slots of a publish/collect mailbox as they fill) or
+//      finalizes the MoE output, applies the mHC post-mix (vllm
+//      ...boundary.boundary, Boundaries.post_only: mhc_post(x, residual, post,
+//      comb)), rounds the new streams to bf16, stores them, sums the squares of
+//      their collapse with the carried pre (BoundaryState.pre) and of the streams;
 //   3. the block projects its rows' n*64 stream values onto the C fn columns on
-//      the tensor cores (mma.sync bf16, fn as three bf16 terms) and writes its
-//      partial sums to the workspace.
+//      the tensor cores (mma.sync bf16, fn as three bf16 terms; single or paired
+//      16-row tiles per warp by row count) and writes its partial sums to the
+//      workspace.
 // The tail kernel (boundary_tail_kernel), once the streaming kernel is done:
 //   4. layer-input blocks normalise 256-column tasks of the rows into the layer
-//      input (and MXFP8); beside them, coefficient blocks finish the rows'
-//      coefficients (logits, sigmoid, Sinkhorn in one thread per row).
+//      input (and MXFP8); beside them, coefficient blocks (placed first for 4-32
+//      rows, so that they start on the SMs the streaming kernel leaves free)
+//      finish the rows' coefficients (logits, sigmoid, Sinkhorn on scale vectors
+//      in one thread per row).
 // The residual-only variant is the streaming kernel alone. All reductions run
 // in a fixed order, so results are bitwise reproducible.
 
