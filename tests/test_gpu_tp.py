@@ -14,7 +14,6 @@ import os
 import socket
 import sys
 
-import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
