@@ -76,9 +76,14 @@ class Heartbeat:
     def __init__(self, rank: int, world: int, store=None, prefix: str = "mhc/heartbeat"):
         self.store = store if store is not None else dist.distributed_c10d._get_default_store()
         self.rank, self.world, self.prefix = rank, world, prefix
+        self.epoch = 0  # advanced by every rank together when rounds restart
 
     def _key(self, r: int) -> str:
-        return f"{self.prefix}/{r}"
+        return f"{self.prefix}/{self.epoch}/{r}"
+
+    def next_epoch(self):
+        """Rounds restart at 0 (every rank calls this at the same point)."""
+        self.epoch += 1
 
     def beat(self, round_: int):
         """This rank has reached `round_`."""
@@ -136,12 +141,24 @@ class PeerPartials:
                                      residual_out, **kw)
 
 
+def _sync(device):
+    """Wait for the work queued on `device` (nothing to wait for off the GPU)."""
+    if torch.device(device).type == "cuda":
+        torch.cuda.current_stream(device).synchronize()
+
+
 class PeerMailbox:
     """Publish/collect over the group: each rank's mailbox lives in its own memory
     and is mapped by every other rank; producers store their rows into every
     mailbox, and each rank's boundary reads the slots of its own mailbox as they
     fill (an element is written once it is not negative zero), so no host barrier
-    sits between the sublayer and the boundary."""
+    sits between the sublayer and the boundary.
+
+    Rounds are checked on the host before anything is launched ([all_reduce]
+    mark_published / reset keep the same kind of state): this rank publishes
+    rounds 0, 1, 2, ... in order, at most one round ahead of its collects, and
+    collects only a round it has published, in order. `reset` drops what an
+    aborted step left behind, on every rank of the group together."""
 
     def __init__(self, max_rows: int, hidden: int, group: Optional[dist.ProcessGroup] = None, device=None,
                  heartbeat: Optional[Heartbeat] = None):
@@ -151,24 +168,50 @@ class PeerMailbox:
         self.world = dist.get_world_size(group)
         self.max_rows = max_rows
         self.local = M.new_mailbox(self.world, max_rows, hidden, device)
-        torch.cuda.current_stream(self.local.device).synchronize()  # initialised before anyone maps it
+        _sync(self.local.device)  # initialised before anyone maps it
         gathered = exchange(M.ipc_export(self.local), tuple(self.local.shape), group)
         self.ptrs, self._imported = partial_table(self.rank, self.local.data_ptr(), gathered, M.ipc_import)
+        self.published = -1  # the last round this rank published
+        self.collected = -1  # the last round this rank collected
 
     def publish(self, x: torch.Tensor, round_: int, stream=None):
         """This rank's contribution of round `round_` into every rank's mailbox.
         With a heartbeat: every peer must have reached the previous round (its
         mailbox is still served), then this rank posts this one."""
+        if round_ != self.published + 1:
+            raise RuntimeError(f"round {round_} published out of order (last published {self.published})")
+        if round_ > self.collected + 2:
+            raise RuntimeError(f"round {round_} published while round {self.collected + 1} is still uncollected "
+                               "(a mailbox holds two rounds)")
         if self.heartbeat is not None and round_ > 0:
             self.heartbeat.require(round_ - 1)
         M.mhc_mailbox_publish(x, self.rank, round_, self.ptrs, self.max_rows, stream)
+        self.published = round_
         if self.heartbeat is not None:
             self.heartbeat.beat(round_)
 
     def collect(self, round_: int, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out, **kw):
         """This rank's boundary of round `round_` over the group's contributions."""
+        if round_ != self.collected + 1 or round_ > self.published:
+            raise RuntimeError(f"round {round_} collected out of order (last collected {self.collected}, "
+                               f"last published {self.published})")
         M.mhc_boundary_collect(self.local, self.world, self.max_rows, round_, residual, post, comb, pre, norm_weight,
                                norm_eps, coeffs, residual_out, **kw)
+        self.collected = round_
+
+    def reset(self, stream=None):
+        """Drop the rounds an aborted step left published but uncollected: every
+        rank of the group calls this together; afterwards rounds restart at 0.
+        The group first finishes the work it has queued (no producer may still
+        be storing into a mailbox), then each rank re-initialises its own."""
+        _sync(self.local.device)
+        dist.barrier(group=self.group)
+        M.mhc_mailbox_init(self.local, stream)
+        _sync(self.local.device)
+        dist.barrier(group=self.group)
+        self.published = self.collected = -1
+        if self.heartbeat is not None:
+            self.heartbeat.next_epoch()
 
     def close(self):
         for a in self._imported:

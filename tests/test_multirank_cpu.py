@@ -203,3 +203,47 @@ def test_exchange_errors_when_a_rank_never_joins():
         p.join(timeout=60)
     rank0 = got[0]
     assert rank0[1] != "no error" and rank0[2] < 30.0, rank0
+
+
+# ---------------------------------------------------------------- mailbox rounds (host logic)
+
+def test_peer_mailbox_round_checks_and_reset(monkeypatch):
+    # one gloo rank in this process; the library calls are replaced by recorders,
+    # so only the host bookkeeping runs
+    import torch
+    import torch.distributed as dist
+    from mhc_residual_stream_b200 import mhc as M
+    from mhc_residual_stream_b200 import tp
+    calls = []
+    monkeypatch.setattr(M, "new_mailbox", lambda W, R, H, device=None: torch.zeros(64, dtype=torch.uint8))
+    monkeypatch.setattr(M, "ipc_export", lambda t: bytes(72))
+    monkeypatch.setattr(M, "mhc_mailbox_publish", lambda x, rank, r, ptrs, mr, stream=None: calls.append(("pub", r)))
+    monkeypatch.setattr(M, "mhc_boundary_collect", lambda mb, W, mr, r, *a, **k: calls.append(("col", r)))
+    monkeypatch.setattr(M, "mhc_mailbox_init", lambda mb, stream=None: calls.append(("init",)))
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        hb = tp.Heartbeat(0, 1)
+        box = tp.PeerMailbox(4, 64, heartbeat=hb)
+        x, args = torch.zeros(4, 64), (None,) * 8
+        box.publish(x, 0)
+        box.publish(x, 1)
+        with pytest.raises(RuntimeError):
+            box.publish(x, 2)          # rounds 0 and 1 both uncollected: the mailbox holds two
+        with pytest.raises(RuntimeError):
+            box.collect(1, *args)      # round 0 first
+        box.collect(0, *args)
+        box.publish(x, 2)
+        with pytest.raises(RuntimeError):
+            box.publish(x, 4)          # round 3 skipped
+        box.collect(1, *args)
+        box.collect(2, *args)
+        with pytest.raises(RuntimeError):
+            box.collect(3, *args)      # not published by this rank
+        assert hb.reached() == [2]
+        box.reset()                    # an aborted step: rounds restart at 0
+        assert hb.epoch == 1 and hb.reached() == [-1]
+        box.publish(x, 0)
+        assert calls == [("pub", 0), ("pub", 1), ("col", 0), ("pub", 2), ("col", 1), ("col", 2), ("init",),
+                         ("pub", 0)]
+    finally:
+        dist.destroy_process_group()
