@@ -17,7 +17,8 @@
   through CUDA IPC (PeerMailbox, with a host heartbeat). Each round both
   publish, a host barrier follows, then both collect: every wait is satisfied
   when its kernel starts, so no kernel waits on another that runs at the same
-  time.
+  time. After three rounds the group resets and replays round 0, which must
+  give bitwise the first round 0.
 """
 
 import datetime
@@ -195,7 +196,10 @@ def _rank(rank, world, port, q):
         R, H, n = 16, 7168, 4
         hb = Heartbeat(rank, world)  # each publish first requires the peer's previous round
         box = PeerMailbox(R, H, device="cuda:0", heartbeat=hb)  # capacity R
-        for t in range(ROUNDS):
+        for step in range(ROUNDS + 1):
+            if step == ROUNDS:
+                box.reset()  # as after an aborted step: rounds restart at 0
+            t = step % ROUNDS
             d = S.draw_boundary(R, H, n=n, partials=world, seed=7400 + t)  # the same draw on both ranks
             x = d["partials"][rank].to("cuda:0").contiguous()  # this rank's sublayer output
             box.publish(x, t)
@@ -213,9 +217,9 @@ def _rank(rank, world, port, q):
             torch.cuda.synchronize()
             st, pst = M.mhc_get_device_status(ws), M.mhc_get_device_status(box.local)
             dist.barrier()  # round t consumed everywhere before anyone publishes round t + 1
-            q.put((rank, t, st, pst, {k: v.cpu() for k, v in dict(residual_out=res_out, layer_input=li, post=post,
-                                                                   comb=comb, pre=pre).items()}))
-        hb.require(ROUNDS - 1, timeout_s=10.0)  # every rank published every round
+            q.put((rank, step, st, pst, {k: v.cpu() for k, v in dict(residual_out=res_out, layer_input=li,
+                                                                      post=post, comb=comb, pre=pre).items()}))
+        hb.require(0, timeout_s=10.0)  # every rank published round 0 again
     finally:
         if box is not None:
             box.close()      # unmap the peer's mailbox ...
@@ -230,7 +234,7 @@ def test_two_processes_publish_and_collect_through_ipc():
     procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    got = [q.get(timeout=240) for _ in range(2 * ROUNDS)]
+    got = [q.get(timeout=240) for _ in range(2 * (ROUNDS + 1))]
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -246,3 +250,6 @@ def test_two_processes_publish_and_collect_through_ipc():
             check_tail(d, dict(res), orc, mxfp8=False, what=f"round {t} rank {rank}")
         for k in by_round[t][0]:  # both ranks computed the same boundary
             assert torch.equal(by_round[t][0][k], by_round[t][1][k]), (t, k)
+    for rank in range(2):  # round 0 after the reset: bitwise the first round 0
+        for k, v in by_round[ROUNDS][rank].items():
+            assert torch.equal(v, by_round[0][rank][k]), (rank, k)
