@@ -3,15 +3,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-sweep]
 
-A step is one decode attention-side boundary at rows=32, H=7168, hc_mult=4 with
-8 bf16 TP-partials, an MXFP8 layer input (swizzled 128x4 scales) and the next
-coefficients (20 Sinkhorn iterations): the partial sum, post-mix, collapse +
-RMSNorm + MXFP8 and coefficient steps of the boundary in one launch. Inputs are
-seeded synthetic tensors of that shape, resident in HBM; enough distinct buffer
-sets (inputs, weights and outputs; 27 sets, ~0.29 GB, at rows 32) to exceed
-twice the 126 MB L2 are
-rotated so that every step reads HBM, not L2. Steps are replayed from CUDA
-graphs and timed with CUDA events on the launching stream; the metric is
+A boundary is one decode attention-side boundary at rows=32, H=7168,
+hc_mult=4 with 8 bf16 TP-partials, an MXFP8 layer input (swizzled 128x4
+scales) and the next coefficients (20 Sinkhorn iterations): the partial sum,
+post-mix, collapse + RMSNorm + MXFP8 and coefficient steps in one launch. A
+step is one replay of a CUDA graph of 240 such boundaries, one after the other
+on one stream, over enough distinct buffer sets (inputs, weights and outputs;
+27 sets, ~0.29 GB, at rows 32) that each set is touched again only after more
+than twice the 126 MB L2 of other traffic: every boundary reads HBM, not L2.
+Steps are timed with CUDA events on the launching stream; the metric is
 microseconds per boundary (lower is better) and the achieved HBM GB/s of the
 algorithmic bytes (each input read once, each output written once).
 
@@ -153,9 +153,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
-# fn is packed once, at weight-load time, into the projection's bf16-term tiles
-# (mhc_projection_pack); --unpacked-fn times the kernels splitting fp32 fn per call
-PACK_FN = True
+# fn is passed as fp32 (the kernels split it into bf16 terms before they wait for
+# their predecessor); --packed-fn times the form packed once at weight load
+# (mhc_projection_pack), 1.34x the bytes of fp32 fn at hc_mult 4
+PACK_FN = False
 
 
 class BoundarySet:
@@ -207,21 +208,19 @@ def capture(fn, n):
     return g
 
 
-def timed_graph_steps(sets, ws, steps, warmup, graph_len=240):
-    """Run `warmup` then time `steps` boundaries (rotating over `sets`) from CUDA graphs;
-    returns elapsed ms of the timed region on the launching stream."""
+GRAPH_LEN = 240  # boundaries per step (one graph replay)
+
+
+def step_graph(sets, ws, graph_len=GRAPH_LEN):
+    """The step: a CUDA graph of graph_len boundaries rotating over `sets`."""
     nset = len(sets)
-    main = capture(lambda i: sets[i % nset].launch(ws), graph_len)
-    tail_len = steps % graph_len
-    tail = capture(lambda i: sets[i % nset].launch(ws), tail_len) if tail_len else None
-    wgraph = capture(lambda i: sets[i % nset].launch(ws), max(1, min(warmup, graph_len)))
-    for _ in range(max(1, (warmup + graph_len - 1) // graph_len)):
-        wgraph.replay()
-    torch.cuda.synchronize()
-    return main, tail
+    return capture(lambda i: sets[i % nset].launch(ws), graph_len)
 
 
-def run_timed(main, tail, steps, graph_len, sampler=None):
+def run_timed(graph, steps, warmup, sampler=None):
+    """`warmup` untimed replays, then the elapsed ms of `steps` replays on the launching stream."""
+    for _ in range(warmup):
+        graph.replay()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     if sampler:
@@ -229,10 +228,8 @@ def run_timed(main, tail, steps, graph_len, sampler=None):
         time.sleep(0.3)
     torch.cuda._sleep(2_000_000)  # keep the GPU busy while the replays are queued behind the start event
     start.record()
-    for _ in range(steps // graph_len):
-        main.replay()
-    if tail is not None:
-        tail.replay()
+    for _ in range(steps):
+        graph.replay()
     end.record()
     torch.cuda.synchronize()
     if sampler:
@@ -294,8 +291,8 @@ def cpu_baseline(budget_s=12.0):
     d = S.draw_boundary(ROWS, HIDDEN, n=HC, partials=PARTIALS, seed=2032)
     f = {k: d[k].double().numpy() for k in ("partials", "residual", "post", "comb", "pre", "norm_weight")}
     cw = {k: (v.double().numpy() if isinstance(v, torch.Tensor) else v) for k, v in d["coeff"].as_dict().items()}
-    info = threadpoolctl.threadpool_info()
-    cores = max([i.get("num_threads", 1) for i in info] + [1])
+    cores = len(os.sched_getaffinity(0))
+    blas = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
     times = []
     t_end = time.perf_counter() + budget_s
     while True:
@@ -320,7 +317,8 @@ def cpu_baseline(budget_s=12.0):
     return {"value": round(us, 1), "unit": "µs/boundary", "cores": cores, "kind": "oracle",
             "single_thread_value": round(statistics.median(one) * 1e6, 1),
             "sample": f"{len(times)} full boundaries (rows 32, H 7168, n 4, P 8, MXFP8, coefficients), median; "
-                      f"numpy float64, BLAS threads {cores}; single_thread_value: {len(one)} more on 1 thread"}
+                      f"numpy float64 on {cores} available cores (BLAS threads {blas}); single_thread_value: "
+                      f"{len(one)} more on 1 thread"}
 
 
 def dist_setup(args):
@@ -375,30 +373,33 @@ def ours(args):
                     (s.partials, s.residual, s.coeffs.fn if s.coeffs.fn is not None else s.coeffs.fn_packed,
                      s.residual_out, s.layer_input, s.q_data))
     assert set_bytes * nsets > 2 * L2_BYTES
-    graph_len = 240
-    main, tail = timed_graph_steps(sets, ws, args.steps, args.warmup, graph_len)
+    graph = step_graph(sets, ws)
     sampler = ClockSampler(device) if rank == 0 else None
     barrier(world)
-    ms = run_timed(main, tail, args.steps, graph_len, sampler)
+    ms = run_timed(graph, args.steps, args.warmup, sampler)
     ms = max_over_ranks(ms, world)
     st = M.mhc_get_device_status(ws)
     if st != M.OK:
         raise RuntimeError(f"device status {M.STATUS_NAMES[st]}")
-    us_per = aggregate_us_per_boundary(ms, args.steps, world)
-    us_kernel = ms * 1000.0 / args.steps                 # per launch on one GPU
+    boundaries = args.steps * GRAPH_LEN
+    us_per = aggregate_us_per_boundary(ms, boundaries, world)
+    us_kernel = ms * 1000.0 / boundaries                 # per launch on one GPU
     bpb = boundary_bytes(ROWS)
     achieved = bpb / (us_kernel * 1e-6) / 1e9
 
     result = {
         "metric": METRIC, "value": round(us_per, 4), "unit": "µs/boundary", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 7),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; decode attention-side boundary inputs, no trained weights)",
         "config": {"workload": "decode attention-side boundary: rows 32, H 7168, hc_mult 4, 8 bf16 partials, "
                                "MXFP8 layer input (swizzled 128x4), coefficients with 20 Sinkhorn iterations",
                    "rows": ROWS, "hidden": HIDDEN, "hc_mult": HC, "partials": PARTIALS,
-                   "l2": f"inputs larger than L2: {nsets} rotating buffer sets, {set_bytes * nsets / 1e6:.0f} MB",
-                   "timing": "CUDA graphs of 240 boundaries, CUDA events on the launching stream",
+                   "step": f"one CUDA-graph replay of {GRAPH_LEN} boundaries on one stream "
+                           f"({boundaries} boundaries timed)",
+                   "l2": f"inputs larger than L2: {nsets} rotating buffer sets, {set_bytes * nsets / 1e6:.0f} MB; "
+                         "a set is reused only after more than twice the L2 size of other traffic",
+                   "timing": "CUDA events on the launching stream around the timed replays",
                    "fn": ("packed once at weight load (mhc_projection_pack)" if PACK_FN
                           else "fp32, split into bf16 terms in every call"),
                    "parallelism": f"replicas x{world}"},
@@ -407,16 +408,16 @@ def ours(args):
                      "frac": round(achieved / peak, 4), "frac_of_nominal_8000": round(achieved / 8000.0, 4),
                      "traffic": load_traffic(),
                      "algorithmic_bytes": bpb, "peak_kind": f"{peak_kind} (copy bandwidth)",
-                     "kernel": "boundary_kernel<4, partials> + boundary_tail_kernel<4>: the two launches "
-                               "of one boundary, timed together; traffic is the streaming kernel's "
-                               "DRAM bytes per launch (the tail reads L2)"},
-        "gpu_launches": 2 * args.steps,
+                     "kernel": "boundary_kernel<4, partials>: the one launch of a boundary; achieved = "
+                               "algorithmic bytes / CUDA-event time per launch; traffic = its DRAM bytes "
+                               "per launch (ncu)"},
+        "gpu_launches": boundaries,
     }
     if sampler is not None:
         result["clocks"] = sampler.summary()
     lf = launch_floor_us()
-    result["launch_floor"] = {"us_per_kernel": round(lf, 3), "kernels_per_boundary": 2,
-                              "us_per_boundary": round(2 * lf, 3),
+    result["launch_floor"] = {"us_per_kernel": round(lf, 3), "kernels_per_boundary": 1,
+                              "us_per_boundary": round(lf, 3),
                               "how": "CUDA graph of 240 empty kernels (torch.cuda._sleep(0)), median of 20 replays"}
 
     if not args.no_sweep:
@@ -424,14 +425,16 @@ def ours(args):
         for R in (1, 2, 4, 8, 16, 32, 64, 128):
             ss = [BoundarySet(R, 800000 + 131 * i + R, device) for i in range(sets_for(R))]
             wsr = M.new_workspace(R, HIDDEN, HC, device)
-            n = min(args.steps, 24000) // graph_len * graph_len or graph_len
-            m, t = timed_graph_steps(ss, wsr, n, 2 * graph_len, graph_len)
-            msr = run_timed(m, t, n, graph_len)
-            us = msr * 1000.0 / n
+            gr = step_graph(ss, wsr)
+            reps = max(3, min(args.steps, 100))
+            msr = run_timed(gr, reps, 3)
+            if M.mhc_get_device_status(wsr) != M.OK:
+                raise RuntimeError(f"rows {R}: device status")
+            us = msr * 1000.0 / (reps * GRAPH_LEN)
             gbs = boundary_bytes(R) / (us * 1e-6) / 1e9
             sweep[str(R)] = {"us": round(us, 3), "gb_per_s": round(gbs, 1), "frac": round(gbs / peak, 4),
                              "algorithmic_bytes": boundary_bytes(R), "sets": len(ss)}
-            del ss, m, t
+            del ss, gr
         result["rows_sweep"] = sweep
         # one decode step: the 123 chained boundaries of the 61-layer loop at rows 32
         from mhc_residual_stream_b200.decode import DecodeLoop
@@ -456,7 +459,7 @@ def ours(args):
         if M.mhc_get_device_status(loop.workspace) != M.OK:
             raise RuntimeError("decode loop device status")
 
-    e2e_us, h2d, d2h = e2e_time(sets[0], ws, min(200, max(10, args.steps // 100)), device)
+    e2e_us, h2d, d2h = e2e_time(sets[0], ws, min(200, max(10, args.steps)), device)
     e2e_us = max_over_ranks(e2e_us, world) / world
     result["e2e"] = {"value": round(e2e_us, 2), "unit": "µs/boundary", "h2d_bytes_per_step": h2d,
                      "d2h_bytes_per_step": d2h}
@@ -499,7 +502,7 @@ def reference(args):
             break
     el = time.perf_counter() - t0
     us = el * 1e6 / done
-    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    cores = len(os.sched_getaffinity(0))
     sample = (f"{done} of {args.steps} requested boundaries timed (bounded at {budget:.0f} s); "
               "full rows-32 boundary each")
     print(json.dumps({
@@ -519,16 +522,16 @@ def reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=240000)
-    ap.add_argument("--warmup", type=int, default=2400)
+    ap.add_argument("--steps", type=int, default=100, help=f"timed steps (graph replays of {GRAPH_LEN} boundaries)")
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rows sweep and the decode-loop step")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--unpacked-fn", action="store_true",
-                    help="pass fp32 fn (split into bf16 terms in every call) instead of the packed form")
+    ap.add_argument("--packed-fn", action="store_true",
+                    help="pass fn packed at weight load (mhc_projection_pack) instead of fp32 fn")
     args = ap.parse_args()
     global PACK_FN
-    PACK_FN = not args.unpacked_fn
+    PACK_FN = args.packed_fn
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

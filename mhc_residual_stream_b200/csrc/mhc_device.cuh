@@ -1,6 +1,7 @@
 // Device helpers of the mHC boundary kernels (sm_100a): PTX wrappers for the
-// bulk-copy engine and mbarriers, bf16 packing, bounded waits, and the
-// E8M0/E4M3 encoders of the MXFP8 layer input.
+// bulk-copy and tensor-map TMA engine, mbarriers, the warp-level tensor-core
+// MMA, thread-block clusters, tagged words between CTAs, bf16 packing, bounded
+// waits, and the E8M0/E4M3 encoders of the MXFP8 layer input.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -24,8 +25,9 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
+// The first error of a launch wins; a null status (a call without a workspace) records nothing.
 __device__ __forceinline__ void record_error(unsigned* status, unsigned code) {
-  atomicCAS(status, 0u, code);
+  if (status != nullptr) atomicCAS(status, 0u, code);
 }
 
 // ---------------------------------------------------------------- shared memory / TMA bulk copies
@@ -162,6 +164,51 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                : "memory");
 }
 
+// ---------------------------------------------------------------- tensor-map TMA loads (no multicast)
+
+// Tiled tensor-map loads into this CTA's shared memory; completion is counted in
+// bytes on `bar` (the full box, out-of-range elements filled with zeros).
+// `map` is the address of a __grid_constant__ kernel parameter.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Four rows y0..y3 of a 2-D tensor map whose box is one row high, columns
+// [x, x + box width), landed as four consecutive box rows at dst.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* map, int x, int y0, int y1, int y2, int y3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Fetch a tensor map (a __grid_constant__ kernel parameter) ahead of its first use.
+__device__ __forceinline__ void prefetch_tensormap(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Generic-proxy writes to shared memory made visible to the async proxy (the
+// tensor cores and the TMA engine) before they read them.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ---------------------------------------------------------------- warp-level tensor core MMA
 
 // Four 8x8 b16 matrices from shared memory; lane l gives the row address of
@@ -187,6 +234,46 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const unsigned (&a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
+
+// ---------------------------------------------------------------- thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// Address of the same shared-memory byte in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// ---------------------------------------------------------------- tagged words between CTAs
+
+// A value and the tag of the launch that wrote it, as one 64-bit word: a
+// reader that sees the expected tag has the value written with it (a 64-bit
+// access is single-copy atomic), with no flag and no fence between them.
+__device__ __forceinline__ void st_tagged(unsigned long long* p, uint32_t tag, float v) {
+  const unsigned long long w = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+__device__ __forceinline__ uint32_t tag_of(unsigned long long w) { return static_cast<uint32_t>(w >> 32); }
+__device__ __forceinline__ float value_of(unsigned long long w) { return __uint_as_float(static_cast<uint32_t>(w)); }
 
 // ---------------------------------------------------------------- bf16 packing
 

@@ -24,3 +24,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The 1-ulp bf16 flips the parity checks counted (GPU runs only)."""
+    mod = sys.modules.get("_parity")
+    flips = getattr(mod, "FLIPS", None) if mod else None
+    if not flips:
+        return
+    total = sum(f for _, f, _ in flips)
+    elems = sum(n for _, _, n in flips)
+    worst = max(flips, key=lambda t: t[1] / max(t[2], 1))
+    terminalreporter.write_line(
+        f"bf16 ulp checks: {len(flips)} arrays, {total} one-ulp flips in {elems} elements "
+        f"({total / max(elems, 1):.2e}); largest share {worst[1]}/{worst[2]} in {worst[0]}")

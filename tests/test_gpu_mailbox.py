@@ -9,8 +9,10 @@
 * The mailbox words: after round t the consumed word of parity t & 1 reads
   t + 1, and every slot element of both parities is back to negative zero.
 * A published negative zero arrives as positive zero.
-* A collect of a round nobody published runs out of its (shortened) wait and
-  records MHC_ERR_DEVICE_TIMEOUT in the workspace; a publish two rounds ahead of
+* A collect of a round nobody published runs out of its (shortened) wait,
+  records MHC_ERR_DEVICE_TIMEOUT in the workspace and leaves the round
+  unconsumed, so that the producer of the round two later runs out of its own
+  wait and reports it too; after a reset the rounds go through. A publish two rounds ahead of
   a consumer runs out of its wait, writes nothing and records the timeout in the
   producer's own mailbox. Both are waits on words that nothing writes.
 * Two processes on the same GPU form a gloo group of 2 and exchange mailboxes
@@ -143,9 +145,26 @@ def test_collect_of_unpublished_round_times_out_and_recovers():
         M.mhc_debug_set_wait(old, 0)
     for c, (out, ws) in enumerate(outs):
         assert M.mhc_get_device_status(ws) == M.OK  # reading cleared it
-        assert _consumed(mbs[c])[0] == 1 and (_slots(mbs[c], W, R, H) == NEG_ZERO).all()
-    # round 1 (the other parity), then round 2 (parity 0 again), go through as usual
-    for t in (1, 2):
+        # the collect gave up: round 0 stays unconsumed and its slots stay marked
+        assert _consumed(mbs[c])[0] == 0 and (_slots(mbs[c], W, R, H) == NEG_ZERO).all()
+    # round 1 (the other parity) goes through as usual
+    _round_trip(mbs, W, R, 1, d)
+    # a producer of round 2 (parity 0 again) finds round 0 unconsumed: its wait runs
+    # out, it writes nothing and reports the timeout in its own mailbox
+    before = [m.clone() for m in mbs]
+    old = M.mhc_debug_set_wait(20_000_000, 0)
+    try:
+        M.mhc_mailbox_publish(d["partials"][0].to(DEV).contiguous(), 0, 2, [m.data_ptr() for m in mbs], R)
+        torch.cuda.synchronize()
+    finally:
+        M.mhc_debug_set_wait(old, 0)
+    assert M.mhc_get_device_status(mbs[0]) == M.DEVICE_TIMEOUT
+    for m, b in zip(mbs, before):
+        assert torch.equal(m, b)
+    # after a reset of every mailbox the rounds start again from 0
+    for m in mbs:
+        M.mhc_mailbox_init(m)
+    for t in (0, 1, 2):
         _round_trip(mbs, W, R, t, d)
 
 

@@ -15,8 +15,8 @@ import oracle as O
 from mhc_residual_stream_b200 import mhc as M
 from mhc_residual_stream_b200 import synthetic as S
 
-from _parity import (DEV, alloc_outputs, assert_bf16_close, assert_coeffs_close, check_tail, coeff_np, f64,
-                     gpu_post_pre, oracle_post_pre, to_dev)
+from _parity import (DEV, alloc_outputs, assert_bf16_close, assert_bf16_ulp, assert_coeffs_close, check_tail,
+                     coeff_np, f64, gpu_post_pre, oracle_post_pre, stream_terms, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +37,8 @@ def _case(R, H, n, P, seed, swizzled=True, mxfp8=True, coeff=True, affine=True, 
     orc = oracle_post_pre(d, mxfp8=mxfp8, swizzled=swizzled, coeff=coeff)
     what = f"R={R} H={H} n={n} P={P}"
     assert_bf16_close(f64(gpu["residual_out"]), orc["residual"], what + " residual")
+    assert_bf16_ulp(f64(gpu["residual_out"]), orc["residual"], what + " residual (ulp)",
+                    terms=stream_terms(f64(d["partials"]), f64(d["residual"]), f64(d["post"]), f64(d["comb"])))
     check_tail(d, gpu, orc, mxfp8=mxfp8, swizzled=swizzled, coeff=coeff, what=what)
     if coeff:  # end to end as well, at the looser level a bf16 flip allows
         for name in ("post", "comb", "pre"):
@@ -146,6 +148,27 @@ def test_sinkhorn_wide_comb_logits(n):
 
 
 @pytest.mark.parametrize("n", [4, 2])
+def test_sinkhorn_comb_logits_at_the_supported_spread(n):
+    # the contract (mhc_coeff_args): parity holds while every comb logit of a row's
+    # matrix lies within 80 of the largest (exp(L - max L) >= e^-80, a normal
+    # float). fn is scaled down so that the logits are base to within ~0.05:
+    # comb[0][0] at 30 and row 1 at 30 - 79.5, 50 iterations
+    d = S.draw_boundary(6, 256, n=n, partials=2, seed=4300 + n, fn_std=1e-4)
+    c = d["coeff"]
+    base = c.base.clone()
+    c0 = 2 * n
+    base[c0:] = 0.0
+    base[c0 + 0] = 30.0
+    base[c0 + 1 * n: c0 + 2 * n] = 30.0 - 79.5
+    c.base = base
+    c.sinkhorn_iters = 50
+    gpu = gpu_post_pre(d)
+    post, comb, pre = O.mhc_coefficients(f64(gpu["residual_out"]), **coeff_np(c))
+    assert np.isfinite(f64(gpu["comb"])).all()
+    assert_coeffs_close(gpu, post, comb, pre, f"comb logit spread 79.5, n={n}")
+
+
+@pytest.mark.parametrize("n", [4, 2])
 def test_sinkhorn_underflowing_comb_row_stays_finite(n):
     # comb row 1 ~280 below the largest logit: its exp(L - max L) is exactly zero
     # in fp32 (float64 keeps ~1e-122 and grows it back into a full row: outside
@@ -189,10 +212,26 @@ def _moe_oracle(d, pre=True, mxfp8=False, coeff=True):
                       coeff=coeff_np(d["coeff"]) if coeff else None, mxfp8=mxfp8)
 
 
+def _moe_terms(d):
+    """Magnitude sums of the new streams' terms with x = shared + sum_t w g (MoE front)."""
+    g = f64(d["gemm2_permuted"])
+    w = f64(d["expert_weights"])
+    idx = d["expanded_idx_to_permuted_idx"].numpy().astype(np.int64)
+    R, k = w.shape
+    xa = np.abs(f64(d["shared_output"]))
+    for r in range(R):
+        for t in range(k):
+            e = idx[r * k + t]
+            if 0 <= e < g.shape[0]:
+                xa[r] += abs(w[r, t]) * np.abs(g[e])
+    return stream_terms(xa[None], f64(d["residual"]), f64(d["post"]), f64(d["comb"]))
+
+
 def test_moe_boundary_rows64_full_size():
     d = S.draw_moe(64, 7168, n=4, top_k=8, seed=3064)
     gpu, _ = _moe_gpu(d)
     orc = _moe_oracle(d)
+    assert_bf16_ulp(f64(gpu["residual_out"]), orc["residual"], "moe rows 64 residual (ulp)", terms=_moe_terms(d))
     assert_bf16_close(f64(gpu["residual_out"]), orc["residual"], "moe residual")
     check_tail(d, gpu, orc, mxfp8=False, what="moe")
 
@@ -203,6 +242,8 @@ def test_moe_shapes_with_mxfp8(R, H, k, extra):
     gpu, _ = _moe_gpu(d, mxfp8=True)
     orc = _moe_oracle(d, mxfp8=True)
     assert_bf16_close(f64(gpu["residual_out"]), orc["residual"], "moe residual")
+    assert_bf16_ulp(f64(gpu["residual_out"]), orc["residual"], f"moe R={R} H={H} k={k} residual (ulp)",
+                    terms=_moe_terms(d))
     check_tail(d, gpu, orc, mxfp8=True, what="moe")
 
 
@@ -439,23 +480,32 @@ def test_packed_projection_moe_and_coeffs_entry():
 
 @pytest.mark.parametrize("n", [1, 4])
 def test_packed_layout_holds_the_three_bf16_terms(n):
-    # element (t, c, k) of block g is term t of fn[(k/64)*H + 64g + k%64][c]; terms add back to fn
+    # block g's image is [n atom columns][arows][128 bytes]: row m = t*C + c holds
+    # term t of fn column c for K values kin = 0..63 of stream j, the 16-byte
+    # chunk kin // 8 stored at chunk (kin // 8) ^ (m % 8); the terms add back to fn
     H = 128
     C = 2 * n + n * n
+    AR = (3 * C + 7) // 8 * 8
     fn = torch.randn(n * H, C, dtype=torch.float32) * 0.02
     pk = M.mhc_projection_pack(fn.to(DEV), H, n)
     torch.cuda.synchronize()
-    KS, CP8 = n * 64 + 8, ((C + 7) // 8) * 8
-    t = pk.cpu().view(torch.bfloat16).view(H // 64, 3, CP8, KS).to(torch.float64)
+    raw = pk.cpu().view(torch.bfloat16).view(H // 64, n, AR, 8, 8).to(torch.float64)  # [g][j][m][chunk][8]
+    assert raw.numel() * 2 == M.mhc_projection_pack_bytes(H, n)
+
+    def term(g, t, c, k):
+        j, kin = divmod(k, 64)
+        m = t * C + c
+        return raw[g, j, m, (kin // 8) ^ (m % 8), kin % 8]
+
     for g in range(H // 64):
         for k in [k for k in (0, 5, 63, 64, 200, n * 64 - 1) if k < n * 64]:
             row = (k // 64) * H + 64 * g + k % 64
-            s = t[g, 0, :C, k] + t[g, 1, :C, k] + t[g, 2, :C, k]
+            s = torch.tensor([term(g, 0, c, k) + term(g, 1, c, k) + term(g, 2, c, k) for c in range(C)])
             assert torch.allclose(s, fn[row].double(), rtol=2 ** -22, atol=0), (g, k)
             hi = fn[row].to(torch.bfloat16).double()
-            assert torch.equal(t[g, 0, :C, k], hi), (g, k)
-    for pad in (t[:, :, C:, :], t[:, :, :, n * 64:]):  # padding columns and gaps are zero
-        assert pad.numel() == 0 or float(pad.abs().max()) == 0.0
+            assert torch.equal(torch.tensor([term(g, 0, c, k) for c in range(C)]).double(), hi), (g, k)
+    pad = raw[:, :, 3 * C:]  # rows past the three terms are zero
+    assert pad.numel() == 0 or float(pad.abs().max()) == 0.0
 
 
 # ---------------------------------------------------------------- bounded waits

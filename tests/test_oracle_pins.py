@@ -284,6 +284,25 @@ def test_moe_finalize_one_hot_row_coded():
         O.moe_finalize(g, w, idx3, np.zeros((R, H)))
 
 
+def test_moe_finalize_weighted_row_coded():
+    # slot weights 1/2, 1/4, 1/8 (exact in binary) on row-coded expert rows
+    # g[p][h] = (p + 1) + h/64 and shared[r][h] = r/2: each output row is
+    # shared + (4 (a+1) + 2 (b+1) + (c+1) + 7 h/64) / 8 for the selected rows a, b, c,
+    # so a weight squared, a weight on the wrong slot or a slot dropped changes it
+    R, k, H = 5, 3, 16
+    num = R * k + 4
+    h = np.arange(H)
+    g = np.stack([(p + 1) + h / 64.0 for p in range(num)])
+    shared = np.stack([np.full(H, r / 2.0) for r in range(R)])
+    idx = np.random.default_rng(9).permutation(num)[: R * k]
+    w = np.tile(np.array([0.5, 0.25, 0.125]), (R, 1))
+    x = O.moe_finalize(g, w, idx, shared)
+    for r in range(R):
+        a, b, c = idx[r * k], idx[r * k + 1], idx[r * k + 2]
+        want = r / 2.0 + (4 * (a + 1) + 2 * (b + 1) + (c + 1) + 7 * h / 64.0) / 8.0
+        assert np.array_equal(x[r], want), r
+
+
 # ---------------------------------------------------------------- collapse / norm / first layer
 
 def test_rms_norm_constant_row():
