@@ -1,34 +1,34 @@
 // mHC decode boundary on B200 (sm_100a): the fused kernel and the C ABI of
 // libmhc.so (declared in include/mhc.h).
 //
-// A boundary is ONE launch of boundary_kernel over G = H/64 CTAs, in thread-block
-// clusters of CL. CTA g owns columns [64g, 64g + 64) of every row, so every
-// weight of fn is read from HBM exactly once per boundary.
+// A boundary is ONE launch of boundary_kernel over G = H/64 CTAs, one per SM.
+// CTA g owns columns [64g, 64g + 64) of every row, so every weight of fn is
+// read from HBM exactly once per boundary.
 //   1. Before it waits for its predecessor on the stream (programmatic dependent
-//      launch), a CTA bulk-copies its fn slice (fp32) into shared memory, where
-//      it splits each weight into three bf16 terms (128B-swizzled rows of K
-//      values, one row per term and fn column).
+//      launch), a CTA starts the bulk copy of its fn slice (fp32) into shared
+//      memory.
 //   2. After the wait, tensor-map TMA loads bring the rows' data into shared
-//      memory in 16-row chunks, two in flight: the partials (one 3-D box), or
-//      the MoE expert rows gathered by index (tile::gather4) and the shared
-//      output, and the residual streams (one 3-D box).
-//   3. Eight warps take a chunk: sum or finalize x, mHC post-mix (vllm
-//      ...boundary.boundary, Boundaries.post_only: mhc_post(x, residual, post,
-//      comb)), store the new streams, stage them in shared memory, and sum per
-//      row the squares of their collapse with the carried pre
-//      (BoundaryState.pre) and of the streams.
+//      memory in 16-row chunks, up to four in flight: the partials (one 3-D
+//      box), or the MoE expert rows gathered by index (tile::gather4) and the
+//      shared output, and the residual streams (one 3-D box). While they are in
+//      flight the CTA splits each fn weight into three bf16 terms (128B-swizzled
+//      rows of K values, one row per term and fn column).
+//   3. Two groups of eight warps take alternate chunks: sum or finalize x, mHC
+//      post-mix (vllm ...boundary.boundary, Boundaries.post_only: mhc_post(x,
+//      residual, post, comb)), store the new streams, stage them in shared
+//      memory, and sum per row the squares of their collapse with the carried
+//      pre (BoundaryState.pre) and of the streams.
 //   4. The same warps project the chunk's 16 rows of staged streams onto the C
 //      fn columns on the tensor cores (mma.sync m16n8k16 bf16, fp32
 //      accumulation; each warp a share of K, the shares added in warp order),
 //      while a control warp refills the chunk's stage.
-//   5. The rows' records (C dot products, sum v^2, sum c^2) are added over the
-//      cluster through distributed shared memory; each cluster publishes its
-//      sums as tagged 64-bit words in the workspace (no flag, no fence, no
-//      second kernel).
-//   6. Every CTA adds the clusters' sums of c^2 of every row and writes its
-//      columns of the layer input (and MXFP8); the CTA that owns a row's
-//      coefficients adds that row's records and runs the logits, sigmoid and
-//      Sinkhorn.
+//   5. Each CTA publishes its row records (C dot products, sum v^2, sum c^2) as
+//      tagged 64-bit words in the workspace, field-major, so that one field of
+//      one row is contiguous over the CTAs (no flag, no fence, no second kernel).
+//   6. In one round over the published words every CTA adds the sum of c^2 of
+//      every row and the records of the rows whose coefficients it finishes
+//      (rows g and g + G), writes its columns of the layer input (and MXFP8),
+//      and runs those rows' logits, sigmoid and Sinkhorn.
 // The residual-only variant is steps 2-3 alone. Every reduction runs in a fixed
 // order, so results are bitwise reproducible.
 
@@ -49,8 +49,9 @@ namespace mhc {
 
 constexpr int kCols = 64;        // columns of H per CTA
 constexpr int kRC = 16;          // rows per chunk (N of one projection MMA)
-constexpr int kMaxStages = 2;    // chunks in flight (1 where two do not fit in shared memory)
-constexpr int kWorkWarps = 8;    // warps of the streaming phase: a warp per row pair of a chunk
+constexpr int kMaxStages = 4;    // chunks in flight (fewer where they do not fit in shared memory)
+constexpr int kWorkWarps = 16;   // warps of the streaming phase: two groups of 8 on alternate chunks
+constexpr int kGroupWarps = 8;   // a group: 2 rows of a chunk per warp, 4 columns per lane
 constexpr int kCtl = kWorkWarps; // index of the control warp
 constexpr int kThreads = (kWorkWarps + 1) * 32;
 constexpr int kWorkThreads = kWorkWarps * 32;
@@ -60,10 +61,10 @@ constexpr int kMaxPartials = 16;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxIters = 1000;
 constexpr int kMaxBlocks = 148;
-constexpr int kMaxCluster = 8;  // CTAs of a cluster
-constexpr int kRecF = 32;        // fields of a row record: C dot products, sum v^2, sum c^2 (padded)
+constexpr int kRecF = 32;        // shared-memory stride of a row record: C dot products, sum v^2, sum c^2
 // Workspace: a 1 KB header (status word at byte 0, the launch epoch at byte 64),
-// then the clusters' row records [NC][R][kRecF] as tagged 64-bit words.
+// then the CTAs' row records as tagged 64-bit words, [G CTAs][R rows][fields],
+// then the rows' total sums of c^2, one copy for each CTA to read, [G][R].
 constexpr size_t kWsHeader = 1024;
 constexpr int kStatusWord = 0;
 constexpr int kEpochWord = 16;
@@ -75,6 +76,9 @@ enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3, kMailbox = 4
 __host__ __device__ constexpr bool lane_partials(int front) { return front == kMailbox || front == kTable; }
 
 __host__ __device__ constexpr int logits_of(int n) { return 2 * n + n * n; }
+// Fields of a published row record: C dot products, sum v^2 and sum c^2, rounded
+// up to an even count (records are read as 16-byte pairs of words).
+__host__ __device__ constexpr int fields_of(int n) { return (logits_of(n) + 3) & ~1; }
 // rows of the fn slice image: three bf16 terms of each of the C fn columns (row
 // t*C + c), rounded up to a whole 8-row swizzle atom
 __host__ __device__ constexpr int arows_of(int n) { return (3 * logits_of(n) + 7) & ~7; }
@@ -116,23 +120,24 @@ struct Params {
   float* pre_out;
   int R, H;
   int write_res, do_layer, do_coeff;
-  int CL;      // cluster size (divides G)
-  int stages;  // chunk stages in flight: 1 or 2
+  int stages;  // chunk stages in flight: 1 .. kMaxStages
   // workspace
   unsigned* ctl;             // header: status, epoch
-  unsigned long long* rec;   // [NC][R][kRecF] tagged words
+  unsigned long long* rec;   // [G][R][fields] tagged words: the CTAs' row records
+  unsigned long long* tot;   // [G][R] tagged words: the rows' sums c^2, one copy per CTA
   int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
   int64_t budget_ns;
 };
 
 // Shared memory of the kernel, offsets from a 1024-byte aligned base.
 struct Layout {
-  int a_off, v_off, st_off, stage_bytes, res_units, part_off, mix_off, moe_off, rec_off, inv_off, bar_off, total;
+  int a_off, v_off, st_off, stage_bytes, res_units, fst_off, part_off, mix_off, moe_off, rec_off, inv_off, cft_off,
+      bar_off, total;
   int r_alloc;
 };
 
 // Bytes of one chunk's projection partials: [warp][16 rows][C] floats.
-__host__ __device__ constexpr int part_bytes(int n) { return kWorkWarps * kRC * logits_of(n) * 4; }
+__host__ __device__ constexpr int part_bytes(int n) { return kGroupWarps * kRC * logits_of(n) * 4; }
 
 // 128-byte box rows of one chunk's stage, and where the residual streams start.
 __host__ __device__ inline void stage_units(int front, int n, int P, int topk, int* units, int* res_units) {
@@ -148,52 +153,53 @@ __host__ __device__ inline void stage_units(int front, int n, int P, int topk, i
 }
 
 template <int N>
-__host__ __device__ inline Layout layout_of(int front, int R, int P, int topk, bool coeff, bool layer, int NC,
-                                          int stages) {
+__host__ __device__ inline Layout layout_of(int front, int R, int G, int P, int topk, bool coeff, bool layer,
+                                          int stages, bool packed) {
   constexpr int C = logits_of(N);
   Layout L{};
   L.r_alloc = (R + kRC - 1) / kRC * kRC;
   int o = 0;
   L.a_off = o;  // fn slice image [n atom columns][arows][128 B]
   if (coeff) o += aimage_bytes(N);
-  L.v_off = o;  // new streams [n atom columns][r_alloc][128 B]
-  if (coeff || layer) o += N * L.r_alloc * 128;
-  L.st_off = o;  // chunk stages; before the wait the fp32 fn slice, after the
-                 // last chunk the c^2 scratch
+  // new streams [n atom columns][r_alloc][128 B]; until the first chunk is
+  // staged, the fp32 fn slice as copied, [n][64][C]
+  L.v_off = L.fst_off = o;
+  int vb = (coeff || layer) ? N * L.r_alloc * 128 : 0;
+  if (coeff && !packed && vb < N * kCols * C * 4) vb = N * kCols * C * 4;
+  o += vb;
+  L.st_off = o;  // chunk stages
   int units, ru;
   stage_units(front, N, P, topk, &units, &ru);
   L.stage_bytes = units * 128;
   L.res_units = ru;
+  // after the last chunk, the row records this CTA adds up: [ceil(R / G) * G][fields]
   int st = stages * L.stage_bytes;
-  if (coeff && st < N * kCols * C * 4) st = N * kCols * C * 4;
-  if (layer && st < NC * R * 4) st = NC * R * 4;
-  o += (st + 1023) & ~1023;
+  if ((coeff || layer) && st < (R + G - 1) / G * G * fields_of(N) * 4) st = (R + G - 1) / G * G * fields_of(N) * 4;
+  o += st;
   // a chunk's projection partials go into its consumed stage when they fit
-  // (the stage is refilled only once the chunk is done), else here
+  // (the stage is refilled only once the chunk is done), else here, one
+  // buffer per group
   L.part_off = -1;
   if (coeff && L.stage_bytes < part_bytes(N)) {
     L.part_off = o;
-    o += part_bytes(N);
+    o += 2 * part_bytes(N);
   }
   L.mix_off = o;  // [R][post n | comb n*n | pre n]
   o += (R * (2 * N + N * N) * 4 + 15) & ~15;
   L.moe_off = o;  // e2p [R*topk], weights [R*topk]
   if (front == kMoe) o += (R * topk * 8 + 15) & ~15;
-  L.rec_off = o;  // [R][kRecF] this CTA's row records
+  L.rec_off = o;  // this CTA's row records [R][kRecF]
   if (coeff || layer) o += R * kRecF * 4;
   L.inv_off = o;  // [R] inverse RMS of the collapse
   if (layer) o += (R * 4 + 15) & ~15;
+  L.cft_off = o;  // [ceil(R / G)][kRecF] the totals of the rows this CTA adds up
+  if (coeff || layer) o += (R + G - 1) / G * kRecF * 4;
   L.bar_off = o;  // full[kMaxStages], vready[kMaxChunks], fnbar, then the tag slot
   o += (kMaxStages + kMaxChunks + 1) * 8 + 16;
   L.total = (o + 15) & ~15;
   return L;
 }
 
-__device__ __forceinline__ float sum16_lanes(float v) {  // over the 16 lanes sharing lane bit 4
-#pragma unroll
-  for (int m = 8; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
-  return v;
-}
 
 __device__ __forceinline__ int swizzled_scale_offset(int r, int c, int col_tiles) {
   const int tile = (r >> 7) * col_tiles + (c >> 2);
@@ -209,23 +215,11 @@ __device__ __forceinline__ int sw128_offset(int row, int v) {
 
 __device__ __forceinline__ uint2 lds_v2(const void* p) { return *reinterpret_cast<const uint2*>(p); }
 
-__device__ __forceinline__ void named_sync_workers() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kWorkThreads) : "memory");
+__device__ __forceinline__ void named_sync_workers() {  // the streaming warps (groups use barriers 1 and 2)
+  asm volatile("bar.sync 3, %0;" ::"n"(kWorkThreads) : "memory");
 }
 
-// A mailbox slot's 4 elements as loaded, re-read until none is negative zero
-// (bounded: on timeout the status records it and the values are used as they are).
-__device__ __forceinline__ uint2 settle_slot(const __nv_bfloat16* src, uint2 v, long long deadline,
-                                             unsigned* status) {
-  while (has_neg_zero(v)) {
-    if (clock64() > deadline) {
-      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-      break;
-    }
-    v = ld_volatile_v2(src);
-  }
-  return v;
-}
+
 
 // fn as three bf16 terms, f = hi + mid + lo to 2^-24: each bf16 x bf16 product is
 // exact in fp32, so three tensor-core products return the fp32 projection up to
@@ -337,58 +331,19 @@ __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, fl
 }
 
 
-// The values of `count` (<= B) tagged words p[i * stride]: every load goes out at
-// once, then the words still stale are re-read together, one round trip per
-// pass, until each carries `tag` (bounded: on timeout the status records it and
-// the values are used as they are).
-template <int B>
-__device__ __forceinline__ void gather_tagged(const unsigned long long* p, size_t stride, int count, uint32_t tag,
-                                              long long deadline, unsigned* status, float (&out)[B]) {
-  unsigned long long w[B];
-#pragma unroll
-  for (int i = 0; i < B; ++i)
-    if (i < count) w[i] = ld_tagged(p + i * stride);
-  while (true) {
-    bool all = true;
-#pragma unroll
-    for (int i = 0; i < B; ++i)
-      if (i < count && tag_of(w[i]) != tag) all = false;
-    if (all) break;
-    if (clock64() > deadline) {
-      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-      break;
-    }
-#pragma unroll
-    for (int i = 0; i < B; ++i)
-      if (i < count && tag_of(w[i]) != tag) w[i] = ld_tagged(p + i * stride);
-  }
-#pragma unroll
-  for (int i = 0; i < B; ++i) out[i] = i < count ? value_of(w[i]) : 0.f;
-}
-
-// The coefficients of row r, by one warp: lane f <= C adds field f of the row's
-// record over the NC clusters in cluster order (C dot products and sum v^2),
-// then the logits (lane c computes logit c), pre / post by sigmoid, and the
-// comb by one exponential per lane and Sinkhorn in lane 0 ([boundary]
-// Boundaries.sublayer: mhc_pre_delayed_overlap(residual, fn, scale, base,
-// rms_norm_eps, hc_eps, hc_eps, hc_post_alpha, hc_sinkhorn_iters)).
+// The coefficients of row r, by one warp, from the row's totals over the CTAs
+// (tot[c]: dot product with fn column c, tot[C]: sum v^2): the logits (lane c
+// computes logit c), pre / post by sigmoid, and the comb by one exponential per
+// lane and Sinkhorn in lane 0 ([boundary] Boundaries.sublayer:
+// mhc_pre_delayed_overlap(residual, fn, scale, base, rms_norm_eps, hc_eps,
+// hc_eps, hc_post_alpha, hc_sinkhorn_iters)).
 template <int N>
-__device__ __forceinline__ void coefficient_row(const Params& p, int r, int NC, uint32_t tag, float scale_l,
-                                                float base_l, long long deadline, unsigned* status, int lane) {
+__device__ __forceinline__ void coefficient_row(const Params& p, int r, const float* tot, float scale_l, float base_l,
+                                                int lane) {
   constexpr int C = logits_of(N);
   constexpr int NN = N * N;
-  float s = 0.f;
-  if (lane <= C) {
-    constexpr int B = 16;
-    for (int c0 = 0; c0 < NC; c0 += B) {
-      float v[B];
-      gather_tagged<B>(p.rec + (static_cast<size_t>(c0) * p.R + r) * kRecF + lane, static_cast<size_t>(p.R) * kRecF,
-                       NC - c0 < B ? NC - c0 : B, tag, deadline, status, v);
-#pragma unroll
-      for (int i = 0; i < B; ++i) s += v[i];  // clusters in order (absent ones add 0)
-    }
-  }
-  const float inv = rsqrtf(__fdiv_rn(__shfl_sync(kFull, s, C), static_cast<float>(N * p.H)) + p.rms_eps);
+  const float s = lane < C ? tot[lane] : 0.f;
+  const float inv = rsqrtf(__fdiv_rn(tot[C], static_cast<float>(N * p.H)) + p.rms_eps);
   const float l = lane < C ? scale_l * inv * s + base_l : 0.f;
   if (lane < N) {
     p.pre_out[r * N + lane] = 1.f / (1.f + expf(-l)) + p.pre_eps;
@@ -417,13 +372,13 @@ __device__ __forceinline__ void coefficient_row(const Params& p, int r, int NC, 
 }
 
 // The projection of chunk c's 16 staged rows (K = n*64 stream values each) onto
-// the C fn columns on the tensor cores: warp w runs K steps w, w + 8, ... (16
-// values each: stream k / 4, offset 16 * (k % 4)), one accumulator per bf16
-// term of fn; the terms are added (hi + mid) + lo and the warp's 16 x C partial
-// sums go to part[w].
+// the C fn columns on the tensor cores, by the 8 warps of the chunk's group:
+// warp wq runs K steps wq, wq + 8, ... (16 values each: stream k / 4, offset
+// 16 * (k % 4)), one accumulator per bf16 term of fn; the terms are added
+// (hi + mid) + lo and the warp's 16 x C partial sums go to part[wq].
 template <int N>
 __device__ __forceinline__ void project_chunk(const unsigned char* f_s, const unsigned char* v_s, int r_alloc, int c,
-                                              int warp, int lane, float* part) {
+                                              int wq, int lane, float* part) {
   constexpr int C = logits_of(N);
   constexpr int AR = arows_of(N);
   constexpr int NT = (C + 7) / 8;  // 8-column tiles
@@ -434,7 +389,7 @@ __device__ __forceinline__ void project_chunk(const unsigned char* f_s, const un
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[t][nt][q] = 0.f;
-  for (int k = warp; k < 4 * N; k += kWorkWarps) {
+  for (int k = wq; k < 4 * N; k += kGroupWarps) {
     const int j = k >> 2, kc0 = (k & 3) * 2;  // two 16-byte chunks of a 128-byte row
     const int row = c * kRC + (lane & 15), kca = kc0 + (lane >> 4);
     unsigned a[4];
@@ -452,7 +407,7 @@ __device__ __forceinline__ void project_chunk(const unsigned char* f_s, const un
     }
   }
   // C fragment: lane holds rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
-  float* dst = part + warp * kRC * C;
+  float* dst = part + wq * kRC * C;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -467,32 +422,49 @@ __device__ __forceinline__ void project_chunk(const unsigned char* f_s, const un
   }
 }
 
+__device__ __forceinline__ float sum16_lanes(float v) {  // over the 16 lanes sharing lane bit 4
+#pragma unroll
+  for (int m = 8; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  return v;
+}
+
+__device__ __forceinline__ void named_sync_group(int q) {  // barrier ids are immediates: 1 and 2
+  if (q == 0) {
+    asm volatile("bar.sync 1, %0;" ::"n"(kGroupWarps * 32) : "memory");
+  } else {
+    asm volatile("bar.sync 2, %0;" ::"n"(kGroupWarps * 32) : "memory");
+  }
+}
+
 // The boundary, one launch. See the top of this file for the steps; the
 // numbered comments below follow them.
 template <int N, int FRONT>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     boundary_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_res, const __grid_constant__ CUtensorMap tm_gather) {
   constexpr int C = logits_of(N);
   constexpr int MIX = 2 * N + N * N;
   constexpr int AR = arows_of(N);
+  constexpr int NFP = fields_of(N);  // record fields: C dot products, sum v^2, sum c^2 (even)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   const int R = p.R, H = p.H;
   const int G = gridDim.x;
-  const int NC = G / p.CL;
   const bool coeff = p.do_coeff != 0, layer = p.do_layer != 0, exch = coeff || layer;
   const int S = p.stages;
-  const Layout L = layout_of<N>(FRONT, R, p.P, p.topk, coeff, layer, NC, S);
+  const bool packed = p.fn_packed != nullptr;
+  const Layout L = layout_of<N>(FRONT, R, G, p.P, p.topk, coeff, layer, S, packed);
   unsigned char* a_s = smem + L.a_off;
   unsigned char* v_s = smem + L.v_off;
   unsigned char* st_s = smem + L.st_off;
+  unsigned char* fst_s = smem + L.fst_off;  // the fp32 fn slice as copied
   float* mix_s = reinterpret_cast<float*>(smem + L.mix_off);
   int* e2p_s = reinterpret_cast<int*>(smem + L.moe_off);
   float* ew_s = reinterpret_cast<float*>(smem + L.moe_off) + R * p.topk;
-  float* rec_s = reinterpret_cast<float*>(smem + L.rec_off);
-  float* inv_s = reinterpret_cast<float*>(smem + L.inv_off);
+  float* rec_s = reinterpret_cast<float*>(smem + L.rec_off);  // [R][kRecF] this CTA's row records
+  float* inv_s = reinterpret_cast<float*>(smem + L.inv_off);  // [R] inverse RMS of the collapse
+  float* cft_s = reinterpret_cast<float*>(smem + L.cft_off);  // [slot][kRecF] this CTA's coefficient rows' totals
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* vready = full + kMaxStages;
   uint64_t* fnbar = vready + kMaxChunks;
@@ -503,19 +475,19 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int nch = (R + kRC - 1) / kRC;
   const long long deadline = wait_deadline(p.budget_ns);
   unsigned* status = p.ctl ? p.ctl + kStatusWord : nullptr;  // null: a residual-only call without a workspace
-  // the streaming lanes: row rl of a chunk, columns h0 .. h0 + 3
-  const int rl = warp * 2 + (lane >> 4);
+  // the streaming lanes: group q of 8 warps takes chunks q, q + 2, ...; in a
+  // chunk, row rl = 2 * (warp % 8) + lane / 16 and columns h0 .. h0 + 3
+  const int q = warp / kGroupWarps, wq = warp % kGroupWarps;
+  const int rl = wq * 2 + (lane >> 4);
   const int v = lane & 15;
   const int h0 = g * kCols + v * 4;
 
-  // ---- 1. set-up and weights, before the wait (no kernel of this library
-  // writes weights, and kernels that do not trigger dependent launches are
-  // waited for in full before this one starts). The fn slice's copy goes out
-  // first: its HBM round trip is the longest step here.
-  const bool packed = p.fn_packed != nullptr;
+  // ---- 1. set-up before the wait (no kernel of this library writes weights,
+  // and kernels that do not trigger dependent launches are waited for in full
+  // before this one starts): the fn slice's copy goes out first
   if (tid == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
-    for (int c = 0; c < nch; ++c) mbar_init(&vready[c], kWorkWarps);
+    for (int c = 0; c < nch; ++c) mbar_init(&vready[c], kGroupWarps);
     mbar_init(fnbar, 1);
     if (coeff) {
       if (packed) {
@@ -526,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive_expect_tx(fnbar, N * JB + 16 * p.extra_tx);
 #pragma unroll
         for (int j = 0; j < N; ++j)
-          bulk_g2s(st_s + j * JB, p.fn + (static_cast<size_t>(j) * H + g * kCols) * C, JB, fnbar);
+          bulk_g2s(fst_s + j * JB, p.fn + (static_cast<size_t>(j) * H + g * kCols) * C, JB, fnbar);
       }
     }
     if (FRONT == kPartials || FRONT == kBroadcast || FRONT == kMoe) prefetch_tensormap(&tm_x);
@@ -541,22 +513,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     base_l = p.base[lane];
   }
   __syncthreads();
-  bool fn_ok = true;
-  if (coeff) {
-    bool ok = mbar_wait_bounded(fnbar, 0, deadline);
-    fn_ok = __syncthreads_and(ok) != 0;
-    if (!fn_ok && tid == 0) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-    if (fn_ok && !packed) {
-      // consecutive threads take consecutive fn columns: conflict-free reads of the
-      // fp32 slice [kin][C]
-      for (int it = tid; it < N * C * 8; it += kThreads) {
-        const int c = it % C, rest = it / C;
-        const int oct = rest & 7, j = rest >> 3;
-        split_octet<N>(reinterpret_cast<const float*>(st_s + j * kCols * C * 4), a_s + j * AR * 128, c, oct);
-      }
-    }
-  }
-  __syncthreads();  // the fn terms complete; the staging area is free for the chunks
 
   // ---- 2. wait for the preceding kernel on the stream, then the row data
   griddep_wait();
@@ -587,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();
     if (p.num_perm > 0) {
-      for (int q = lane; q < K * 4; q += 32) {  // slot t, rows 4*quad .. 4*quad + 3 of the chunk
-        const int t = q >> 2, quad = q & 3;
+      for (int qq = lane; qq < K * 4; qq += 32) {  // slot t, rows 4*quad .. 4*quad + 3 of the chunk
+        const int t = qq >> 2, quad = qq & 3;
         int idx[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -625,18 +581,41 @@ __global__ void __launch_bounds__(kThreads, 2)
       cp_async4(ew_s + k, p.ew + k);
     }
   }
+  // the fn slice's three bf16 terms, while the row data is in flight: one thread
+  // waits on the copy, the others block in the barrier (no issue slots)
+  bool fn_ok = true;
+  if (coeff) {
+    const bool ok = tid == 0 ? mbar_wait_bounded(fnbar, 0, deadline) : true;
+    fn_ok = __syncthreads_and(ok) != 0;
+    if (!fn_ok && tid == 0) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (fn_ok && !packed) {
+      // consecutive threads take consecutive fn columns: conflict-free reads of the
+      // fp32 slice [kin][C]
+      for (int it = tid; it < N * C * 8; it += kThreads) {
+        const int c = it % C, rest = it / C;
+        const int oct = rest & 7, j = rest >> 3;
+        split_octet<N>(reinterpret_cast<const float*>(fst_s + j * kCols * C * 4), a_s + j * AR * 128, c, oct);
+      }
+    }
+  }
   cp_async_wait_all();
-  __syncthreads();
+  __syncthreads();  // the mixes (and MoE routing) staged, the fn terms complete
   const uint32_t tag = exch ? *tag_slot : 0u;
   if (FRONT == kMoe && warp == kCtl) {
     for (int c = 0; c < nch && c < S; ++c) issue_moe_chunk(c);
   }
 
   if (warp < kWorkWarps) {
-    // ---- 3. the chunks: x, post-mix, new streams, staged B operand, row sums
-    for (int c = 0; c < nch; ++c) {
+    // ---- 3. the chunks of group q: x, post-mix, new streams, staged streams, row sums
+    // with one stage, group 0 takes every chunk in order (two groups on one stage
+    // could each see the other's phase of its barrier as their own)
+    const int c0 = S > 1 ? q : (q == 0 ? 0 : nch), cstep = S > 1 ? 2 : 1;
+    for (int c = c0; c < nch; c += cstep) {
       const int s = c % S;
-      if (!mbar_wait_bounded(&full[s], (c / S) & 1, deadline)) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+      // one lane of the group waits for the chunk's data; the group blocks in its barrier
+      if (wq == 0 && lane == 0 && !mbar_wait_bounded(&full[s], (c / S) & 1, deadline))
+        record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+      named_sync_group(q);
       const int r = c * kRC + rl;
       const bool valid = r < R;
       const unsigned char* sp = st_s + s * L.stage_bytes;
@@ -676,7 +655,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int u = 0; u < p.P; ++u) {
               const __nv_bfloat16* src = p.pptr[u] + off;
               uint2 w = ld_cg_v2(src);
-              if (FRONT == kMailbox) w = settle_slot(src, w, deadline, status);
+              if (FRONT == kMailbox) {
+                while (has_neg_zero(w)) {  // re-read until its producer has written every element
+                  if (clock64() > deadline) {
+                    record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+                    break;
+                  }
+                  w = ld_volatile_v2(src);
+                }
+              }
               float2 f[2];
               unpack4x2(w, f);
 #pragma unroll
@@ -733,8 +720,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (p.aux_out != nullptr && valid) {  // mean over the streams, in stream order, rounded once
         constexpr float kInvN = 1.f / N;    // exact: n is a power of two
-        uint2 ab;
-        unsigned* aw = reinterpret_cast<unsigned*>(&ab);
+        unsigned aw[2];
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           float2 m = nf[0][t];
@@ -743,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           m = __fmul2_rn(m, make_float2(kInvN, kInvN));
           aw[t] = pack_bf16x2(m.x, m.y);
         }
-        st_v2(p.aux_out + static_cast<size_t>(r) * H + h0, ab);
+        st_v2(p.aux_out + static_cast<size_t>(r) * H + h0, make_uint2(aw[0], aw[1]));
       }
       if (exch) {  // the new streams staged for the projection and the layer input
 #pragma unroll
@@ -778,12 +764,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int t = 0; t < 2; ++t) sv = __ffma2_rn(nf[i][t], nf[i][t], sv);
         const float sv2 = sum16_lanes(sv.x + sv.y);
         if (valid && v == 0) rec_s[r * kRecF + C] = sv2;
-        named_sync_workers();  // every warp's rows of the chunk staged; the stage read
-        float* part = L.part_off >= 0 ? reinterpret_cast<float*>(smem + L.part_off) : reinterpret_cast<float*>(st_s + s * L.stage_bytes);
-        if (fn_ok) project_chunk<N>(a_s, v_s, L.r_alloc, c, warp, lane, part);
-        named_sync_workers();
-        const int kw = 4 * N < kWorkWarps ? 4 * N : kWorkWarps;  // warps that ran K steps
-        for (int it = tid; it < kRC * C; it += kWorkThreads) {  // partials added in warp order
+        named_sync_group(q);  // the group's rows of the chunk staged; its stage read
+        float* part = L.part_off >= 0 ? reinterpret_cast<float*>(smem + L.part_off + q * part_bytes(N))
+                                      : reinterpret_cast<float*>(st_s + s * L.stage_bytes);
+        if (fn_ok) project_chunk<N>(a_s, v_s, L.r_alloc, c, wq, lane, part);
+        named_sync_group(q);
+        const int kw = 4 * N < kGroupWarps ? 4 * N : kGroupWarps;  // warps that ran K steps
+        for (int it = wq * 32 + lane; it < kRC * C; it += kGroupWarps * 32) {  // partials added in warp order
           const int rr = it / C, col = it - rr * C;
           if (c * kRC + rr < R) {
             float a = 0.f;
@@ -814,89 +801,142 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  __syncthreads();  // row records complete
   if (exch) {
-    // ---- 5. the cluster's sums: CTA `rank` adds rows rank, rank + CL, ... over
-    // the cluster's CTAs (distributed shared memory) in CTA order and publishes them
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    const int CL = p.CL;
-    const uint32_t rank = cluster_ctarank();
-    const int cl = g / CL;
-    const int f0 = coeff ? 0 : C + 1;
-    const int nf = C + 2 - f0;
-    const int nr = static_cast<int>(rank) < R ? (R - static_cast<int>(rank) + CL - 1) / CL : 0;
-    for (int it = tid; it < nr * nf; it += kThreads) {
-      const int r = static_cast<int>(rank) + (it / nf) * CL, f = f0 + it % nf;
-      const float* src = rec_s + r * kRecF + f;
-      float v[kMaxCluster];
-#pragma unroll
-      for (int k = 0; k < kMaxCluster; ++k)
-        if (k < CL) v[k] = ld_dsmem_f32(dsmem_addr(src, k));
-      float a = 0.f;
-#pragma unroll
-      for (int k = 0; k < kMaxCluster; ++k)
-        if (k < CL) a += v[k];
-      st_tagged(p.rec + (static_cast<size_t>(cl) * R + r) * kRecF + f, tag, a);
+    // ---- 5. publish this CTA's row records as tagged words at rec[g][r][f]: one
+    // contiguous run per CTA
+    __syncthreads();  // every row's records complete
+    for (int it = tid; it < R * NFP; it += kThreads) {
+      const int r = it / NFP, f = it - r * NFP;
+      const bool has = f <= C ? coeff : (f == C + 1 && layer);
+      st_tagged(p.rec + static_cast<size_t>(g) * R * NFP + it, tag, has ? rec_s[r * kRecF + f] : 0.f);
     }
     griddep_launch_dependents();  // this boundary's HBM stream is done: the next may start its set-up
-    cluster_arrive_release();     // done reading the cluster's shared memory
 
-    // ---- 6. layer input and coefficients from every cluster's published sums
-    if (warp == kCtl && coeff) {
-      for (int r = g; r < R; r += G) coefficient_row<N>(p, r, NC, tag, scale_l, base_l, deadline, status, lane);
-    }
-    if (warp < kWorkWarps && layer) {
-      float* sc = reinterpret_cast<float*>(st_s);  // [NC][R] the clusters' sums of c^2
-      // as few pollers as take at most 16 words each (many threads re-reading the
-      // same lines slow every poller down)
-      constexpr int B = 16;
-      const int words = NC * R;
-      int pollers = ((words + B - 1) / B + 31) & ~31;
-      if (pollers > kWorkThreads) pollers = kWorkThreads;
-      for (int i0 = tid; i0 < words && tid < pollers; i0 += B * pollers) {
-        float vals[B];
-        const int cnt = (words - i0 + pollers - 1) / pollers;
-        gather_tagged<B>(p.rec + static_cast<size_t>(i0) * kRecF + C + 1, static_cast<size_t>(pollers) * kRecF,
-                         cnt < B ? cnt : B, tag, deadline, status, vals);
+    // ---- 6. CTA g adds up rows g, g + G, ...: their records from every CTA, read
+    // as 16-byte pairs of words (all of a record with the coefficients, else the
+    // pair holding sum c^2), each field summed over the CTAs by 8 lanes
+    const int nslot = g < R ? (R - 1 - g) / G + 1 : 0;
+    if (nslot > 0) {
+      constexpr int B = 8;
+      const int kc0 = coeff ? 0 : (C + 1) / 2, nk = coeff ? NFP / 2 : 1;
+      float* gb = reinterpret_cast<float*>(st_s);  // [slot][G][NFP] the records' values
+      const int total = nslot * G * nk;
+      auto chunk = [&](int i) -> const unsigned long long* {
+        const int slot = i / (G * nk), rem = i - slot * G * nk;
+        const int gg = rem / nk, k = kc0 + rem - gg * nk;
+        return p.rec + (static_cast<size_t>(gg) * R + g + slot * G) * NFP + 2 * k;
+      };
+      for (int i0 = tid; i0 < total; i0 += B * kThreads) {
+        ulonglong2 w[B];
 #pragma unroll
         for (int b = 0; b < B; ++b)
-          if (i0 + b * pollers < words) sc[i0 + b * pollers] = vals[b];
+          if (i0 + b * kThreads < total) w[b] = ld_tagged2(chunk(i0 + b * kThreads));
+        while (true) {  // the stale pairs re-read together until they carry the tag (bounded)
+          bool all = true;
+#pragma unroll
+          for (int b = 0; b < B; ++b)
+            if (i0 + b * kThreads < total && (tag_of(w[b].x) != tag || tag_of(w[b].y) != tag)) all = false;
+          if (all) break;
+          if (clock64() > deadline) {
+            record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+            break;
+          }
+#pragma unroll
+          for (int b = 0; b < B; ++b)
+            if (i0 + b * kThreads < total && (tag_of(w[b].x) != tag || tag_of(w[b].y) != tag))
+              w[b] = ld_tagged2(chunk(i0 + b * kThreads));
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int i = i0 + b * kThreads;
+          if (i < total) {
+            const int slot = i / (G * nk), rem = i - slot * G * nk;
+            const int gg = rem / nk, k = kc0 + rem - gg * nk;
+            float* d = gb + (slot * G + gg) * NFP + 2 * k;
+            d[0] = value_of(w[b].x);
+            d[1] = value_of(w[b].y);
+          }
+        }
       }
-      named_sync_workers();
+      __syncthreads();
+      const int f0 = coeff ? 0 : C + 1, nf = (layer ? C + 2 : C + 1) - f0;
+      const int units = nslot * nf;
+      const int gs = (G + 7) / 8;
+      for (int u0 = 0; u0 < units; u0 += kThreads / 8) {
+        if (u0 + warp * 4 >= units) continue;  // (warp-uniform) no unit for this warp
+        const int u = u0 + tid / 8, pp = tid & 7;
+        // every lane of the warp takes part in the butterfly
+        const bool active = u < units;
+        const int uu = active ? u : 0;
+        const int slot = uu / nf, f = f0 + uu - slot * nf;
+        const float* col = gb + slot * G * NFP + f;
+        float sum = 0.f;
+        const int ge = (pp + 1) * gs < G ? (pp + 1) * gs : G;
+        if (active)
+          for (int gg = pp * gs; gg < ge; ++gg) sum += col[gg * NFP];  // lane pp: CTAs pp*gs .. in order
+#pragma unroll
+        for (int m = 1; m <= 4; m <<= 1) sum += __shfl_xor_sync(kFull, sum, m);
+        if (active && pp == 0) cft_s[slot * kRecF + f] = sum;
+      }
+      __syncthreads();
+      if (layer) {  // the rows' sums c^2, one copy for every CTA: tot[c][r]
+        for (int it = tid; it < nslot * G; it += kThreads) {
+          const int sl = it / G, c = it - sl * G;
+          st_tagged(p.tot + static_cast<size_t>(c) * R + g + sl * G, tag, cft_s[sl * kRecF + C + 1]);
+        }
+      }
+    }
+    if (warp == kCtl && coeff) {
+      for (int sl = 0; sl < nslot; ++sl)
+        coefficient_row<N>(p, g + sl * G, cft_s + sl * kRecF, scale_l, base_l, lane);
+    }
+    if (warp < kWorkWarps && layer) {
+      // every row's sum c^2, from this CTA's copy
       for (int r = tid; r < R; r += kWorkThreads) {
-        float a = 0.f;
-        for (int k = 0; k < NC; ++k) a += sc[k * R + r];
-        inv_s[r] = rsqrtf(__fdiv_rn(a, static_cast<float>(H)) + p.norm_eps);
+        const unsigned long long* src = p.tot + static_cast<size_t>(g) * R + r;
+        unsigned long long w = ld_tagged(src);
+        while (tag_of(w) != tag) {
+          if (clock64() > deadline) {
+            record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+            break;
+          }
+          w = ld_tagged(src);
+        }
+        inv_s[r] = rsqrtf(__fdiv_rn(value_of(w), static_cast<float>(H)) + p.norm_eps);
       }
       named_sync_workers();
+    }
+    if (warp < kWorkWarps && layer) {
+      // ---- 7. the layer input (and MXFP8) of this CTA's columns, rows 2 * warp +
+      // lane / 16 of each 32-row pass, the lane's 4 columns
       const int scols = H / 32;
       const int col_tiles = (scols + 3) / 4;
       float2 wv[2];
       unpack4x2(nw, wv);
-      for (int c = 0; c < nch; ++c) {
+      for (int r0 = 0; r0 < R; r0 += 2 * kWorkWarps) {
         // every lane takes part in the block shuffles; rows past R store nothing
-        const int r = c * kRC + rl;
+        const int r = r0 + warp * 2 + (lane >> 4);
         const bool valid = r < R;
-        const float* mix = mix_s + (valid ? r : 0) * MIX;
+        const int rr = valid ? r : 0;
+        const float* mix = mix_s + rr * MIX;
         // the collapse recomputed from the staged bf16 streams exactly as its squares were summed
         float2 cc[2];
         if (FRONT == kBroadcast) {
-          unpack4x2(lds_v2(v_s + sw128_offset(r, v)), cc);
+          unpack4x2(lds_v2(v_s + sw128_offset(rr, v)), cc);
         } else {
           cc[0] = cc[1] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int j = 0; j < N; ++j) {
             float2 f[2];
-            unpack4x2(lds_v2(v_s + j * L.r_alloc * 128 + sw128_offset(r, v)), f);
+            unpack4x2(lds_v2(v_s + j * L.r_alloc * 128 + sw128_offset(rr, v)), f);
             const float pj = mix[N + N * N + j];
 #pragma unroll
             for (int t = 0; t < 2; ++t) cc[t] = __ffma2_rn(make_float2(pj, pj), f[t], cc[t]);
           }
         }
-        const float inv = inv_s[valid ? r : 0];
-        float y[4] = {cc[0].x * inv * wv[0].x, cc[0].y * inv * wv[0].y, cc[1].x * inv * wv[1].x,
-                      cc[1].y * inv * wv[1].y};
+        const float inv = inv_s[rr];
+        const float y[4] = {cc[0].x * inv * wv[0].x, cc[0].y * inv * wv[0].y, cc[1].x * inv * wv[1].x,
+                            cc[1].y * inv * wv[1].y};
         const uint2 yb = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
         if (valid) st_v2(p.layer_input + static_cast<size_t>(r) * H + h0, yb);
         if (p.q_data != nullptr) {
@@ -953,17 +993,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-    // CTA 0 has now seen a published word of every cluster, so every CTA of this
-    // launch has read the epoch: the next launch may use the next tag.
-    if (g == 0) {
-      __syncthreads();
-      if (tid == 0) p.ctl[kEpochWord] = tag;
-    }
-    cluster_wait_acquire();  // no CTA leaves while the cluster may still read its shared memory
+    // CTA 0 has read row 0's records from every CTA, so every CTA of this launch
+    // has read the epoch: the next launch may use the next tag.
+    if (g == 0 && tid == 0) p.ctl[kEpochWord] = tag;
   } else {
     griddep_launch_dependents();
   }
 }
+
 
 // Mailbox of a consumer (one per rank of a TP group, in that rank's memory):
 // a 256-byte header (the status word at byte 0, the consumed round + 1 per parity
@@ -1151,16 +1188,17 @@ int g_extra_tx = 0;
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// The cluster sizes a launch over G CTAs may use: the largest of 8, 4, 2 that
-// divides G, falling back to smaller ones (down to the workspace's smallest, 2
-// for even G, 1 for odd G) when the larger clusters cannot all be resident.
-inline int smallest_cluster(int G) { return G % 2 == 0 ? 2 : 1; }
-
+// Workspace bytes: the header, then [G][R][fields] and [R] tagged words.
 size_t ws_layout(int R, int H, int n) {
-  (void)n;
-  const int G = H / kCols;
-  const size_t nc = static_cast<size_t>(G / smallest_cluster(G));
-  return kWsHeader + nc * static_cast<size_t>(R) * kRecF * 8;
+  const size_t G = static_cast<size_t>(H / kCols);
+  return kWsHeader + static_cast<size_t>(fields_of(n) + 1) * G * static_cast<size_t>(R) * 8;
+}
+
+// The workspace's parts for a call of p.R rows over p.H columns.
+void set_workspace(Params& p, void* ws, int n) {
+  p.ctl = static_cast<unsigned*>(ws);
+  p.rec = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kWsHeader);
+  p.tot = p.rec + static_cast<size_t>(p.H / kCols) * p.R * fields_of(n);
 }
 
 bool shape_ok(int R, int H, int n) {
@@ -1236,8 +1274,8 @@ struct Sources {
 constexpr int kSmemMax = 227 * 1024;  // the largest dynamic shared memory a block may have
 
 std::mutex g_cfg_mu;
-// (kernel, device, smem bytes, cluster) -> whether all clusters of a grid can be resident
-std::map<std::tuple<const void*, int, int, int, int>, bool> g_fit;
+// (kernel, device, grid, smem bytes) -> whether every CTA of the grid can be resident
+std::map<std::tuple<const void*, int, int, int>, bool> g_fit;
 
 // The kernel's shared-memory limit and carveout, set once per kernel and device.
 std::map<std::pair<const void*, int>, bool> g_configured;
@@ -1257,29 +1295,20 @@ bool configure(Kern kern, int dev) {
   return true;
 }
 
-// Whether `grid` CTAs in clusters of `cl` can all be resident at once (every
-// CTA waits, bounded, for the others' published sums).
+// Whether all `grid` CTAs can be resident at once (every CTA waits, bounded, for
+// the others' published records).
 template <typename Kern>
-bool clusters_fit(Kern kern, int dev, int grid, int cl, int smem) {
-  const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), dev, grid, cl, smem);
+bool blocks_fit(Kern kern, int dev, int grid, int smem) {
+  const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), dev, grid, smem);
   {
     std::lock_guard<std::mutex> lock(g_cfg_mu);
     auto it = g_fit.find(key);
     if (it != g_fit.end()) return it->second;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  bool ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n * cl >= grid;
+  int per_sm = 0, sms = 0;
+  const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) == cudaSuccess &&
+                  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                  per_sm * sms >= grid;
   (void)cudaGetLastError();
   std::lock_guard<std::mutex> lock(g_cfg_mu);
   g_fit[key] = ok;
@@ -1329,40 +1358,34 @@ mhc_status launch_boundary(Params& p, const Sources& src, cudaStream_t stream) {
     if (!make_map(&maps[2], p.gemm2, 2, dims, strides, box)) return MHC_ERR_CUDA;
   }
 
-  // cluster size and shared memory: the largest cluster whose grid can be resident
-  const int cmin = smallest_cluster(G);
-  int cl = 0, smem = 0;
-  for (int c : {8, 4, 2, 1}) {
-    if (c < cmin || G % c != 0) continue;
-    for (int st = kMaxStages; st >= 1 && cl == 0; --st) {
-      const Layout L = layout_of<N>(FRONT, R, p.P, p.topk, coeff, layer, G / c, st);
-      const int bytes = L.total + 1024;
-      if (bytes > kSmemMax) continue;
-      if (clusters_fit(kern, dev, G, c, bytes)) {
-        cl = c;
-        smem = bytes;
-        p.stages = st;
-      }
-    }
-    if (cl != 0) break;
+  // stages in flight: as many as the chunks need and shared memory holds, with
+  // every CTA of the grid resident
+  const int nch = (R + kRC - 1) / kRC;
+  int smem = 0;
+  p.stages = 0;
+  for (int st = nch < kMaxStages ? nch : kMaxStages; st >= 1; --st) {
+    // a stage that is refilled serves one group only: an even count, or one stage
+    // and one group
+    if (st < nch && st % 2 == 1 && st != 1) continue;
+    const Layout L = layout_of<N>(FRONT, R, G, p.P, p.topk, coeff, layer, st, p.fn_packed != nullptr);
+    const int bytes = L.total + 1024;
+    if (bytes > kSmemMax || !blocks_fit(kern, dev, G, bytes)) continue;
+    smem = bytes;
+    p.stages = st;
+    break;
   }
-  if (cl == 0) return MHC_ERR_UNSUPPORTED_SHAPE;
-  p.CL = cl;
+  if (p.stages == 0) return MHC_ERR_UNSUPPORTED_SHAPE;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cl;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, p, maps[0], maps[1], maps[2]) != cudaSuccess) {
     (void)cudaGetLastError();
     return MHC_ERR_CUDA;
@@ -1440,8 +1463,7 @@ mhc_status fill_tail(Params& p, const float* pre, const mhc_bf16* norm_weight, f
     p.comb_out = comb_out;
     p.pre_out = pre_out;
   }
-  p.ctl = static_cast<unsigned*>(ws);
-  p.rec = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kWsHeader);
+  set_workspace(p, ws, n);
   return MHC_OK;
 }
 
@@ -1752,8 +1774,7 @@ mhc_status mhc_coeffs(const mhc_bf16* residual, const mhc_coeff_args* coeffs, co
   p.post_out = post_out;
   p.comb_out = comb_out;
   p.pre_out = pre_out;
-  p.ctl = static_cast<unsigned*>(workspace);
-  p.rec = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + kWsHeader);
+  set_workspace(p, workspace, hc_mult);
   if (layer_input) {
     if (!norm_weight || !aligned(norm_weight, 16) || !aligned(layer_input, 16) || !(norm_eps >= 0.f))
       return MHC_ERR_INVALID_ARG;
@@ -1966,10 +1987,11 @@ namespace {
 constexpr int kNoAllocMaxRows = 128;
 constexpr int kNoAllocMaxHidden = 7168;
 constexpr int kNoAllocMaxHc = 4;
-// 1,893,376 bytes: more than mhc_workspace_bytes(128, 7168, 4) (the header and
-// the row records of 56 two-CTA clusters, the smallest clusters a launch over
-// 112 CTAs falls back to)
-constexpr size_t kNoAllocBytes = 1893376;
+// 3,097,600 bytes: mhc_workspace_bytes(128, 7168, 4), the header, the row
+// records [112 CTAs][128 rows][26 fields] and the totals [112 copies][128 rows]
+constexpr size_t kNoAllocBytes =
+    kWsHeader + static_cast<size_t>(fields_of(kNoAllocMaxHc) + 1) * (kNoAllocMaxHidden / kCols) * kNoAllocMaxRows * 8;
+static_assert(kNoAllocBytes == 3097600, "the no-alloc scratch size");
 
 // The array is zero at module load, as a workspace must be before first use
 // (mhc_workspace_init): the status word, and the launch epoch that tags the

@@ -57,19 +57,23 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       : "memory");
 }
 
+// Test phase `parity` of `bar`; while it is incomplete the thread is suspended
+// (up to the hint, 1 ms, and woken when the phase completes) rather than spinning,
+// so waiting warps take no issue slots from working ones.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   unsigned ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`, giving up at `deadline` (clock64 cycles).
+// Wait for phase `parity` of `bar`, giving up at `deadline` (clock64 cycles; each
+// test may sleep up to 1 ms, so the wait ends by deadline + 1 ms).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, long long deadline) {
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() > deadline) return false;
@@ -145,6 +149,30 @@ __device__ __forceinline__ bool has_neg_zero(const uint2 v) {
 __device__ __forceinline__ unsigned clear_neg_zero2(unsigned w) { return w & __vcmpne2(w, kNegZero2); }
 __device__ __forceinline__ void st_v2(void* p, uint2 v) {
   asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {  // L2 only: data other agents write
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_volatile_v4(const void* p) {  // re-read on every call
+  uint4 v;
+  asm volatile("ld.volatile.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ bool has_neg_zero4(const uint4 v) {
+  return (__vcmpeq2(v.x, kNegZero2) | __vcmpeq2(v.y, kNegZero2) | __vcmpeq2(v.z, kNegZero2) |
+          __vcmpeq2(v.w, kNegZero2)) != 0u;
+}
+// 8 bf16 as four column pairs: f[m] = (element 2m, element 2m + 1).
+__device__ __forceinline__ void unpack8x2(const uint4 v, float2 (&f)[4]) {
+  f[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
+  f[1] = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+  f[2] = make_float2(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u));
+  f[3] = make_float2(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
 }
 // 4 bf16 as two column pairs: f[m] = (element 2m, element 2m + 1).
 __device__ __forceinline__ void unpack4x2(const uint2 v, float2 (&f)[2]) {
@@ -252,10 +280,27 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
+// Bulk copy from this CTA's shared memory into CTA-of-the-cluster shared memory
+// (dst and bar are addresses from dsmem_addr); completion is counted in bytes on
+// the destination CTA's mbarrier. src, dst and bytes multiples of 16.
+__device__ __forceinline__ void bulk_s2dsmem(uint32_t dst, const void* src, unsigned bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk copy of this thread has read its source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Make this CTA's mbarrier initialisations visible to the cluster (before a
+// relaxed cluster arrive).
+__device__ __forceinline__ void fence_mbarrier_init_cluster() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Arrive on the cluster barrier without ordering memory (the start-up barrier
+// that makes every CTA of the cluster resident before shared memory is shared).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tagged words between CTAs
@@ -270,6 +315,13 @@ __device__ __forceinline__ void st_tagged(unsigned long long* p, uint32_t tag, f
 __device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
   unsigned long long w;
   asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+// Two consecutive tagged words (16-byte aligned); each word is read as one
+// single-copy atomic access.
+__device__ __forceinline__ ulonglong2 ld_tagged2(const unsigned long long* p) {
+  ulonglong2 w;
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p) : "memory");
   return w;
 }
 __device__ __forceinline__ uint32_t tag_of(unsigned long long w) { return static_cast<uint32_t>(w >> 32); }

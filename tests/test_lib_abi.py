@@ -50,9 +50,12 @@ def test_sizes(L):
     assert M.mhc_mxfp8_scale_bytes(5, 7168, False) == 5 * 224
     assert M.mhc_mxfp8_scale_bytes(5, 100, True) == 0
     ws = M.mhc_workspace_bytes(32, 7168, 4)
-    # a 1 KB header and, per row, a 32-word record (8-byte tagged words) of each of
-    # up to 56 two-CTA clusters over the 112 column blocks
-    assert ws == 1024 + 56 * 32 * 32 * 8
+    # a 1 KB header, then per row the record of each of the 112 column blocks
+    # (C + 2 fields, 8-byte tagged words, rounded up to an even count: 26, 10, 6)
+    # and one copy of the row's total per block
+    assert ws == 1024 + (26 + 1) * 112 * 32 * 8
+    assert M.mhc_workspace_bytes(32, 7168, 2) == 1024 + (10 + 1) * 112 * 32 * 8
+    assert M.mhc_workspace_bytes(32, 7168, 1) == 1024 + (6 + 1) * 112 * 32 * 8
     assert M.mhc_workspace_bytes(16, 7168, 4) <= ws  # smaller rows fit a larger workspace
     for bad in ((0, 7168, 4), (129, 7168, 4), (4, 7100, 4), (4, 7168, 3), (4, 7168, 8), (4, 9536, 4)):
         assert M.mhc_workspace_bytes(*bad) == 0
