@@ -125,12 +125,8 @@ typedef struct {
 } mhc_mxfp8_out;
 
 /* Bytes of workspace the boundary entry points need for (rows, hidden, hc_mult):
- * a 1 KB header (the status word kernels record errors in, the launch epoch)
- * and the per-block row records that the tail of a boundary adds up: F fields
- * (C = 2n + n*n dot products, sum v^2, sum c^2; F = C + 2 rounded up to even) of
- * each row from each of the G = H/64 column blocks, then the rows' totals of sum
- * c^2, one copy per block, 8-byte words, 1024 + (F + 1) * G * rows * 8 bytes in
- * all. A workspace sized for R rows
+ * a 1 KB header (the status word kernels record errors in) and the per-block
+ * partial sums that the tail of a boundary adds up. A workspace sized for R rows
  * serves every call with rows <= R and the same hidden and hc_mult. It must be
  * 256-byte aligned, zeroed once before first use (mhc_workspace_init; the
  * partial sums are rewritten by every call) and used by one stream at a time:
@@ -332,7 +328,7 @@ MHC_API mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden,
  * tensors), code running while a CUDA graph is captured (cudaMalloc is not a
  * stream operation), or a serving loop that must not take the allocator's locks.
  * Arguments and results are those of mhc_boundary_post_pre without the
- * workspace: the scratch is a fixed device array inside the library, 3,097,600
+ * workspace: the scratch is a fixed device array inside the library, 1,893,376
  * bytes (the workspace of rows 128, hidden 7168, hc_mult 4), which every GPU
  * that loads the library holds until the process exits. Limits: rows <= 128,
  * hidden <= 7168, hc_mult <= 4; larger shapes return MHC_ERR_WORKSPACE.

@@ -1,38 +1,32 @@
 // mHC decode boundary on B200 (sm_100a): the fused kernel and the C ABI of
 // libmhc.so (declared in include/mhc.h).
 //
-// A boundary is ONE launch of boundary_kernel over G = H/64 CTAs, one per SM.
-// CTA g owns columns [64g, 64g + 64) of every row, so every weight of fn is
-// read from HBM exactly once per boundary.
-//   1. Before it waits for its predecessor on the stream (programmatic dependent
-//      launch), a CTA starts the bulk copy of its fn slice (fp32) into shared
-//      memory.
-//   2. After the wait, tensor-map TMA loads bring the rows' data into shared
-//      memory in 16-row chunks, up to four in flight: the partials (one 3-D
-//      box), or the MoE expert rows gathered by index (tile::gather4) and the
-//      shared output, and the residual streams (one 3-D box). While they are in
-//      flight the CTA splits each fn weight into three bf16 terms (128B-swizzled
-//      rows of K values, one row per term and fn column).
-//   3. Two groups of eight warps take alternate chunks: sum or finalize x, mHC
-//      post-mix (vllm ...boundary.boundary, Boundaries.post_only: mhc_post(x,
-//      residual, post, comb)), store the new streams, stage them in shared
-//      memory, and sum per row the squares of their collapse with the carried
-//      pre (BoundaryState.pre) and of the streams.
-//   4. The same warps project the chunk's 16 rows of staged streams onto the C
-//      fn columns on the tensor cores (mma.sync m16n8k16 bf16, fp32
-//      accumulation; each warp a share of K, the shares added in warp order),
-//      while a control warp refills the chunk's stage.
-//   5. Each CTA publishes its row records (C dot products, sum v^2, sum c^2) as
-//      tagged 64-bit words in the workspace, field-major, so that one field of
-//      one row is contiguous over the CTAs (no flag, no fence, no second kernel).
-//   6. In one round over the published words every CTA adds the sum of c^2 of
-//      every row and the records of the rows whose coefficients it finishes
-//      (rows g and g + G), writes its columns of the layer input (and MXFP8),
-//      and runs those rows' logits, sigmoid and Sinkhorn.
-// The residual-only variant is steps 2-3 alone. Every reduction runs in a fixed
-// order, so results are bitwise reproducible.
+// A boundary is two launches chained by programmatic dependent launch (PDL).
+// The streaming kernel (boundary_kernel): block g owns columns [64g, 64g+64)
+// of H for every row, so each weight of fn is read from HBM exactly once.
+//   1. A TMA bulk copy brings the block's fn slice into shared memory (packed
+//      bf16 terms, or fp32 that the block splits into bf16 terms) and the
+//      block's activations are prefetched into L2, both before the kernel waits
+//      for its predecessor on the stream;
+//   2. per (row, 4 columns) a lane sums the partials (local buffers, peers'
+//      buffers, or the slots of a publish/collect mailbox as they fill) or
+//      finalizes the MoE output, applies the mHC post-mix (vllm
+//      ...boundary.boundary, Boundaries.post_only: mhc_post(x, residual, post,
+//      comb)), rounds the new streams to bf16, stores them, sums the squares of
+//      their collapse with the carried pre (BoundaryState.pre) and of the streams;
+//   3. the block projects its rows' n*64 stream values onto the C fn columns on
+//      the tensor cores (mma.sync bf16, fn as three bf16 terms; single or paired
+//      16-row tiles per warp by row count) and writes its partial sums to the
+//      workspace.
+// The tail kernel (boundary_tail_kernel), once the streaming kernel is done:
+//   4. layer-input blocks normalise 256-column tasks of the rows into the layer
+//      input (and MXFP8); beside them, coefficient blocks (placed first for 4-32
+//      rows, so that they start on the SMs the streaming kernel leaves free)
+//      finish the rows' coefficients (logits, sigmoid, Sinkhorn on scale vectors
+//      in one thread per row).
+// The residual-only variant is the streaming kernel alone. All reductions run
+// in a fixed order, so results are bitwise reproducible.
 
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -47,68 +41,61 @@
 
 namespace mhc {
 
-constexpr int kCols = 64;        // columns of H per CTA
-constexpr int kRC = 16;          // rows per chunk (N of one projection MMA)
-constexpr int kMaxStages = 4;    // chunks in flight (fewer where they do not fit in shared memory)
-constexpr int kWorkWarps = 16;   // warps of the streaming phase: two groups of 8 on alternate chunks
-constexpr int kGroupWarps = 8;   // a group: 2 rows of a chunk per warp, 4 columns per lane
-constexpr int kCtl = kWorkWarps; // index of the control warp
-constexpr int kThreads = (kWorkWarps + 1) * 32;
-constexpr int kWorkThreads = kWorkWarps * 32;
+constexpr int kCols = 64;      // columns of H per block
+constexpr int kThreads = 256;  // 8 warps
+constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRows = 128;
-constexpr int kMaxChunks = kMaxRows / kRC;
 constexpr int kMaxPartials = 16;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxIters = 1000;
-constexpr int kMaxBlocks = 148;
-constexpr int kRecF = 32;        // shared-memory stride of a row record: C dot products, sum v^2, sum c^2
-// Workspace: a 1 KB header (status word at byte 0, the launch epoch at byte 64),
-// then the CTAs' row records as tagged 64-bit words, [G CTAs][R rows][fields],
-// then the rows' total sums of c^2, one copy for each CTA to read, [G][R].
+constexpr int kMaxBlocks = 148;  // most H/64 blocks: the tail's per-lane loads are sized for it
+// Workspace header: the status word (byte 0); the partial sums follow.
 constexpr size_t kWsHeader = 1024;
 constexpr int kStatusWord = 0;
-constexpr int kEpochWord = 16;
 
-enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3, kMailbox = 4, kTable = 5 };
-// Fronts whose x is a sum of P bf16 partials read by the lanes themselves (a table
-// of pointers that may be other GPUs' memory, or the slots of a mailbox that
+enum Front { kPartials = 0, kMoe = 1, kStreams = 2, kBroadcast = 3, kMailbox = 4 };
+// Fronts whose x is a sum of P bf16 partials (kMailbox: slots of a mailbox that
 // producers fill concurrently, each element valid once it is not negative zero).
-__host__ __device__ constexpr bool lane_partials(int front) { return front == kMailbox || front == kTable; }
+__host__ __device__ constexpr bool sums_partials(int front) { return front == kPartials || front == kMailbox; }
 
 __host__ __device__ constexpr int logits_of(int n) { return 2 * n + n * n; }
-// Fields of a published row record: C dot products, sum v^2 and sum c^2, rounded
-// up to an even count (records are read as 16-byte pairs of words).
-__host__ __device__ constexpr int fields_of(int n) { return (logits_of(n) + 3) & ~1; }
-// rows of the fn slice image: three bf16 terms of each of the C fn columns (row
-// t*C + c), rounded up to a whole 8-row swizzle atom
-__host__ __device__ constexpr int arows_of(int n) { return (3 * logits_of(n) + 7) & ~7; }
-// Bytes of a CTA's fn slice image (mhc_projection_pack).
-__host__ __device__ constexpr int aimage_bytes(int n) { return n * arows_of(n) * 128; }
+// logit count padded to a multiple of 4 (the tail's base array in shared memory)
+__host__ __device__ constexpr int cpad_of(int n) { return (logits_of(n) + 3) & ~3; }
+// Per-block record of a row in the workspace: C dot products, then sum v^2,
+// padded to a power of two >= 8 floats.
+__host__ __device__ constexpr int red_of(int n) {
+  return logits_of(n) + 1 <= 8 ? 8 : (logits_of(n) + 1 <= 16 ? 16 : 32);
+}
+// fp32 fn slice in shared memory as the bulk copies land it (unpacked fn): pieces
+// of 8 rows of C floats followed by a 16-byte gap, which spreads the split
+// loop's reads over the banks.
+__host__ __device__ constexpr int fn_piece_bytes(int n) { return 8 * logits_of(n) * 4 + 16; }
 
 struct Params {
   // front ends
-  const __nv_bfloat16* pptr[kMaxPartials];  // lane-read partials: [R, H] at pptr[u]
+  const __nv_bfloat16* pptr[kMaxPartials];  // partial u: [R, H] at pptr[u]
+  int premote;  // partials may be other GPUs' memory: L2-only loads, no prefetch
   int P;
-  int premote;  // partials may be other GPUs' memory (L2-only loads)
   const __nv_bfloat16* gemm2;
   int num_perm;
   const float* ew;
   const int32_t* e2p;
   int topk;
+  const __nv_bfloat16* shared_out;
+  const __nv_bfloat16* residual;
+  const __nv_bfloat16* x;
   const float* post;
   const float* comb;
   const float* pre;  // carried pre (boundary) or pre_mix (coefficients entry)
-  // layer input
+  // tail
   const __nv_bfloat16* norm_weight;
   float norm_eps;
-  // coefficients
   const float* fn;
-  const unsigned char* fn_packed;  // [G] A operand images, or null
+  const __nv_bfloat16* fn_packed;  // [G][3][CP8][n*64 + 8] bf16 terms of fn, or null
   const float* scale;
   const float* base;
   float rms_eps, pre_eps, sk_eps, alpha;
   int iters;
-  // outputs
   __nv_bfloat16* residual_out;
   __nv_bfloat16* aux_out;  // stream mean of the new streams [R, H], or null
   __nv_bfloat16* layer_input;
@@ -120,86 +107,84 @@ struct Params {
   float* pre_out;
   int R, H;
   int write_res, do_layer, do_coeff;
-  int stages;  // chunk stages in flight: 1 .. kMaxStages
   // workspace
-  unsigned* ctl;             // header: status, epoch
-  unsigned long long* rec;   // [G][R][fields] tagged words: the CTAs' row records
-  unsigned long long* tot;   // [G][R] tagged words: the rows' sums c^2, one copy per CTA
+  unsigned* ctl;
+  float* sc2_part;  // [R][G]
+  float* dot_part;  // [R][G][RED]
+  // the streams the tail normalises: the new streams, the given streams, or the
+  // embedding of the first layer (whose identity pre-mix selects it)
+  const __nv_bfloat16* tail_streams;
+  int tail_broadcast;
+  int tail_layer_blocks;  // tail blocks that write the layer input (at most G, or 0)
+  int tail_coeff_blocks;  // tail blocks that finish the coefficients of rows j, j + this, ...
+  int tail_coeff_first;   // coefficient blocks take the tail's first block indices
   int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
   int64_t budget_ns;
 };
 
-// Shared memory of the kernel, offsets from a 1024-byte aligned base.
-struct Layout {
-  int a_off, v_off, st_off, stage_bytes, res_units, fst_off, part_off, mix_off, moe_off, rec_off, inv_off, cft_off,
-      bar_off, total;
-  int r_alloc;
+struct SmemLayout {
+  int fn_off, bs_off, v_off, mix_off, moe_off, misc_off, total;
 };
 
-// Bytes of one chunk's projection partials: [warp][16 rows][C] floats.
-__host__ __device__ constexpr int part_bytes(int n) { return kGroupWarps * kRC * logits_of(n) * 4; }
+// Projection operands: n-tiles of 8 logit columns; staged stream rows and fn
+// columns are n*64 bf16 plus a 16-byte gap (ldmatrix rows in distinct banks).
+__host__ __device__ constexpr int ntiles_of(int n) { return (logits_of(n) + 7) / 8; }
+__host__ __device__ constexpr int kstride_of(int n) { return n * kCols + 8; }
 
-// 128-byte box rows of one chunk's stage, and where the residual streams start.
-__host__ __device__ inline void stage_units(int front, int n, int P, int topk, int* units, int* res_units) {
-  int u = 0, ru = 0;
-  switch (front) {
-    case kPartials: ru = P * kRC; u = ru + n * kRC; break;
-    case kMoe: ru = (topk + 1) * kRC; u = ru + n * kRC; break;
-    case kBroadcast: ru = 0; u = kRC; break;
-    default: ru = 0; u = n * kRC; break;  // streams, table, mailbox: the residual streams only
-  }
-  *units = u;
-  *res_units = ru;
+// Shared memory of the streaming kernel (packed: fn arrives already split, so
+// the fp32 staging area is not needed).
+template <int N>
+__host__ __device__ inline SmemLayout smem_layout(int R, int topk, bool moe, bool packed) {
+  constexpr int CP8 = ntiles_of(N) * 8;
+  SmemLayout L{};
+  int o = 0;
+  L.fn_off = o;  // fn slice as the bulk copies land it
+  if (!packed) o += N * 8 * fn_piece_bytes(N);
+  L.bs_off = o;  // fn slice as three bf16 terms, [3][CP8][n*64 + 8]
+  o += 3 * CP8 * kstride_of(N) * 2;
+  L.v_off = o;  // new streams, bf16 [roundup(R, 16)][n*64 + 8]
+  o += ((R + 15) & ~15) * kstride_of(N) * 2;
+  L.mix_off = o;  // [R][post n | comb n*n | pre n]
+  o += R * (2 * N + N * N) * 4;
+  o = (o + 15) & ~15;
+  L.moe_off = o;
+  if (moe) o += R * topk * 8;
+  o = (o + 15) & ~15;
+  L.misc_off = o;  // mbarrier
+  o += 16;
+  L.total = o;
+  return L;
 }
 
+// Shared memory of the tail kernel.
+struct TailLayout {
+  int part_off, cst_off, total;
+};
+
 template <int N>
-__host__ __device__ inline Layout layout_of(int front, int R, int G, int P, int topk, bool coeff, bool layer,
-                                          int stages, bool packed) {
-  constexpr int C = logits_of(N);
-  Layout L{};
-  L.r_alloc = (R + kRC - 1) / kRC * kRC;
+__host__ __device__ inline TailLayout tail_layout() {
+  constexpr int CP = cpad_of(N);
+  TailLayout L{};
   int o = 0;
-  L.a_off = o;  // fn slice image [n atom columns][arows][128 B]
-  if (coeff) o += aimage_bytes(N);
-  // new streams [n atom columns][r_alloc][128 B]; until the first chunk is
-  // staged, the fp32 fn slice as copied, [n][64][C]
-  L.v_off = L.fst_off = o;
-  int vb = (coeff || layer) ? N * L.r_alloc * 128 : 0;
-  if (coeff && !packed && vb < N * kCols * C * 4) vb = N * kCols * C * 4;
-  o += vb;
-  L.st_off = o;  // chunk stages
-  int units, ru;
-  stage_units(front, N, P, topk, &units, &ru);
-  L.stage_bytes = units * 128;
-  L.res_units = ru;
-  // after the last chunk, the row records this CTA adds up: [ceil(R / G) * G][fields]
-  int st = stages * L.stage_bytes;
-  if ((coeff || layer) && st < (R + G - 1) / G * G * fields_of(N) * 4) st = (R + G - 1) / G * G * fields_of(N) * 4;
-  o += st;
-  // a chunk's projection partials go into its consumed stage when they fit
-  // (the stage is refilled only once the chunk is done), else here, one
-  // buffer per group
-  L.part_off = -1;
-  if (coeff && L.stage_bytes < part_bytes(N)) {
-    L.part_off = o;
-    o += 2 * part_bytes(N);
-  }
-  L.mix_off = o;  // [R][post n | comb n*n | pre n]
-  o += (R * (2 * N + N * N) * 4 + 15) & ~15;
-  L.moe_off = o;  // e2p [R*topk], weights [R*topk]
-  if (front == kMoe) o += (R * topk * 8 + 15) & ~15;
-  L.rec_off = o;  // this CTA's row records [R][kRecF]
-  if (coeff || layer) o += R * kRecF * 4;
-  L.inv_off = o;  // [R] inverse RMS of the collapse
-  if (layer) o += (R * 4 + 15) & ~15;
-  L.cft_off = o;  // [ceil(R / G)][kRecF] the totals of the rows this CTA adds up
-  if (coeff || layer) o += (R + G - 1) / G * kRecF * 4;
-  L.bar_off = o;  // full[kMaxStages], vready[kMaxChunks], fnbar, then the tag slot
-  o += (kMaxStages + kMaxChunks + 1) * 8 + 16;
+  L.part_off = o;  // [kWarps rows][kWarps][RED] floats: the warps' shares of a row's records
+  o += kWarps * kWarps * red_of(N) * 4;
+  L.cst_off = o;  // scale[4], base[CP]
+  o += (4 + CP) * 4;
   L.total = (o + 15) & ~15;
   return L;
 }
 
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  return v;
+}
+
+__device__ __forceinline__ float sum16_lanes(float v) {  // over the 16 lanes sharing lane bit 4
+#pragma unroll
+  for (int m = 8; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  return v;
+}
 
 __device__ __forceinline__ int swizzled_scale_offset(int r, int c, int col_tiles) {
   const int tile = (r >> 7) * col_tiles + (c >> 2);
@@ -207,19 +192,68 @@ __device__ __forceinline__ int swizzled_scale_offset(int r, int c, int col_tiles
   return tile * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (c & 3);
 }
 
-// Byte offset of (row, 4-column group v of 16) in a 128B-swizzled K-major atom
-// column: rows of 128 bytes, 16-byte chunk index XOR-ed with row % 8.
-__device__ __forceinline__ int sw128_offset(int row, int v) {
-  return row * 128 + ((((v >> 1) ^ row) & 7) << 4) + (v & 1) * 8;
+// Registers of one row-pair step of a lane (4 columns of one row): the stream
+// vectors and up to 8 partial (or gathered) vectors, plus the shared-output /
+// embedding vector.
+template <int N>
+struct PairLoads {
+  uint2 rv[N];
+  uint2 pv[8];
+  uint2 sv;
+};
+// The streaming kernel runs 16 warps; a warp covers a row pair x 64 columns,
+// a lane 4 columns of one row.
+constexpr int kT1 = 512;
+constexpr int kW1 = kT1 / 32;
+
+template <int N, int FRONT>
+__device__ __forceinline__ void load_pair(const Params& p, int r, int h0, const int* e2p_s, PairLoads<N>& Q) {
+  const int H = p.H;
+  if (r >= p.R) return;
+  if constexpr (FRONT == kBroadcast) {
+    Q.sv = ld_nc_v2(p.x + static_cast<size_t>(r) * H + h0);
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; ++j) Q.rv[j] = ld_v2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
+  }
+  if (sums_partials(FRONT)) {
+    const size_t off = static_cast<size_t>(r) * H + h0;
+    if (FRONT == kMailbox || p.premote) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < p.P) Q.pv[u] = ld_cg_v2(p.pptr[u] + off);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < p.P) Q.pv[u] = ld_nc_v2(p.pptr[u] + off);
+    }
+  } else if (FRONT == kMoe) {
+    Q.sv = ld_nc_v2(p.shared_out + static_cast<size_t>(r) * H + h0);
+    const int* idx = e2p_s + r * p.topk;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (u < p.topk) {
+        const int e = idx[u];
+        Q.pv[u] = (e >= 0 && e < p.num_perm) ? ld_nc_v2(p.gemm2 + static_cast<size_t>(e) * H + h0)
+                                             : make_uint2(0, 0);
+      }
+    }
+  }
 }
 
-__device__ __forceinline__ uint2 lds_v2(const void* p) { return *reinterpret_cast<const uint2*>(p); }
-
-__device__ __forceinline__ void named_sync_workers() {  // the streaming warps (groups use barriers 1 and 2)
-  asm volatile("bar.sync 3, %0;" ::"n"(kWorkThreads) : "memory");
+// A mailbox slot's 4 elements as loaded, re-read until none is negative zero
+// (bounded: on timeout the status records it and the values are used as they are).
+__device__ __forceinline__ uint2 settle_slot(const __nv_bfloat16* src, uint2 v, long long deadline,
+                                             unsigned* status) {
+  while (has_neg_zero(v)) {
+    if (clock64() > deadline) {
+      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+      break;
+    }
+    v = ld_volatile_v2(src);
+  }
+  return v;
 }
-
-
 
 // fn as three bf16 terms, f = hi + mid + lo to 2^-24: each bf16 x bf16 product is
 // exact in fp32, so three tensor-core products return the fp32 projection up to
@@ -231,28 +265,415 @@ __device__ __forceinline__ void split3(float f, __nv_bfloat16& hi, __nv_bfloat16
   lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
 }
 
-// Eight consecutive K values (kin = 8*oct .. 8*oct + 7) of fn column c, read from
-// the fp32 slice [kin][C], written as the three terms' 16-byte chunks of A rows
-// c, C + c and 2C + c in atom column j.
-template <int N>
-__device__ __forceinline__ void split_octet(const float* slice, unsigned char* a_col, int c, int oct) {
+// Bytes of a block's packed fn slice: the B operand of the projection exactly as
+// it sits in shared memory, [3][CP8][n*64 + 8] bf16.
+__host__ __device__ constexpr int packed_slice_bytes(int n) { return 3 * ntiles_of(n) * 8 * kstride_of(n) * 2; }
+static_assert(packed_slice_bytes(1) % 16 == 0 && packed_slice_bytes(2) % 16 == 0 && packed_slice_bytes(4) % 16 == 0,
+              "a bulk copy moves a multiple of 16 bytes");
+
+// 80 registers a thread: 512 threads leave room on the SM for the tail kernel's
+// blocks, which launch early (programmatic dependent launch).
+// PAIRED: the projection takes pairs of row tiles (launched from four row tiles
+// on; a separate instantiation, so that the other keeps its registers and code).
+template <int N, int FRONT, bool PAIRED>
+__global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   constexpr int C = logits_of(N);
-  unsigned w[3][4];
-#pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    __nv_bfloat16 h0, m0, l0, h1, m1, l1;
-    split3(slice[(oct * 8 + e) * C + c], h0, m0, l0);
-    split3(slice[(oct * 8 + e + 1) * C + c], h1, m1, l1);
-    w[0][e / 2] = static_cast<unsigned>(__bfloat16_as_ushort(h0)) | (static_cast<unsigned>(__bfloat16_as_ushort(h1)) << 16);
-    w[1][e / 2] = static_cast<unsigned>(__bfloat16_as_ushort(m0)) | (static_cast<unsigned>(__bfloat16_as_ushort(m1)) << 16);
-    w[2][e / 2] = static_cast<unsigned>(__bfloat16_as_ushort(l0)) | (static_cast<unsigned>(__bfloat16_as_ushort(l1)) << 16);
+  constexpr int KC = N * kCols;       // stream values per row in this block
+  constexpr int KS = kstride_of(N);   // staged row stride (bf16)
+  constexpr int NT = ntiles_of(N);    // 8-column tiles of the projection
+  constexpr int CP8 = NT * 8;
+  constexpr int RED = red_of(N);
+  constexpr int MIX = 2 * N + N * N;
+  constexpr int PIECE = fn_piece_bytes(N);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe, p.fn_packed != nullptr);
+  unsigned char* fn_s = smem + L.fn_off;
+  __nv_bfloat16* bs_s = reinterpret_cast<__nv_bfloat16*>(smem + L.bs_off);
+  __nv_bfloat16* v_s = reinterpret_cast<__nv_bfloat16*>(smem + L.v_off);
+  float* mix_s = reinterpret_cast<float*>(smem + L.mix_off);
+  int* e2p_s = reinterpret_cast<int*>(smem + L.moe_off);
+  float* ew_s = reinterpret_cast<float*>(smem + L.moe_off) + p.R * p.topk;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.misc_off);
+
+  const int g = blockIdx.x;
+  const int G = gridDim.x;
+  const int H = p.H;
+  const int R = p.R;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rq = lane >> 4, vec = lane & 15;
+  const int h0 = g * kCols + vec * 4;  // this lane's 4 columns in the row-pair phase
+  const long long deadline = wait_deadline(p.budget_ns);
+  unsigned* status = p.ctl + kStatusWord;
+  const int npairs = (R + 1) >> 1;
+
+  // ---- 1. the block's fn slice by TMA bulk copies. Weights are never written by
+  // the kernel that precedes this one on the stream, so this runs before the
+  // wait on that kernel (programmatic dependent launch).
+  const bool packed = p.fn_packed != nullptr;
+  if (p.do_coeff) {
+    if (tid == 0) mbar_init(bar, 1);
+    __syncthreads();
+    if (packed) {  // pre-split terms (mhc_projection_pack): one copy, waited for at step 5
+      if (tid == 0) {
+        constexpr int PB = packed_slice_bytes(N);
+        mbar_arrive_expect_tx(bar, PB + 16 * p.extra_tx);
+        bulk_g2s(bs_s, reinterpret_cast<const unsigned char*>(p.fn_packed) + static_cast<size_t>(g) * PB, PB, bar);
+      }
+    } else if (warp == 0) {
+      if (lane == 0) mbar_arrive_expect_tx(bar, KC * C * 4 + 16 * p.extra_tx);
+      __syncwarp();
+      for (int m = lane; m < N * 8; m += 32) {
+        const int i = m >> 3, piece = m & 7;
+        bulk_g2s(fn_s + m * PIECE, p.fn + (static_cast<size_t>(i) * H + g * kCols + piece * 8) * C, 8 * C * 4, bar);
+      }
+    }
   }
+
+  // ---- 2. bring this block's activations into L2 while the preceding kernel may
+  // still run: a prefetch is only a hint and L2 is the point of coherence, so
+  // it is safe before the wait; gather indices read now only steer prefetches.
+  if (vec == 0 || vec == 15) {
+    for (int q = warp; q < npairs; q += kW1) {
+      const int r = q * 2 + rq;
+      if (r >= R) break;
+      if constexpr (FRONT == kBroadcast) {
+        prefetch_l2(p.x + static_cast<size_t>(r) * H + h0);
+      } else {
+        for (int j = 0; j < N; ++j) prefetch_l2(p.residual + (static_cast<size_t>(r) * N + j) * H + h0);
+      }
+      if (sums_partials(FRONT)) {  // (a mailbox's slots are this GPU's memory)
+        if (FRONT == kMailbox || !p.premote)
+          for (int pp = 0; pp < p.P; ++pp) prefetch_l2(p.pptr[pp] + static_cast<size_t>(r) * H + h0);
+      } else if (FRONT == kMoe) {
+        prefetch_l2(p.shared_out + static_cast<size_t>(r) * H + h0);
+        for (int t = 0; t < p.topk; ++t) {
+          int e = p.e2p[r * p.topk + t];
+          e = e < 0 ? 0 : (e >= p.num_perm ? p.num_perm - 1 : e);
+          if (p.num_perm > 0) prefetch_l2(p.gemm2 + static_cast<size_t>(e) * H + h0);
+        }
+      }
+    }
+  }
+
+  if (p.do_coeff && !packed) {
+    // Split the fn slice into three bf16 terms (split3), stored column-major for
+    // the MMA's B operand (weights only: before the wait).
+    const bool ok = mbar_wait_bounded(bar, 0, deadline);
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
+    for (int e = tid; e < CP8 * KC; e += kT1) {
+      const int c = e / KC, k = e - c * KC;
+      const float f = c < C ? reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4)[c] : 0.f;
+      __nv_bfloat16 hi, mid, lo;
+      split3(f, hi, mid, lo);
+      bs_s[(0 * CP8 + c) * KS + k] = hi;
+      bs_s[(1 * CP8 + c) * KS + k] = mid;
+      bs_s[(2 * CP8 + c) * KS + k] = lo;
+    }
+  }
+  if (warp == 1 && lane < 3) {  // the mixes' first lines: L2 and address translation warm before the wait
+    const float* mp = lane == 0 ? p.post : (lane == 1 ? p.comb : p.pre);
+    if (mp != nullptr) prefetch_l2(mp);
+  }
+  // ---- 3. wait for the preceding kernel, let the next one launch, and read
+  griddep_wait();
+  griddep_launch_dependents();
+  PairLoads<N> cur;  // the row data first: the longest round trip goes out first
+  if (FRONT != kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
+  for (int k = tid; k < R * MIX; k += kT1) {  // [R][post n | comb n*n | pre n]
+    const int r = k / MIX, c = k - r * MIX;
+    if (c < N + N * N) {
+      if (FRONT == kStreams || FRONT == kBroadcast) {
+        mix_s[k] = 0.f;
+      } else if (c < N) {
+        cp_async4(mix_s + k, p.post + r * N + c);
+      } else {
+        cp_async4(mix_s + k, p.comb + r * N * N + (c - N));
+      }
+    } else if (p.pre != nullptr) {
+      cp_async4(mix_s + k, p.pre + r * N + (c - N - N * N));
+    } else {
+      mix_s[k] = 0.f;
+    }
+  }
+  if (FRONT == kMoe) {
+    for (int k = tid; k < R * p.topk; k += kT1) {
+      cp_async4(e2p_s + k, p.e2p + k);
+      cp_async4(ew_s + k, p.ew + k);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (FRONT == kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);
+
+  // ---- 4. row pairs: sum / finalize, post-mix, store the streams, sum c^2
+  for (int q = warp; q < npairs; q += kW1) {
+    PairLoads<N> nxt;
+    if (q + kW1 < npairs) load_pair<N, FRONT>(p, (q + kW1) * 2 + rq, h0, e2p_s, nxt);
+    const int r = q * 2 + rq;
+    const bool valid = r < R;
+    const float* mix = mix_s + (valid ? r : 0) * MIX;
+    // Pairs of columns in packed f32x2 arithmetic (each element the same fp32
+    // operations, in the same order, as one at a time).
+    float2 nf[N][2];  // the new streams, as rounded to bf16
+    uint2 nb[N];
+    float2 xs[2];
 #pragma unroll
-  for (int t = 0; t < 3; ++t) {
-    const int m = t * C + c;
-    *reinterpret_cast<uint4*>(a_col + m * 128 + (((oct ^ m) & 7) << 4)) = make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+    for (int t = 0; t < 2; ++t) xs[t] = make_float2(0.f, 0.f);
+    if (sums_partials(FRONT) || FRONT == kMoe) {
+      float2 rf[N][2];
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < N; ++j) unpack4x2(cur.rv[j], rf[j]);
+        if (sums_partials(FRONT)) {
+          const size_t off = static_cast<size_t>(r) * H + h0;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (u < p.P) {
+              if (FRONT == kMailbox) cur.pv[u] = settle_slot(p.pptr[u] + off, cur.pv[u], deadline, status);
+              float2 f[2];
+              unpack4x2(cur.pv[u], f);
+#pragma unroll
+              for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
+            }
+          }
+          for (int u = 8; u < p.P; ++u) {  // partials beyond the first 8
+            float2 f[2];
+            const __nv_bfloat16* src = p.pptr[u] + off;
+            uint2 v = (FRONT == kMailbox || p.premote) ? ld_cg_v2(src) : ld_nc_v2(src);
+            if (FRONT == kMailbox) v = settle_slot(src, v, deadline, status);
+            unpack4x2(v, f);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
+          }
+          if (FRONT == kMailbox) {  // consumed: back to "not written" for the round after next
+            for (int u = 0; u < p.P; ++u)
+              st_v2(const_cast<__nv_bfloat16*>(p.pptr[u]) + off, make_uint2(kNegZero2, kNegZero2));
+          }
+        } else {
+          unpack4x2(cur.sv, xs);
+          const int* idx = e2p_s + r * p.topk;
+          const float* wt = ew_s + r * p.topk;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {  // the first 8 slots, loaded ahead
+            if (u < p.topk) {
+              const int e = idx[u];
+              if (e >= p.num_perm) {
+                if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
+              } else if (e >= 0) {
+                float2 f[2];
+                unpack4x2(cur.pv[u], f);
+                const float2 w2 = make_float2(wt[u], wt[u]);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
+              }
+            }
+          }
+          for (int u = 8; u < p.topk; ++u) {  // slots beyond 8
+            const int e = idx[u];
+            if (e >= p.num_perm) {
+              if (vec == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
+            } else if (e >= 0) {
+              float2 f[2];
+              unpack4x2(ld_nc_v2(p.gemm2 + static_cast<size_t>(e) * H + h0), f);
+              const float2 w2 = make_float2(wt[u], wt[u]);
+#pragma unroll
+              for (int t = 0; t < 2; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < N; ++j)
+#pragma unroll
+          for (int t = 0; t < 2; ++t) rf[j][t] = make_float2(0.f, 0.f);
+      }
+      // mHC post: new[i] = bf16(post[i] * x + sum_j comb[j][i] * res[j])
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        float2 a[2];
+        const float2 po = make_float2(mix[i], mix[i]);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          float2 s2 = __fmul2_rn(po, xs[t]);
+#pragma unroll
+          for (int j = 0; j < N; ++j) {
+            const float cj = mix[N + j * N + i];
+            s2 = __ffma2_rn(make_float2(cj, cj), rf[j][t], s2);
+          }
+          a[t] = s2;
+        }
+        nb[i] = make_uint2(pack_bf16x2(a[0].x, a[0].y), pack_bf16x2(a[1].x, a[1].y));
+        unpack4x2(nb[i], nf[i]);
+      }
+    } else if (FRONT == kStreams) {
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        nb[j] = valid ? cur.rv[j] : make_uint2(0, 0);
+        unpack4x2(nb[j], nf[j]);
+      }
+    } else {  // kBroadcast: every stream is the embedding row
+      const uint2 xv = valid ? cur.sv : make_uint2(0, 0);
+      unpack4x2(xv, xs);
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        nb[j] = xv;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) nf[j][t] = xs[t];
+      }
+    }
+    if (p.write_res && valid) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) st_v2(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
+    }
+    if (p.aux_out != nullptr && valid) {  // mean over the streams, in stream order, rounded once
+      constexpr float kInvN = 1.f / N;    // exact: n is a power of two
+      uint2 ab;
+      unsigned* aw = reinterpret_cast<unsigned*>(&ab);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        float2 m = nf[0][t];
+#pragma unroll
+        for (int j = 1; j < N; ++j) m = __fadd2_rn(m, nf[j][t]);
+        m = __fmul2_rn(m, make_float2(kInvN, kInvN));
+        aw[t] = pack_bf16x2(m.x, m.y);
+      }
+      st_v2(p.aux_out + static_cast<size_t>(r) * H + h0, ab);
+    }
+    if (p.do_layer) {  // collapse with the carried pre (identity pre-mix for the broadcast)
+      float2 sq = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        float2 c;
+        if (FRONT == kBroadcast) {
+          c = xs[t];
+        } else {
+          c = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < N; ++j) {
+            const float pj = mix[N + N * N + j];
+            c = __ffma2_rn(make_float2(pj, pj), nf[j][t], c);
+          }
+        }
+        sq = __ffma2_rn(c, c, sq);
+      }
+      const float sc2 = sum16_lanes(sq.x + sq.y);
+      if (valid && vec == 0) p.sc2_part[r * G + g] = sc2;
+    }
+    if (p.do_coeff) {  // stage the streams for the projection; sum v^2 of the row
+      float2 sv = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < N; ++i)
+#pragma unroll
+        for (int t = 0; t < 2; ++t) sv = __ffma2_rn(nf[i][t], nf[i][t], sv);
+      const float sv2 = sum16_lanes(sv.x + sv.y);
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) *reinterpret_cast<uint2*>(v_s + r * KS + i * kCols + vec * 4) = nb[i];
+        if (vec == 0) p.dot_part[(static_cast<size_t>(r) * G + g) * RED + C] = sv2;
+      }
+    }
+    cur = nxt;
+  }
+  if (!p.do_coeff) return;
+
+  // ---- 5. projection of this block's n*64 stream values per row onto the C fn
+  // columns on the tensor cores: [rows x n*64] bf16 x [n*64 x C] as three bf16
+  // terms, fp32 accumulation (mma.sync m16n8k16).
+  if (packed) {  // the packed slice, copied before the wait, has surely landed by now
+    const bool ok = mbar_wait_bounded(bar, 0, deadline);
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (__syncthreads_or(!ok)) return;  // also the barrier for the staged streams
+  } else {
+    __syncthreads();  // staged streams
+  }
+  // PAIRED (four row tiles or more): items are pairs of row tiles, so each B
+  // fragment serves both tiles and the operand reads from shared memory, which
+  // bound the projection with one tile per item, fall by ~30% (19.5 against
+  // 20.2 us per boundary at 128 rows, 10.74 against 10.90 at 64). The single-tile
+  // instantiation keeps the smaller kernel that fewer rows run faster with
+  // (with both loops in one kernel: 7.82 against 7.76 us at 32 rows). Per
+  // element the same operations in the same order either way.
+  const int mtiles = (R + 15) >> 4;
+  int mt0 = 0;  // first tile of the single-tile loop
+  if constexpr (PAIRED) {
+    const int mpairs = mtiles >> 1;
+    mt0 = 2 * mpairs;  // an odd last tile goes to the single-tile loop
+    for (int item = warp; item < mpairs * NT; item += kW1) {
+      const int mp = item / NT, nt = item - mp * NT;
+      float acc[2][3][4];
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int sp = 0; sp < 3; ++sp)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[t][sp][q] = 0.f;
+      const __nv_bfloat16* arow = v_s + (mp * 32 + (lane & 15)) * KS + (lane >> 4) * 8;
+      const __nv_bfloat16* brow = bs_s + (nt * 8 + (lane & 7)) * KS + ((lane >> 3) & 1) * 8;
+#pragma unroll 2
+      for (int k0 = 0; k0 < KC; k0 += 16) {
+        unsigned a0[4], a1[4], b[3][2];
+        ldmatrix_x4(a0, arow + k0);
+        ldmatrix_x4(a1, arow + 16 * KS + k0);
+#pragma unroll
+        for (int sp = 0; sp < 3; ++sp) ldmatrix_x2(b[sp], brow + sp * CP8 * KS + k0);
+#pragma unroll
+        for (int sp = 0; sp < 3; ++sp) {
+          mma_bf16_16816(acc[0][sp], a0, b[sp]);
+          mma_bf16_16816(acc[1][sp], a1, b[sp]);
+        }
+      }
+      const int col = nt * 8 + 2 * (lane & 3);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = (2 * mp + t) * 16 + (lane >> 2) + 8 * h;
+          if (r < R && col < C) {
+            float* dst = p.dot_part + (static_cast<size_t>(r) * G + g) * RED + col;
+            dst[0] = (acc[t][0][2 * h] + acc[t][1][2 * h]) + acc[t][2][2 * h];
+            if (col + 1 < C) dst[1] = (acc[t][0][2 * h + 1] + acc[t][1][2 * h + 1]) + acc[t][2][2 * h + 1];
+          }
+        }
+      }
+    }
+  }
+  // Single-tile items: (16-row tile, 8-column tile) of the block's rows x C
+  // logits. A warp takes items w, w + 16, ...; for its item it runs every k-step, with
+  // one accumulator per bf16 term of fn (three independent MMA chains), adds
+  // the terms and stores its rows' dot products itself: no cross-warp sums.
+  for (int item = warp; item < (mtiles - mt0) * NT; item += kW1) {
+    const int mt = mt0 + item / NT, nt = item % NT;
+    float acc[3][4];
+#pragma unroll
+    for (int sp = 0; sp < 3; ++sp)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[sp][q] = 0.f;
+    const __nv_bfloat16* arow = v_s + (mt * 16 + (lane & 15)) * KS + (lane >> 4) * 8;
+    const __nv_bfloat16* brow = bs_s + (nt * 8 + (lane & 7)) * KS + ((lane >> 3) & 1) * 8;
+#pragma unroll 4
+    for (int k0 = 0; k0 < KC; k0 += 16) {
+      unsigned a[4], b[3][2];
+      ldmatrix_x4(a, arow + k0);
+#pragma unroll
+      for (int sp = 0; sp < 3; ++sp) ldmatrix_x2(b[sp], brow + sp * CP8 * KS + k0);
+#pragma unroll
+      for (int sp = 0; sp < 3; ++sp) mma_bf16_16816(acc[sp], a, b[sp]);
+    }
+    // C fragment: lane holds rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
+    const int col = nt * 8 + 2 * (lane & 3);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = mt * 16 + (lane >> 2) + 8 * h;
+      if (r < R && col < C) {
+        float* dst = p.dot_part + (static_cast<size_t>(r) * G + g) * RED + col;
+        dst[0] = (acc[0][2 * h] + acc[1][2 * h]) + acc[2][2 * h];
+        if (col + 1 < C) dst[1] = (acc[0][2 * h + 1] + acc[1][2 * h + 1]) + acc[2][2 * h + 1];
+      }
+    }
   }
 }
+
 // Sinkhorn normalisation of an n x n matrix in one thread's registers: `iters`
 // times, each row divided by (its sum + eps), then each column by (its sum +
 // eps). For n = 4 the matrix stays as it came, K, and the steps update scale
@@ -330,674 +751,292 @@ __device__ __forceinline__ void sinkhorn_iterate(float (&M)[N][N], int iters, fl
   }
 }
 
-
-// The coefficients of row r, by one warp, from the row's totals over the CTAs
-// (tot[c]: dot product with fn column c, tot[C]: sum v^2): the logits (lane c
-// computes logit c), pre / post by sigmoid, and the comb by one exponential per
-// lane and Sinkhorn in lane 0 ([boundary] Boundaries.sublayer:
-// mhc_pre_delayed_overlap(residual, fn, scale, base, rms_norm_eps, hc_eps,
-// hc_eps, hc_post_alpha, hc_sinkhorn_iters)).
+// Loads of one layer-input task of a lane (row r, 8 columns): the row's
+// per-block sums of c^2, its carried pre, the stream vectors and norm weights.
 template <int N>
-__device__ __forceinline__ void coefficient_row(const Params& p, int r, const float* tot, float scale_l, float base_l,
-                                                int lane) {
-  constexpr int C = logits_of(N);
-  constexpr int NN = N * N;
-  const float s = lane < C ? tot[lane] : 0.f;
-  const float inv = rsqrtf(__fdiv_rn(tot[C], static_cast<float>(N * p.H)) + p.rms_eps);
-  const float l = lane < C ? scale_l * inv * s + base_l : 0.f;
-  if (lane < N) {
-    p.pre_out[r * N + lane] = 1.f / (1.f + expf(-l)) + p.pre_eps;
-  } else if (lane < 2 * N) {
-    p.post_out[r * N + (lane - N)] = p.alpha / (1.f + expf(-l));
-  }
-  // M = exp(L - max L) with one exp per lane, then Sinkhorn in one thread
-  const float lk = __shfl_sync(kFull, l, (lane + 2 * N) & 31);  // lane k < n*n: comb logit k
-  const float mx = warp_max(lane < NN ? lk : -INFINITY);
-  const float ek = expf(lk - mx);
-  float lc[NN];
-#pragma unroll
-  for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, ek, k);
-  if (lane == 0) {
-    float M[N][N];
-#pragma unroll
-    for (int j = 0; j < N; ++j)
-#pragma unroll
-      for (int i = 0; i < N; ++i) M[j][i] = lc[j * N + i];
-    sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
-#pragma unroll
-    for (int j = 0; j < N; ++j)
-#pragma unroll
-      for (int i = 0; i < N; ++i) p.comb_out[r * NN + j * N + i] = M[j][i];
-  }
-}
+struct LayerLoads {
+  static constexpr int MAXM = (kMaxBlocks + 31) / 32;
+  float sq[MAXM];
+  float pr[N];
+  uint4 sv[N];
+  uint4 nw;
+};
 
-// The projection of chunk c's 16 staged rows (K = n*64 stream values each) onto
-// the C fn columns on the tensor cores, by the 8 warps of the chunk's group:
-// warp wq runs K steps wq, wq + 8, ... (16 values each: stream k / 4, offset
-// 16 * (k % 4)), one accumulator per bf16 term of fn; the terms are added
-// (hi + mid) + lo and the warp's 16 x C partial sums go to part[wq].
 template <int N>
-__device__ __forceinline__ void project_chunk(const unsigned char* f_s, const unsigned char* v_s, int r_alloc, int c,
-                                              int wq, int lane, float* part) {
-  constexpr int C = logits_of(N);
-  constexpr int AR = arows_of(N);
-  constexpr int NT = (C + 7) / 8;  // 8-column tiles
-  float acc[3][NT][4];
+__device__ __forceinline__ void layer_load(const Params& p, int r, int g, int lane, bool weights,
+                                           LayerLoads<N>& Q) {
+  const int G = p.H / kCols;
 #pragma unroll
-  for (int t = 0; t < 3; ++t)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[t][nt][q] = 0.f;
-  for (int k = wq; k < 4 * N; k += kGroupWarps) {
-    const int j = k >> 2, kc0 = (k & 3) * 2;  // two 16-byte chunks of a 128-byte row
-    const int row = c * kRC + (lane & 15), kca = kc0 + (lane >> 4);
-    unsigned a[4];
-    ldmatrix_x4(a, v_s + j * r_alloc * 128 + row * 128 + (((kca ^ row) & 7) << 4));
-    const int kcb = kc0 + ((lane >> 3) & 1);
-#pragma unroll
-    for (int t = 0; t < 3; ++t) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int m = t * C + nt * 8 + (lane & 7);  // columns past C read other rows: ignored below
-        unsigned b[2];
-        ldmatrix_x2(b, f_s + j * AR * 128 + m * 128 + (((kcb ^ m) & 7) << 4));
-        mma_bf16_16816(acc[t][nt], a, b);
-      }
-    }
+  for (int m = 0; m < LayerLoads<N>::MAXM; ++m) {
+    const int k = lane + 32 * m;
+    Q.sq[m] = k < G ? __ldcg(p.sc2_part + r * G + k) : 0.f;
   }
-  // C fragment: lane holds rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
-  float* dst = part + wq * kRC * C;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int rr = (lane >> 2) + 8 * h;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = nt * 8 + 2 * (lane & 3) + e;
-        if (col < C) dst[rr * C + col] = (acc[0][nt][2 * h + e] + acc[1][nt][2 * h + e]) + acc[2][nt][2 * h + e];
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ float sum16_lanes(float v) {  // over the 16 lanes sharing lane bit 4
-#pragma unroll
-  for (int m = 8; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
-  return v;
-}
-
-__device__ __forceinline__ void named_sync_group(int q) {  // barrier ids are immediates: 1 and 2
-  if (q == 0) {
-    asm volatile("bar.sync 1, %0;" ::"n"(kGroupWarps * 32) : "memory");
+  if (g >= G) return;
+  const int h0 = g * kCols + (lane & 7) * 8;
+  if (weights) Q.nw = ld_nc_v4(p.norm_weight + h0);
+  if (p.tail_broadcast) {
+    Q.sv[0] = ld_v4(p.tail_streams + static_cast<size_t>(r) * p.H + h0);
   } else {
-    asm volatile("bar.sync 2, %0;" ::"n"(kGroupWarps * 32) : "memory");
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      Q.pr[j] = p.pre[r * N + j];
+      Q.sv[j] = ld_v4(p.tail_streams + (static_cast<size_t>(r) * N + j) * p.H + h0);
+    }
   }
 }
 
-// The boundary, one launch. See the top of this file for the steps; the
-// numbered comments below follow them.
-template <int N, int FRONT>
-__global__ void __launch_bounds__(kThreads, 1)
-    boundary_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
-                    const __grid_constant__ CUtensorMap tm_res, const __grid_constant__ CUtensorMap tm_gather) {
+// The tail of a boundary, launched after the streaming kernel (programmatic
+// dependent launch). Layer-input blocks split the rows into tasks of 256
+// columns (4 units of 64), one task per warp at a time: a lane normalises 8
+// columns of the row into the layer input (and MXFP8), recomputing the
+// collapse from the bf16 streams, after summing the row's per-block c^2 itself.
+// Coefficient blocks finish rows j, j + Gc, ... (logits, sigmoid, Sinkhorn).
+template <int N>
+__global__ void __launch_bounds__(kThreads, 2) boundary_tail_kernel(const Params p) {
   constexpr int C = logits_of(N);
-  constexpr int MIX = 2 * N + N * N;
-  constexpr int AR = arows_of(N);
-  constexpr int NFP = fields_of(N);  // record fields: C dot products, sum v^2, sum c^2 (even)
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  constexpr int RED = red_of(N);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const TailLayout L = tail_layout<N>();
+  float* slot_s = reinterpret_cast<float*>(smem + L.part_off);  // [kWarps rows][kWarps][RED]
+  float* scale_s = reinterpret_cast<float*>(smem + L.cst_off);
+  float* base_s = scale_s + 4;
 
-  const int R = p.R, H = p.H;
-  const int G = gridDim.x;
-  const bool coeff = p.do_coeff != 0, layer = p.do_layer != 0, exch = coeff || layer;
-  const int S = p.stages;
-  const bool packed = p.fn_packed != nullptr;
-  const Layout L = layout_of<N>(FRONT, R, G, p.P, p.topk, coeff, layer, S, packed);
-  unsigned char* a_s = smem + L.a_off;
-  unsigned char* v_s = smem + L.v_off;
-  unsigned char* st_s = smem + L.st_off;
-  unsigned char* fst_s = smem + L.fst_off;  // the fp32 fn slice as copied
-  float* mix_s = reinterpret_cast<float*>(smem + L.mix_off);
-  int* e2p_s = reinterpret_cast<int*>(smem + L.moe_off);
-  float* ew_s = reinterpret_cast<float*>(smem + L.moe_off) + R * p.topk;
-  float* rec_s = reinterpret_cast<float*>(smem + L.rec_off);  // [R][kRecF] this CTA's row records
-  float* inv_s = reinterpret_cast<float*>(smem + L.inv_off);  // [R] inverse RMS of the collapse
-  float* cft_s = reinterpret_cast<float*>(smem + L.cft_off);  // [slot][kRecF] this CTA's coefficient rows' totals
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* vready = full + kMaxStages;
-  uint64_t* fnbar = vready + kMaxChunks;
-  uint32_t* tag_slot = reinterpret_cast<uint32_t*>(fnbar + 1);
-
-  const int g = blockIdx.x;
+  const int G = p.H / kCols;
+  const int H = p.H;
+  const int R = p.R;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nch = (R + kRC - 1) / kRC;
-  const long long deadline = wait_deadline(p.budget_ns);
-  unsigned* status = p.ctl ? p.ctl + kStatusWord : nullptr;  // null: a residual-only call without a workspace
-  // the streaming lanes: group q of 8 warps takes chunks q, q + 2, ...; in a
-  // chunk, row rl = 2 * (warp % 8) + lane / 16 and columns h0 .. h0 + 3
-  const int q = warp / kGroupWarps, wq = warp % kGroupWarps;
-  const int rl = wq * 2 + (lane >> 4);
-  const int v = lane & 15;
-  const int h0 = g * kCols + v * 4;
+  const int rq = lane >> 3, vec = lane & 7;
 
-  // ---- 1. set-up before the wait (no kernel of this library writes weights,
-  // and kernels that do not trigger dependent launches are waited for in full
-  // before this one starts): the fn slice's copy goes out first
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
-    for (int c = 0; c < nch; ++c) mbar_init(&vready[c], kGroupWarps);
-    mbar_init(fnbar, 1);
-    if (coeff) {
-      if (packed) {
-        mbar_arrive_expect_tx(fnbar, aimage_bytes(N) + 16 * p.extra_tx);
-        bulk_g2s(a_s, p.fn_packed + static_cast<size_t>(g) * aimage_bytes(N), aimage_bytes(N), fnbar);
-      } else {
-        constexpr int JB = kCols * C * 4;  // one stream's 64 rows of fn: contiguous
-        mbar_arrive_expect_tx(fnbar, N * JB + 16 * p.extra_tx);
-#pragma unroll
-        for (int j = 0; j < N; ++j)
-          bulk_g2s(fst_s + j * JB, p.fn + (static_cast<size_t>(j) * H + g * kCols) * C, JB, fnbar);
-      }
+  // block roles: coefficient blocks first or last in the grid (the first blocks
+  // are placed first, on the SMs the streaming kernel leaves free)
+  const int bid = blockIdx.x;
+  const int lbid = p.tail_coeff_first ? bid - p.tail_coeff_blocks : bid;
+  if (lbid >= 0 && lbid < p.tail_layer_blocks) {
+    const int GT = (G + 3) >> 2;  // tasks per row
+    const int T = R * GT;
+    const int W = p.tail_layer_blocks * kWarps;
+    const int w0 = lbid * kWarps + warp;
+    LayerLoads<N> cur;
+    if (w0 < T) {  // norm weights of the first task: weights, so before the wait
+      const int g = (w0 % GT) * 4 + rq;
+      if (g < G) cur.nw = ld_nc_v4(p.norm_weight + g * kCols + vec * 8);
+      // lines the first task reads after the wait: L2 and address translation warm
+      const int r = w0 / GT;
+      if (lane == 0) prefetch_l2(p.sc2_part + r * G);
+      if (lane == 1 && !p.tail_broadcast) prefetch_l2(p.pre + r * N);
+      if (lane == 2) prefetch_l2(p.tail_streams + static_cast<size_t>(r) * (p.tail_broadcast ? 1 : N) * H);
     }
-    if (FRONT == kPartials || FRONT == kBroadcast || FRONT == kMoe) prefetch_tensormap(&tm_x);
-    if (FRONT != kBroadcast) prefetch_tensormap(&tm_res);
-    if (FRONT == kMoe && p.num_perm > 0) prefetch_tensormap(&tm_gather);
-  }
-  uint2 nw = make_uint2(0, 0);  // this lane's 4 norm weights
-  if (layer && warp < kWorkWarps) nw = ld_nc_v2(p.norm_weight + h0);
-  float scale_l = 0.f, base_l = 0.f;  // the control warp's lane c: scale of c's group, base[c]
-  if (coeff && warp == kCtl && lane < C) {
-    scale_l = p.scale[lane < N ? 0 : (lane < 2 * N ? 1 : 2)];
-    base_l = p.base[lane];
-  }
-  __syncthreads();
-
-  // ---- 2. wait for the preceding kernel on the stream, then the row data
-  griddep_wait();
-  if (tid == 0 && exch) {
-    const uint32_t e = ld_relaxed_gpu(p.ctl + kEpochWord);
-    *tag_slot = e + 1u == 0u ? 1u : e + 1u;
-  }
-  auto issue_chunk = [&](int c) {  // one thread; MoE gathers are issued by the whole warp below
-    const int s = c % S;
-    unsigned char* dst = st_s + s * L.stage_bytes;
-    mbar_arrive_expect_tx(&full[s], L.stage_bytes);
-    if constexpr (FRONT == kPartials) {
-      tma_load_3d(dst, &tm_x, g * kCols, c * kRC, 0, &full[s]);
-    } else if constexpr (FRONT == kBroadcast) {
-      tma_load_2d(dst, &tm_x, g * kCols, c * kRC, &full[s]);
-    }
-    if constexpr (FRONT != kBroadcast) tma_load_3d(dst + L.res_units * 128, &tm_res, g * kCols, 0, c * kRC, &full[s]);
-  };
-  auto issue_moe_chunk = [&](int c) {  // the control warp
-    const int s = c % S;
-    unsigned char* dst = st_s + s * L.stage_bytes;
-    const int K = p.topk;
-    if (lane == 0) {
-      const int gathered = p.num_perm > 0 ? K * kRC * 128 : 0;
-      mbar_arrive_expect_tx(&full[s], L.stage_bytes - (K * kRC * 128 - gathered));
-      tma_load_2d(dst + K * kRC * 128, &tm_x, g * kCols, c * kRC, &full[s]);  // shared output
-      tma_load_3d(dst + L.res_units * 128, &tm_res, g * kCols, 0, c * kRC, &full[s]);
-    }
-    __syncwarp();
-    if (p.num_perm > 0) {
-      for (int qq = lane; qq < K * 4; qq += 32) {  // slot t, rows 4*quad .. 4*quad + 3 of the chunk
-        const int t = qq >> 2, quad = qq & 3;
-        int idx[4];
+    griddep_wait();
+    griddep_launch_dependents();
+    if (w0 < T) layer_load<N>(p, w0 / GT, (w0 % GT) * 4 + rq, lane, false, cur);
+    const int scols = H / 32;
+    const int col_tiles = (scols + 3) / 4;
+    for (int t = w0; t < T; t += W) {
+      LayerLoads<N> nxt;
+      if (t + W < T) layer_load<N>(p, (t + W) / GT, ((t + W) % GT) * 4 + rq, lane, true, nxt);
+      const int r = t / GT;
+      const int g = (t - r * GT) * 4 + rq;
+      // ---- 7. the row's inverse RMS of the collapse: block sums in a fixed order
+      float a = cur.sq[0];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = c * kRC + quad * 4 + i;
-          const int e = r < R ? e2p_s[r * K + t] : 0;
-          idx[i] = (e >= 0 && e < p.num_perm) ? e : 0;  // such slots add nothing below
-        }
-        tma_gather4(dst + (t * kRC + quad * 4) * 128, &tm_gather, g * kCols, idx[0], idx[1], idx[2], idx[3], &full[s]);
-      }
-    }
-  };
-  if (FRONT != kMoe && tid == kCtl * 32) {
-    for (int c = 0; c < nch && c < S; ++c) issue_chunk(c);
-  }
-  for (int k = tid; k < R * MIX; k += kThreads) {  // [R][post n | comb n*n | pre n]
-    const int r = k / MIX, c = k - r * MIX;
-    if (c < N + N * N) {
-      if (FRONT == kStreams || FRONT == kBroadcast) {
-        mix_s[k] = 0.f;
-      } else if (c < N) {
-        cp_async4(mix_s + k, p.post + r * N + c);
-      } else {
-        cp_async4(mix_s + k, p.comb + r * N * N + (c - N));
-      }
-    } else if (p.pre != nullptr) {
-      cp_async4(mix_s + k, p.pre + r * N + (c - N - N * N));
-    } else {
-      mix_s[k] = 0.f;
-    }
-  }
-  if (FRONT == kMoe) {
-    for (int k = tid; k < R * p.topk; k += kThreads) {
-      cp_async4(e2p_s + k, p.e2p + k);
-      cp_async4(ew_s + k, p.ew + k);
-    }
-  }
-  // the fn slice's three bf16 terms, while the row data is in flight: one thread
-  // waits on the copy, the others block in the barrier (no issue slots)
-  bool fn_ok = true;
-  if (coeff) {
-    const bool ok = tid == 0 ? mbar_wait_bounded(fnbar, 0, deadline) : true;
-    fn_ok = __syncthreads_and(ok) != 0;
-    if (!fn_ok && tid == 0) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-    if (fn_ok && !packed) {
-      // consecutive threads take consecutive fn columns: conflict-free reads of the
-      // fp32 slice [kin][C]
-      for (int it = tid; it < N * C * 8; it += kThreads) {
-        const int c = it % C, rest = it / C;
-        const int oct = rest & 7, j = rest >> 3;
-        split_octet<N>(reinterpret_cast<const float*>(fst_s + j * kCols * C * 4), a_s + j * AR * 128, c, oct);
-      }
-    }
-  }
-  cp_async_wait_all();
-  __syncthreads();  // the mixes (and MoE routing) staged, the fn terms complete
-  const uint32_t tag = exch ? *tag_slot : 0u;
-  if (FRONT == kMoe && warp == kCtl) {
-    for (int c = 0; c < nch && c < S; ++c) issue_moe_chunk(c);
-  }
-
-  if (warp < kWorkWarps) {
-    // ---- 3. the chunks of group q: x, post-mix, new streams, staged streams, row sums
-    // with one stage, group 0 takes every chunk in order (two groups on one stage
-    // could each see the other's phase of its barrier as their own)
-    const int c0 = S > 1 ? q : (q == 0 ? 0 : nch), cstep = S > 1 ? 2 : 1;
-    for (int c = c0; c < nch; c += cstep) {
-      const int s = c % S;
-      // one lane of the group waits for the chunk's data; the group blocks in its barrier
-      if (wq == 0 && lane == 0 && !mbar_wait_bounded(&full[s], (c / S) & 1, deadline))
-        record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-      named_sync_group(q);
-      const int r = c * kRC + rl;
-      const bool valid = r < R;
-      const unsigned char* sp = st_s + s * L.stage_bytes;
-      const float* mix = mix_s + (valid ? r : 0) * MIX;
-      float2 nf[N][2];  // the new streams, as rounded to bf16
-      uint2 nb[N];
-      float2 xs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      if constexpr (FRONT == kPartials || FRONT == kMoe || lane_partials(FRONT)) {
-        if constexpr (FRONT == kPartials) {
-          for (int u = 0; u < p.P; ++u) {  // the partials in order
-            float2 f[2];
-            unpack4x2(lds_v2(sp + (u * kRC + rl) * 128 + v * 8), f);
-#pragma unroll
-            for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
-          }
-        } else if constexpr (FRONT == kMoe) {
-          unpack4x2(lds_v2(sp + (p.topk * kRC + rl) * 128 + v * 8), xs);  // shared output first
-          if (valid) {
-            const int* idx = e2p_s + r * p.topk;
-            const float* wt = ew_s + r * p.topk;
-            for (int u = 0; u < p.topk; ++u) {  // then the top_k slots in order
-              const int e = idx[u];
-              if (e >= p.num_perm) {
-                if (v == 0) record_error(status, MHC_ERR_DEVICE_INDEX);
-              } else if (e >= 0) {
-                float2 f[2];
-                unpack4x2(lds_v2(sp + (u * kRC + rl) * 128 + v * 8), f);
-                const float2 w2 = make_float2(wt[u], wt[u]);
-#pragma unroll
-                for (int t = 0; t < 2; ++t) xs[t] = __ffma2_rn(w2, f[t], xs[t]);
-              }
-            }
-          }
-        } else {  // lane-read partials: a table of (peer) pointers, or mailbox slots
-          if (valid) {
-            const size_t off = static_cast<size_t>(r) * H + h0;
-            for (int u = 0; u < p.P; ++u) {
-              const __nv_bfloat16* src = p.pptr[u] + off;
-              uint2 w = ld_cg_v2(src);
-              if (FRONT == kMailbox) {
-                while (has_neg_zero(w)) {  // re-read until its producer has written every element
-                  if (clock64() > deadline) {
-                    record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-                    break;
-                  }
-                  w = ld_volatile_v2(src);
-                }
-              }
-              float2 f[2];
-              unpack4x2(w, f);
-#pragma unroll
-              for (int t = 0; t < 2; ++t) xs[t] = __fadd2_rn(xs[t], f[t]);
-            }
-            if (FRONT == kMailbox) {  // consumed: back to "not written" for the round after next
-              for (int u = 0; u < p.P; ++u)
-                st_v2(const_cast<__nv_bfloat16*>(p.pptr[u]) + off, make_uint2(kNegZero2, kNegZero2));
-            }
-          }
-        }
-        float2 rf[N][2];
-#pragma unroll
-        for (int j = 0; j < N; ++j) unpack4x2(lds_v2(sp + (L.res_units + rl * N + j) * 128 + v * 8), rf[j]);
-        // mHC post: new[i] = bf16(post[i] * x + sum_j comb[j][i] * res[j]), column
-        // pairs in packed f32x2 arithmetic (per element the same fp32 operations,
-        // in the same order, as one at a time)
-#pragma unroll
-        for (int i = 0; i < N; ++i) {
-          float2 a[2];
-          const float2 po = make_float2(mix[i], mix[i]);
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            float2 s2 = __fmul2_rn(po, xs[t]);
-#pragma unroll
-            for (int j = 0; j < N; ++j) {
-              const float cj = mix[N + j * N + i];
-              s2 = __ffma2_rn(make_float2(cj, cj), rf[j][t], s2);
-            }
-            a[t] = s2;
-          }
-          nb[i] = make_uint2(pack_bf16x2(a[0].x, a[0].y), pack_bf16x2(a[1].x, a[1].y));
-          unpack4x2(nb[i], nf[i]);
-        }
-      } else if constexpr (FRONT == kStreams) {
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          nb[j] = lds_v2(sp + (rl * N + j) * 128 + v * 8);
-          unpack4x2(nb[j], nf[j]);
-        }
-      } else {  // kBroadcast: every stream is the embedding row
-        const uint2 xv = lds_v2(sp + rl * 128 + v * 8);
-        unpack4x2(xv, xs);
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          nb[j] = xv;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) nf[j][t] = xs[t];
-        }
-      }
-      if (p.write_res && valid) {
-#pragma unroll
-        for (int i = 0; i < N; ++i) st_v2(p.residual_out + (static_cast<size_t>(r) * N + i) * H + h0, nb[i]);
-      }
-      if (p.aux_out != nullptr && valid) {  // mean over the streams, in stream order, rounded once
-        constexpr float kInvN = 1.f / N;    // exact: n is a power of two
-        unsigned aw[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          float2 m = nf[0][t];
-#pragma unroll
-          for (int j = 1; j < N; ++j) m = __fadd2_rn(m, nf[j][t]);
-          m = __fmul2_rn(m, make_float2(kInvN, kInvN));
-          aw[t] = pack_bf16x2(m.x, m.y);
-        }
-        st_v2(p.aux_out + static_cast<size_t>(r) * H + h0, make_uint2(aw[0], aw[1]));
-      }
-      if (exch) {  // the new streams staged for the projection and the layer input
-#pragma unroll
-        for (int i = 0; i < N; ++i)
-          *reinterpret_cast<uint2*>(v_s + i * L.r_alloc * 128 + sw128_offset(r, v)) = nb[i];
-      }
-      if (layer) {  // collapse with the carried pre (identity pre-mix for the broadcast)
-        float2 sq = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          float2 cc;
-          if (FRONT == kBroadcast) {
-            cc = xs[t];
-          } else {
-            cc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int j = 0; j < N; ++j) {
-              const float pj = mix[N + N * N + j];
-              cc = __ffma2_rn(make_float2(pj, pj), nf[j][t], cc);
-            }
-          }
-          sq = __ffma2_rn(cc, cc, sq);
-        }
-        const float sc2 = sum16_lanes(sq.x + sq.y);
-        if (valid && v == 0) rec_s[r * kRecF + C + 1] = sc2;
-      }
-      if (coeff) {  // sum of v^2 of the row's streams, then the chunk's projection
-        float2 sv = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < N; ++i)
-#pragma unroll
-          for (int t = 0; t < 2; ++t) sv = __ffma2_rn(nf[i][t], nf[i][t], sv);
-        const float sv2 = sum16_lanes(sv.x + sv.y);
-        if (valid && v == 0) rec_s[r * kRecF + C] = sv2;
-        named_sync_group(q);  // the group's rows of the chunk staged; its stage read
-        float* part = L.part_off >= 0 ? reinterpret_cast<float*>(smem + L.part_off + q * part_bytes(N))
-                                      : reinterpret_cast<float*>(st_s + s * L.stage_bytes);
-        if (fn_ok) project_chunk<N>(a_s, v_s, L.r_alloc, c, wq, lane, part);
-        named_sync_group(q);
-        const int kw = 4 * N < kGroupWarps ? 4 * N : kGroupWarps;  // warps that ran K steps
-        for (int it = wq * 32 + lane; it < kRC * C; it += kGroupWarps * 32) {  // partials added in warp order
-          const int rr = it / C, col = it - rr * C;
-          if (c * kRC + rr < R) {
-            float a = 0.f;
-            for (int w = 0; w < kw; ++w) a += part[(w * kRC + rr) * C + col];
-            rec_s[(c * kRC + rr) * kRecF + col] = a;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&vready[c]);
-    }
-  } else {
-    // ---- 4. the control warp: a stage is refilled once its chunk is done
-    for (int c = 0; c + S < nch; ++c) {
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait_bounded(&vready[c], 0, deadline);
-      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-      if (!ok) {
-        if (lane == 0) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-        break;  // the chunks not refilled run out of their own waits
-      }
-      if constexpr (FRONT == kMoe) {
-        issue_moe_chunk(c + S);
-      } else {
-        if (lane == 0) issue_chunk(c + S);
-      }
-      __syncwarp();
-    }
-  }
-
-  if (exch) {
-    // ---- 5. publish this CTA's row records as tagged words at rec[g][r][f]: one
-    // contiguous run per CTA
-    __syncthreads();  // every row's records complete
-    for (int it = tid; it < R * NFP; it += kThreads) {
-      const int r = it / NFP, f = it - r * NFP;
-      const bool has = f <= C ? coeff : (f == C + 1 && layer);
-      st_tagged(p.rec + static_cast<size_t>(g) * R * NFP + it, tag, has ? rec_s[r * kRecF + f] : 0.f);
-    }
-    griddep_launch_dependents();  // this boundary's HBM stream is done: the next may start its set-up
-
-    // ---- 6. CTA g adds up rows g, g + G, ...: their records from every CTA, read
-    // as 16-byte pairs of words (all of a record with the coefficients, else the
-    // pair holding sum c^2), each field summed over the CTAs by 8 lanes
-    const int nslot = g < R ? (R - 1 - g) / G + 1 : 0;
-    if (nslot > 0) {
-      constexpr int B = 8;
-      const int kc0 = coeff ? 0 : (C + 1) / 2, nk = coeff ? NFP / 2 : 1;
-      float* gb = reinterpret_cast<float*>(st_s);  // [slot][G][NFP] the records' values
-      const int total = nslot * G * nk;
-      auto chunk = [&](int i) -> const unsigned long long* {
-        const int slot = i / (G * nk), rem = i - slot * G * nk;
-        const int gg = rem / nk, k = kc0 + rem - gg * nk;
-        return p.rec + (static_cast<size_t>(gg) * R + g + slot * G) * NFP + 2 * k;
-      };
-      for (int i0 = tid; i0 < total; i0 += B * kThreads) {
-        ulonglong2 w[B];
-#pragma unroll
-        for (int b = 0; b < B; ++b)
-          if (i0 + b * kThreads < total) w[b] = ld_tagged2(chunk(i0 + b * kThreads));
-        while (true) {  // the stale pairs re-read together until they carry the tag (bounded)
-          bool all = true;
-#pragma unroll
-          for (int b = 0; b < B; ++b)
-            if (i0 + b * kThreads < total && (tag_of(w[b].x) != tag || tag_of(w[b].y) != tag)) all = false;
-          if (all) break;
-          if (clock64() > deadline) {
-            record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-            break;
-          }
-#pragma unroll
-          for (int b = 0; b < B; ++b)
-            if (i0 + b * kThreads < total && (tag_of(w[b].x) != tag || tag_of(w[b].y) != tag))
-              w[b] = ld_tagged2(chunk(i0 + b * kThreads));
-        }
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          const int i = i0 + b * kThreads;
-          if (i < total) {
-            const int slot = i / (G * nk), rem = i - slot * G * nk;
-            const int gg = rem / nk, k = kc0 + rem - gg * nk;
-            float* d = gb + (slot * G + gg) * NFP + 2 * k;
-            d[0] = value_of(w[b].x);
-            d[1] = value_of(w[b].y);
-          }
-        }
-      }
-      __syncthreads();
-      const int f0 = coeff ? 0 : C + 1, nf = (layer ? C + 2 : C + 1) - f0;
-      const int units = nslot * nf;
-      const int gs = (G + 7) / 8;
-      for (int u0 = 0; u0 < units; u0 += kThreads / 8) {
-        if (u0 + warp * 4 >= units) continue;  // (warp-uniform) no unit for this warp
-        const int u = u0 + tid / 8, pp = tid & 7;
-        // every lane of the warp takes part in the butterfly
-        const bool active = u < units;
-        const int uu = active ? u : 0;
-        const int slot = uu / nf, f = f0 + uu - slot * nf;
-        const float* col = gb + slot * G * NFP + f;
-        float sum = 0.f;
-        const int ge = (pp + 1) * gs < G ? (pp + 1) * gs : G;
-        if (active)
-          for (int gg = pp * gs; gg < ge; ++gg) sum += col[gg * NFP];  // lane pp: CTAs pp*gs .. in order
-#pragma unroll
-        for (int m = 1; m <= 4; m <<= 1) sum += __shfl_xor_sync(kFull, sum, m);
-        if (active && pp == 0) cft_s[slot * kRecF + f] = sum;
-      }
-      __syncthreads();
-      if (layer) {  // the rows' sums c^2, one copy for every CTA: tot[c][r]
-        for (int it = tid; it < nslot * G; it += kThreads) {
-          const int sl = it / G, c = it - sl * G;
-          st_tagged(p.tot + static_cast<size_t>(c) * R + g + sl * G, tag, cft_s[sl * kRecF + C + 1]);
-        }
-      }
-    }
-    if (warp == kCtl && coeff) {
-      for (int sl = 0; sl < nslot; ++sl)
-        coefficient_row<N>(p, g + sl * G, cft_s + sl * kRecF, scale_l, base_l, lane);
-    }
-    if (warp < kWorkWarps && layer) {
-      // every row's sum c^2, from this CTA's copy
-      for (int r = tid; r < R; r += kWorkThreads) {
-        const unsigned long long* src = p.tot + static_cast<size_t>(g) * R + r;
-        unsigned long long w = ld_tagged(src);
-        while (tag_of(w) != tag) {
-          if (clock64() > deadline) {
-            record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-            break;
-          }
-          w = ld_tagged(src);
-        }
-        inv_s[r] = rsqrtf(__fdiv_rn(value_of(w), static_cast<float>(H)) + p.norm_eps);
-      }
-      named_sync_workers();
-    }
-    if (warp < kWorkWarps && layer) {
-      // ---- 7. the layer input (and MXFP8) of this CTA's columns, rows 2 * warp +
-      // lane / 16 of each 32-row pass, the lane's 4 columns
-      const int scols = H / 32;
-      const int col_tiles = (scols + 3) / 4;
-      float2 wv[2];
-      unpack4x2(nw, wv);
-      for (int r0 = 0; r0 < R; r0 += 2 * kWorkWarps) {
-        // every lane takes part in the block shuffles; rows past R store nothing
-        const int r = r0 + warp * 2 + (lane >> 4);
-        const bool valid = r < R;
-        const int rr = valid ? r : 0;
-        const float* mix = mix_s + rr * MIX;
-        // the collapse recomputed from the staged bf16 streams exactly as its squares were summed
-        float2 cc[2];
-        if (FRONT == kBroadcast) {
-          unpack4x2(lds_v2(v_s + sw128_offset(rr, v)), cc);
+      for (int m = 1; m < LayerLoads<N>::MAXM; ++m) a += cur.sq[m];
+      a = warp_sum(a);
+      const float inv = rsqrtf(__fdiv_rn(a, static_cast<float>(H)) + p.norm_eps);
+      if (g < G) {  // the 8 lanes of a unit share g: whole MXFP8 groups
+        const int h0 = g * kCols + vec * 8;
+        // ---- 7b. layer input: the collapse recomputed from the bf16 streams exactly
+        // as the streaming kernel summed its squares
+        float c[8];
+        if (p.tail_broadcast) {
+          unpack8(cur.sv[0], c);
         } else {
-          cc[0] = cc[1] = make_float2(0.f, 0.f);
+          float nf[N][8];
 #pragma unroll
-          for (int j = 0; j < N; ++j) {
-            float2 f[2];
-            unpack4x2(lds_v2(v_s + j * L.r_alloc * 128 + sw128_offset(rr, v)), f);
-            const float pj = mix[N + N * N + j];
+          for (int j = 0; j < N; ++j) unpack8(cur.sv[j], nf[j]);
 #pragma unroll
-            for (int t = 0; t < 2; ++t) cc[t] = __ffma2_rn(make_float2(pj, pj), f[t], cc[t]);
+          for (int e = 0; e < 8; ++e) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < N; ++j) s = fmaf(cur.pr[j], nf[j][e], s);
+            c[e] = s;
           }
         }
-        const float inv = inv_s[rr];
-        const float y[4] = {cc[0].x * inv * wv[0].x, cc[0].y * inv * wv[0].y, cc[1].x * inv * wv[1].x,
-                            cc[1].y * inv * wv[1].y};
-        const uint2 yb = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
-        if (valid) st_v2(p.layer_input + static_cast<size_t>(r) * H + h0, yb);
+        float w[8], y[8], yr[8];
+        unpack8(cur.nw, w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = c[e] * inv * w[e];
+        const uint4 yb = round8(y, yr);
+        st_v4(p.layer_input + static_cast<size_t>(r) * H + h0, yb);
         if (p.q_data != nullptr) {
-          float2 yr[2];
-          unpack4x2(yb, yr);
-          const float ys[4] = {yr[0].x, yr[0].y, yr[1].x, yr[1].y};
           float amax = 0.f;
           bool finite = true;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            amax = fmaxf(amax, fabsf(ys[e]));
-            finite = finite && isfinite(ys[e]);
+          for (int e = 0; e < 8; ++e) {
+            amax = fmaxf(amax, fabsf(yr[e]));
+            finite = finite && isfinite(yr[e]);
           }
-          // the 8 lanes of a 32-column block: lanes sharing lane bits 3 and 4
-#pragma unroll
-          for (int m = 1; m <= 4; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
-          const unsigned fin = __ballot_sync(kFull, finite);
-          const bool grp_ok = ((fin >> (lane & 24)) & 0xffu) == 0xffu;
-          unsigned d;
+          // the 4 lanes of a 32-column block are vec 0-3 or 4-7 of the same unit
+          const unsigned grp_mask = 0xffu << (lane & 24);
+          amax = fmaxf(amax, __shfl_xor_sync(grp_mask, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(grp_mask, amax, 2));
+          const unsigned fin_mask = __ballot_sync(grp_mask, finite);
+          const unsigned grp = (fin_mask >> (lane & 28)) & 0xfu;
+          uint2 d;
           unsigned char sbyte;
-          if (grp_ok) {
+          if (grp == 0xfu) {
             const int e = e8m0_exponent(amax);
-            const float sc8 = exp2_neg(e);
-            d = static_cast<unsigned>(e4m3x2(ys[0] * sc8, ys[1] * sc8)) |
-                (static_cast<unsigned>(e4m3x2(ys[2] * sc8, ys[3] * sc8)) << 16);
+            const float sc = exp2_neg(e);
+            d.x = static_cast<unsigned>(e4m3x2(yr[0] * sc, yr[1] * sc)) |
+                  (static_cast<unsigned>(e4m3x2(yr[2] * sc, yr[3] * sc)) << 16);
+            d.y = static_cast<unsigned>(e4m3x2(yr[4] * sc, yr[5] * sc)) |
+                  (static_cast<unsigned>(e4m3x2(yr[6] * sc, yr[7] * sc)) << 16);
             sbyte = static_cast<unsigned char>(e + 127);
           } else {
-            d = 0x7f7f7f7fu;
+            d.x = d.y = 0x7f7f7f7fu;
             sbyte = 0xff;
           }
-          if (valid) *reinterpret_cast<unsigned*>(p.q_data + static_cast<size_t>(r) * H + h0) = d;
-          if (valid && (v & 7) == 0) {
-            const int sc32 = h0 / 32;
-            p.q_scale[p.q_swizzled ? swizzled_scale_offset(r, sc32, col_tiles) : r * scols + sc32] = sbyte;
+          *reinterpret_cast<uint2*>(p.q_data + static_cast<size_t>(r) * H + h0) = d;
+          if ((vec & 3) == 0) {
+            const int sc = h0 / 32;
+            const int off = p.q_swizzled ? swizzled_scale_offset(r, sc, col_tiles) : r * scols + sc;
+            p.q_scale[off] = sbyte;
           }
         }
       }
-      if (p.q_data != nullptr && p.q_swizzled) {
-        // the padding of the swizzled scale buffer, spread over every CTA: rows R..
-        // whole, then the padding columns of rows below R
-        const int rows_p = (R + 127) & ~127;
-        const int pad_cols = col_tiles * 4 - scols;
-        const int n_rows = (rows_p - R) * col_tiles * 4;
-        const int n_cols = R * pad_cols;
-        for (int k = g * kWorkThreads + tid; k < n_rows + n_cols; k += G * kWorkThreads) {
-          if (k < n_rows) {
-            const int r = R + k / (col_tiles * 4), u = k % (col_tiles * 4);
+      cur = nxt;
+    }
+    if (p.q_data != nullptr && p.q_swizzled) {
+      // zero the padding of the swizzled scale buffer: rows R.. whole (4-byte words
+      // of a tile row when the buffer is 4-byte aligned), then the padding columns
+      // of rows below R
+      const int rows_p = (R + 127) & ~127;
+      const int pad_cols = col_tiles * 4 - scols;
+      const bool words = (reinterpret_cast<uintptr_t>(p.q_scale) & 3) == 0;
+      const int per_row = words ? col_tiles : col_tiles * 4;
+      const int n_rows = (rows_p - R) * per_row;
+      const int n_cols = R * pad_cols;
+      for (int k = w0 * 32 + lane; k < n_rows + n_cols; k += W * 32) {
+        if (k < n_rows) {
+          const int r = R + k / per_row, u = k % per_row;
+          if (words)
+            *reinterpret_cast<uint32_t*>(p.q_scale + swizzled_scale_offset(r, u * 4, col_tiles)) = 0u;
+          else
             p.q_scale[swizzled_scale_offset(r, u, col_tiles)] = 0;
-          } else {
-            const int kk = k - n_rows;
-            const int r = kk / pad_cols, sc32 = scols + kk % pad_cols;
-            p.q_scale[swizzled_scale_offset(r, sc32, col_tiles)] = 0;
-          }
+        } else {
+          const int kk = k - n_rows;
+          const int r = kk / pad_cols, sc = scols + kk % pad_cols;
+          p.q_scale[swizzled_scale_offset(r, sc, col_tiles)] = 0;
         }
       }
     }
-    // CTA 0 has read row 0's records from every CTA, so every CTA of this launch
-    // has read the epoch: the next launch may use the next tag.
-    if (g == 0 && tid == 0) p.ctl[kEpochWord] = tag;
   } else {
+    // Coefficient rows jb, jb + CB, ...: in batches of up to kWarps rows, every
+    // warp adds a share of each row's per-block records (fixed order) into a
+    // slot, then warp s finishes row s of the batch: logits, sigmoid, Sinkhorn.
+    const int jb = p.tail_coeff_first ? bid : bid - p.tail_layer_blocks;
+    const int CB = p.tail_coeff_blocks;
+    if (tid < 3) cp_async4(scale_s + tid, p.scale + tid);  // weights: before the wait
+    if (tid >= 32 && tid < 32 + C) cp_async4(base_s + tid - 32, p.base + (tid - 32));
+    if (tid == 64) prefetch_l2(p.dot_part + static_cast<size_t>(jb) * G * RED);  // warm, as above
+    griddep_wait();
     griddep_launch_dependents();
+    constexpr int V4 = RED / 4;
+    constexpr int MAXK = (kMaxBlocks * V4 + kThreads - 1) / kThreads;
+    constexpr int NN = N * N;
+    const int F = G * V4;
+    const int rho = (R - jb + CB - 1) / CB;
+    cp_async_wait_all();
+    for (int k0 = 0; k0 < rho; k0 += kWarps) {
+      const int nk = rho - k0 < kWarps ? rho - k0 : kWarps;
+      float4 v[MAXK];
+      {
+        const float4* base = reinterpret_cast<const float4*>(p.dot_part + static_cast<size_t>(jb + k0 * CB) * G * RED);
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k) {
+          const int f = tid + k * kThreads;
+          v[k] = f < F ? __ldcg(base + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      for (int s = 0; s < nk; ++s) {
+        float4 nx[MAXK];
+        if (s + 1 < nk) {  // the next row's loads go out before this row is added up
+          const float4* base =
+              reinterpret_cast<const float4*>(p.dot_part + static_cast<size_t>(jb + (k0 + s + 1) * CB) * G * RED);
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int f = tid + k * kThreads;
+            nx[k] = f < F ? __ldcg(base + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float4 a = v[0];
+#pragma unroll
+        for (int k = 1; k < MAXK; ++k) {
+          a.x += v[k].x;
+          a.y += v[k].y;
+          a.z += v[k].z;
+          a.w += v[k].w;
+        }
+        // lanes sharing lane % V4 hold the same 4 record values: add them up
+#pragma unroll
+        for (int m = V4; m < 32; m <<= 1) {
+          a.x += __shfl_xor_sync(kFull, a.x, m);
+          a.y += __shfl_xor_sync(kFull, a.y, m);
+          a.z += __shfl_xor_sync(kFull, a.z, m);
+          a.w += __shfl_xor_sync(kFull, a.w, m);
+        }
+        if (lane < V4) reinterpret_cast<float4*>(slot_s + (s * kWarps + warp) * RED)[lane] = a;
+        if (s + 1 < nk) {
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) v[k] = nx[k];
+        }
+      }
+      __syncthreads();
+      // warp s < nk: the comb (Sinkhorn) of row s of the batch; the pre and post of
+      // row s go to warp s + nk where there is one, else warp s does them after
+      const int s_comb = warp < nk ? warp : -1;
+      const int s_pp = warp < nk ? (warp + nk < kWarps ? -1 : warp) : (warp - nk < nk ? warp - nk : -1);
+      if (s_comb >= 0 || s_pp >= 0) {
+        const int sl = s_comb >= 0 ? s_comb : s_pp;
+        const int r = jb + (k0 + sl) * CB;
+        float s = 0.f;  // lane c: record value c, the warps' shares added in order
+        if (lane < RED) {
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) s += slot_s[(sl * kWarps + w) * RED + lane];
+        }
+        const float inv = rsqrtf(__fdiv_rn(__shfl_sync(kFull, s, C), static_cast<float>(N * H)) + p.rms_eps);
+        const int grp = lane < N ? 0 : (lane < 2 * N ? 1 : 2);
+        const float l = lane < C ? scale_s[grp] * inv * s + base_s[lane] : 0.f;
+        if (s_comb >= 0) {
+          // M = exp(L - max L) with one exp per lane, then Sinkhorn in one thread
+          float lk = __shfl_sync(kFull, l, (lane + 2 * N) & 31);  // lane k < n*n: comb logit k
+          const float mx = warp_max(lane < NN ? lk : -INFINITY);
+          const float ek = expf(lk - mx);
+          float lc[NN];
+#pragma unroll
+          for (int k = 0; k < NN; ++k) lc[k] = __shfl_sync(kFull, ek, k);
+          if (lane == 0) {
+            float M[N][N];
+#pragma unroll
+            for (int j = 0; j < N; ++j)
+#pragma unroll
+              for (int i = 0; i < N; ++i) M[j][i] = lc[j * N + i];
+            sinkhorn_iterate<N>(M, p.iters, p.sk_eps);
+#pragma unroll
+            for (int j = 0; j < N; ++j)
+#pragma unroll
+              for (int i = 0; i < N; ++i) p.comb_out[r * NN + j * N + i] = M[j][i];
+          }
+        }
+        if (s_pp >= 0) {
+          if (lane < N) {
+            p.pre_out[r * N + lane] = 1.f / (1.f + expf(-l)) + p.pre_eps;
+          } else if (lane < 2 * N) {
+            p.post_out[r * N + (lane - N)] = p.alpha / (1.f + expf(-l));
+          }
+        }
+      }
+      __syncthreads();  // the slots are refilled by the next batch
+    }
   }
 }
 
@@ -1073,33 +1112,26 @@ __global__ void mailbox_init_kernel(unsigned char* mb, size_t units) {
     st_v4(mb + kMailboxHeader + i * 16, z);
 }
 
-
-// fn [n*H, C] fp32 -> per CTA g the A operand image of its projection, the
-// bytes the kernel would build in shared memory: [n atom columns][arows][128 B],
-// row t*C + c holding term t of fn column c over the 64 K values of stream j
-// (fn row j*H + 64g + kin), 16-byte chunks XOR-swizzled by row; rows >= 3C zero.
+// fn [n*H, C] fp32 -> per block g the B operand of its projection as three bf16
+// terms, [G][3][CP8][n*64 + 8]: entry (t, c, k) is term t of fn[(k/64)*H + 64g + k%64][c];
+// columns c >= C and the 8-entry gap after each column are zero.
 template <int N>
 __global__ void __launch_bounds__(256) pack_projection_kernel(const float* __restrict__ fn, int H,
-                                                              unsigned char* __restrict__ out) {
+                                                              __nv_bfloat16* __restrict__ out) {
   constexpr int C = logits_of(N);
-  constexpr int AR = arows_of(N);
+  constexpr int KS = kstride_of(N);
+  constexpr int CP8 = ntiles_of(N) * 8;
   const int g = blockIdx.x;
-  unsigned char* dst = out + static_cast<size_t>(g) * aimage_bytes(N);
-  for (int it = threadIdx.x; it < N * AR * 8; it += blockDim.x) {
-    const int oct = it & 7, jm = it >> 3;
-    const int m = jm % AR, j = jm / AR;
-    unsigned w[4] = {0u, 0u, 0u, 0u};
-    if (m < 3 * C) {
-      const int t = m / C, c = m - t * C;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float f = fn[(static_cast<size_t>(j) * H + g * kCols + oct * 8 + e) * C + c];
-        __nv_bfloat16 term[3];
-        split3(f, term[0], term[1], term[2]);
-        w[e >> 1] |= static_cast<unsigned>(__bfloat16_as_ushort(term[t])) << ((e & 1) * 16);
-      }
-    }
-    *reinterpret_cast<uint4*>(dst + j * AR * 128 + m * 128 + (((oct ^ m) & 7) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  __nv_bfloat16* dst = out + static_cast<size_t>(g) * (packed_slice_bytes(N) / 2);
+  for (int e = threadIdx.x; e < CP8 * KS; e += blockDim.x) {
+    const int c = e / KS, k = e - c * KS;
+    float f = 0.f;
+    if (c < C && k < N * kCols) f = fn[(static_cast<size_t>(k / kCols) * H + g * kCols + k % kCols) * C + c];
+    __nv_bfloat16 hi, mid, lo;
+    split3(f, hi, mid, lo);
+    dst[(0 * CP8 + c) * KS + k] = hi;
+    dst[(1 * CP8 + c) * KS + k] = mid;
+    dst[(2 * CP8 + c) * KS + k] = lo;
   }
 }
 
@@ -1172,11 +1204,10 @@ __global__ void scale_padding_kernel(uint8_t* scale, int R, int H) {
   }
 }
 
-
 }  // namespace mhc
 
 // =====================================================================================
-// Host side: argument checks, tensor maps, launch configuration, C ABI
+// Host side: argument checks, launch configuration, C ABI
 // =====================================================================================
 
 namespace {
@@ -1188,17 +1219,14 @@ int g_extra_tx = 0;
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Workspace bytes: the header, then [G][R][fields] and [R] tagged words.
-size_t ws_layout(int R, int H, int n) {
-  const size_t G = static_cast<size_t>(H / kCols);
-  return kWsHeader + static_cast<size_t>(fields_of(n) + 1) * G * static_cast<size_t>(R) * 8;
-}
-
-// The workspace's parts for a call of p.R rows over p.H columns.
-void set_workspace(Params& p, void* ws, int n) {
-  p.ctl = static_cast<unsigned*>(ws);
-  p.rec = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kWsHeader);
-  p.tot = p.rec + static_cast<size_t>(p.H / kCols) * p.R * fields_of(n);
+size_t ws_layout(int R, int H, int n, size_t* sc2_off, size_t* dot_off) {
+  const int G = H / kCols;
+  const size_t a = kWsHeader;
+  const size_t sc2 = (static_cast<size_t>(R) * G * 4 + 255) & ~static_cast<size_t>(255);
+  const size_t dot = static_cast<size_t>(R) * G * red_of(n) * 4;
+  if (sc2_off) *sc2_off = a;
+  if (dot_off) *dot_off = a + sc2;
+  return a + sc2 + dot;
 }
 
 bool shape_ok(int R, int H, int n) {
@@ -1222,185 +1250,33 @@ mhc_status check_mxfp8(const mhc_mxfp8_out* q) {
   return MHC_OK;
 }
 
-// ---------------------------------------------------------------- tensor maps
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-    else
-      (void)cudaGetLastError();
-  });
-  return fn;
-}
-
-// A bf16 tensor map of `rank` dimensions (innermost first), strides in bytes of
-// dimensions 1.., box sizes; no swizzle, out-of-range elements read as zero.
-bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-              const uint32_t* box) {
-  EncodeTiledFn enc = encode_tiled();
-  if (enc == nullptr) return false;
-  cuuint64_t d[3], s[2];
-  cuuint32_t b[3], e[3] = {1, 1, 1};
-  for (int i = 0; i < rank; ++i) {
-    d[i] = dims[i];
-    b[i] = box[i];
-  }
-  for (int i = 0; i + 1 < rank; ++i) s[i] = strides[i];
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, s, b, e,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// What the host needs beyond Params to build a launch's tensor maps.
-struct Sources {
-  const __nv_bfloat16* partials = nullptr;  // kPartials: [P] x [R, H] with a stride
-  int64_t partial_stride = 0;
-  const __nv_bfloat16* residual = nullptr;  // [R, n, H]
-  const __nv_bfloat16* rows2d = nullptr;    // kBroadcast: x [R, H]; kMoe: shared_output [R, H]
-};
-
-// ---------------------------------------------------------------- launch
-
-constexpr int kSmemMax = 227 * 1024;  // the largest dynamic shared memory a block may have
-
-std::mutex g_cfg_mu;
-// (kernel, device, grid, smem bytes) -> whether every CTA of the grid can be resident
-std::map<std::tuple<const void*, int, int, int>, bool> g_fit;
-
-// The kernel's shared-memory limit and carveout, set once per kernel and device.
-std::map<std::pair<const void*, int>, bool> g_configured;
-
+// Launch with programmatic stream serialization: the kernel may start while the
+// preceding kernel on the stream finishes, and waits for it (griddepcontrol.wait)
+// before reading anything that kernel may have written.
+// A carveout >= 0 sets this launch's preferred shared-memory share (percent).
 template <typename Kern>
-bool configure(Kern kern, int dev) {
-  const auto key = std::make_pair(reinterpret_cast<const void*>(kern), dev);
-  std::lock_guard<std::mutex> lock(g_cfg_mu);
-  if (g_configured.count(key)) return true;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess ||
-      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           static_cast<int>(cudaSharedmemCarveoutMaxShared)) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return false;
-  }
-  g_configured[key] = true;
-  return true;
-}
-
-// Whether all `grid` CTAs can be resident at once (every CTA waits, bounded, for
-// the others' published records).
-template <typename Kern>
-bool blocks_fit(Kern kern, int dev, int grid, int smem) {
-  const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), dev, grid, smem);
-  {
-    std::lock_guard<std::mutex> lock(g_cfg_mu);
-    auto it = g_fit.find(key);
-    if (it != g_fit.end()) return it->second;
-  }
-  int per_sm = 0, sms = 0;
-  const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) == cudaSuccess &&
-                  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-                  per_sm * sms >= grid;
-  (void)cudaGetLastError();
-  std::lock_guard<std::mutex> lock(g_cfg_mu);
-  g_fit[key] = ok;
-  return ok;
-}
-
-template <int N, int FRONT>
-mhc_status launch_boundary(Params& p, const Sources& src, cudaStream_t stream) {
-  const int G = p.H / kCols;
-  const int R = p.R;
-  const bool coeff = p.do_coeff != 0, layer = p.do_layer != 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MHC_ERR_CUDA;
-  auto kern = boundary_kernel<N, FRONT>;
-  if (!configure(kern, dev)) return MHC_ERR_CUDA;
-  p.extra_tx = g_extra_tx;
-  p.budget_ns = g_budget_ns;
-
-  // tensor maps of this call's buffers (the maps are kernel parameters, so a
-  // captured graph keeps them)
-  CUtensorMap maps[3];
-  std::memset(maps, 0, sizeof(maps));
-  const uint64_t H = static_cast<uint64_t>(p.H);
-  if (FRONT == kPartials) {
-    const uint64_t pstride = p.P > 1 ? static_cast<uint64_t>(src.partial_stride) * 2 : static_cast<uint64_t>(R) * H * 2;
-    const uint64_t dims[3] = {H, static_cast<uint64_t>(R), static_cast<uint64_t>(p.P)};
-    const uint64_t strides[2] = {H * 2, pstride};
-    const uint32_t box[3] = {kCols, kRC, static_cast<uint32_t>(p.P)};
-    if (!make_map(&maps[0], src.partials, 3, dims, strides, box)) return MHC_ERR_CUDA;
-  }
-  if (FRONT == kBroadcast || FRONT == kMoe) {
-    const uint64_t dims[2] = {H, static_cast<uint64_t>(R)};
-    const uint64_t strides[1] = {H * 2};
-    const uint32_t box[2] = {kCols, kRC};
-    if (!make_map(&maps[0], src.rows2d, 2, dims, strides, box)) return MHC_ERR_CUDA;
-  }
-  if (FRONT != kBroadcast) {
-    const uint64_t dims[3] = {H, static_cast<uint64_t>(N), static_cast<uint64_t>(R)};
-    const uint64_t strides[2] = {H * 2, H * 2 * N};
-    const uint32_t box[3] = {kCols, static_cast<uint32_t>(N), kRC};
-    if (!make_map(&maps[1], src.residual, 3, dims, strides, box)) return MHC_ERR_CUDA;
-  }
-  if (FRONT == kMoe && p.num_perm > 0) {
-    const uint64_t dims[2] = {H, static_cast<uint64_t>(p.num_perm)};
-    const uint64_t strides[1] = {H * 2};
-    const uint32_t box[2] = {kCols, 1};
-    if (!make_map(&maps[2], p.gemm2, 2, dims, strides, box)) return MHC_ERR_CUDA;
-  }
-
-  // stages in flight: as many as the chunks need and shared memory holds, with
-  // every CTA of the grid resident
-  const int nch = (R + kRC - 1) / kRC;
-  int smem = 0;
-  p.stages = 0;
-  for (int st = nch < kMaxStages ? nch : kMaxStages; st >= 1; --st) {
-    // a stage that is refilled serves one group only: an even count, or one stage
-    // and one group
-    if (st < nch && st % 2 == 1 && st != 1) continue;
-    const Layout L = layout_of<N>(FRONT, R, G, p.P, p.topk, coeff, layer, st, p.fn_packed != nullptr);
-    const int bytes = L.total + 1024;
-    if (bytes > kSmemMax || !blocks_fit(kern, dev, G, bytes)) continue;
-    smem = bytes;
-    p.stages = st;
-    break;
-  }
-  if (p.stages == 0) return MHC_ERR_UNSUPPORTED_SHAPE;
-
+mhc_status launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, const Params& p, int threads = kThreads,
+                      int carveout = -1) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(G);
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, p, maps[0], maps[1], maps[2]) != cudaSuccess) {
+  if (carveout >= 0) {
+    attr[1].id = cudaLaunchAttributePreferredSharedMemoryCarveout;
+    attr[1].val.sharedMemCarveout = static_cast<unsigned>(carveout);
+    cfg.numAttrs = 2;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return MHC_ERR_CUDA;
   }
   return MHC_OK;
-}
-
-template <int FRONT>
-mhc_status dispatch_n(Params& p, const Sources& src, int n, cudaStream_t s) {
-  switch (n) {
-    case 1: return launch_boundary<1, FRONT>(p, src, s);
-    case 2: return launch_boundary<2, FRONT>(p, src, s);
-    case 4: return launch_boundary<4, FRONT>(p, src, s);
-    default: return MHC_ERR_UNSUPPORTED_SHAPE;
-  }
 }
 
 // Number of SMs of the current device (cached per device; safe to call from
@@ -1417,8 +1293,81 @@ int sm_count() {
   return n;
 }
 
-// Checks and fills the layer input, MXFP8, coefficients and workspace shared by
-// the full-boundary entry points.
+// Raise a kernel's dynamic shared memory limit to 200 KB, once per device
+// (idempotent, so concurrent first calls only repeat the same setting).
+constexpr int kSmemLimit = 200 * 1024;
+
+// Placement of the tail's blocks. An SM changes its L1 / shared-memory split only
+// when it is empty, and the split the driver picks for the streaming kernel alone
+// (just above its shared memory) leaves no room for a tail block beside it. Up to
+// kCoexistRows rows the streaming kernel asks for the largest shared-memory split,
+// so tail blocks launch early on its SMs too, and from kCoeffFirstRows rows the
+// coefficient blocks take the first block indices, which land on the SMs the
+// streaming kernel leaves free. Measured on B200 (whole boundaries in CUDA graphs,
+// us per boundary): 7.84 against 8.26 at 32 rows, 6.84 against 7.05 at 16, 5.85
+// against 5.94 at 4; the largest split is slower from 48 rows on (10.23 against
+// 9.95 at 48, 11.6 against 10.9 at 64, 22.2 against 19.9 at 128), and at 2 rows
+// the coefficient blocks first are (6.20 against 6.07).
+constexpr int kCoexistRows = 32;
+constexpr int kCoeffFirstRows = 4;
+template <typename Kern>
+bool allow_smem(Kern kern, int bytes, std::atomic<int>* configured) {
+  int dev = 0;
+  if (bytes > kSmemLimit || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (configured[dev].load(std::memory_order_acquire) != 0) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  configured[dev].store(1, std::memory_order_release);
+  return true;
+}
+
+template <int N, int FRONT>
+mhc_status launch_boundary(Params& p, cudaStream_t stream) {
+  const SmemLayout L = smem_layout<N>(p.R, p.topk, FRONT == kMoe, p.fn_packed != nullptr);
+  static std::atomic<int> configured[2][64];
+  const bool paired = ((p.R + 15) >> 4) >= 4;
+  auto kern = paired ? boundary_kernel<N, FRONT, true> : boundary_kernel<N, FRONT, false>;
+  if (!allow_smem(kern, L.total, configured[paired ? 1 : 0])) return MHC_ERR_CUDA;
+  p.extra_tx = g_extra_tx;
+  p.budget_ns = g_budget_ns;
+  const int G = p.H / kCols;
+  const bool few_rows = p.R <= kCoexistRows;
+  mhc_status st = launch_pdl(kern, G, L.total, stream, p, kT1,
+                             few_rows ? static_cast<int>(cudaSharedmemCarveoutMaxShared) : -1);
+  if (st != MHC_OK || !(p.do_layer || p.do_coeff)) return st;
+  if (FRONT == kBroadcast) {
+    p.tail_streams = p.x;
+    p.tail_broadcast = 1;
+  } else {
+    p.tail_streams = FRONT == kStreams ? p.residual : p.residual_out;
+    p.tail_broadcast = 0;
+  }
+  // layer-input blocks: one 256-column task per warp, at most G blocks; coefficient
+  // blocks run beside them, on the SMs those leave
+  const int tasks = p.R * ((G + 3) / 4);
+  const int lb = (tasks + kWarps - 1) / kWarps;
+  p.tail_layer_blocks = p.do_layer ? (lb < G ? lb : G) : 0;
+  const int spare = sm_count() - p.tail_layer_blocks;
+  p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
+  p.tail_coeff_first = few_rows && p.R >= kCoeffFirstRows;
+  return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>().total,
+                    stream, p);
+}
+
+template <int FRONT>
+mhc_status dispatch_n(Params& p, int n, cudaStream_t s) {
+  switch (n) {
+    case 1: return launch_boundary<1, FRONT>(p, s);
+    case 2: return launch_boundary<2, FRONT>(p, s);
+    case 4: return launch_boundary<4, FRONT>(p, s);
+    default: return MHC_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
+// Checks and fills the tail (layer input, MXFP8, coefficients, workspace) shared by
+// the two full-boundary entry points.
 mhc_status fill_tail(Params& p, const float* pre, const mhc_bf16* norm_weight, float norm_eps,
                      const mhc_coeff_args* coeffs, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
                      float* post_out, float* comb_out, float* pre_out, int R, int H, int n, void* ws,
@@ -1437,7 +1386,9 @@ mhc_status fill_tail(Params& p, const float* pre, const mhc_bf16* norm_weight, f
   st = check_mxfp8(mxfp8);
   if (st != MHC_OK) return st;
   if (coeffs && (!post_out || !comb_out || !pre_out)) return MHC_ERR_INVALID_ARG;
-  if (!ws || !aligned(ws, 256) || ws_bytes < ws_layout(R, H, n)) return MHC_ERR_WORKSPACE;
+  size_t sc2_off, dot_off;
+  const size_t need = ws_layout(R, H, n, &sc2_off, &dot_off);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return MHC_ERR_WORKSPACE;
   p.pre = pre;
   p.norm_weight = reinterpret_cast<const __nv_bfloat16*>(norm_weight);
   p.norm_eps = norm_eps;
@@ -1451,7 +1402,7 @@ mhc_status fill_tail(Params& p, const float* pre, const mhc_bf16* norm_weight, f
   if (coeffs) {
     p.do_coeff = 1;
     p.fn = coeffs->fn;
-    p.fn_packed = static_cast<const unsigned char*>(coeffs->fn_packed);
+    p.fn_packed = static_cast<const __nv_bfloat16*>(coeffs->fn_packed);
     p.scale = coeffs->scale;
     p.base = coeffs->base;
     p.rms_eps = coeffs->rms_eps;
@@ -1463,7 +1414,9 @@ mhc_status fill_tail(Params& p, const float* pre, const mhc_bf16* norm_weight, f
     p.comb_out = comb_out;
     p.pre_out = pre_out;
   }
-  set_workspace(p, ws, n);
+  p.ctl = static_cast<unsigned*>(ws);
+  p.sc2_part = reinterpret_cast<float*>(static_cast<char*>(ws) + sc2_off);
+  p.dot_part = reinterpret_cast<float*>(static_cast<char*>(ws) + dot_off);
   return MHC_OK;
 }
 
@@ -1480,7 +1433,7 @@ extern "C" {
 
 size_t mhc_workspace_bytes(int rows, int hidden, int hc_mult) {
   if (!shape_ok(rows, hidden, hc_mult)) return 0;
-  return ws_layout(rows, hidden, hc_mult);
+  return ws_layout(rows, hidden, hc_mult, nullptr, nullptr);
 }
 
 size_t mhc_mxfp8_scale_bytes(int rows, int hidden, int swizzled_128x4) {
@@ -1500,20 +1453,20 @@ mhc_status mhc_workspace_init(void* workspace, size_t ws_bytes, mhc_stream strea
 
 namespace {
 
-// mhc_boundary_post_pre over a table of partial pointers (checked by the callers):
-// the lanes load the partials themselves (peer memory, or mailbox slots).
-mhc_status post_pre_table(const __nv_bfloat16* const* pptr, int num_partials, const mhc_bf16* residual,
-                          const float* post, const float* comb, const float* pre, const mhc_bf16* norm_weight,
-                          float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out, mhc_bf16* aux_out,
-                          mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out,
-                          float* pre_out, int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
-                          mhc_stream stream, bool mailbox) {
+// mhc_boundary_post_pre over a table of partial pointers (checked by the callers).
+mhc_status post_pre_impl(const __nv_bfloat16* const* pptr, int num_partials, bool remote, const mhc_bf16* residual,
+                         const float* post, const float* comb, const float* pre, const mhc_bf16* norm_weight,
+                         float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out, mhc_bf16* aux_out,
+                         mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8, float* post_out, float* comb_out,
+                         float* pre_out, int rows, int hidden, int hc_mult, void* workspace, size_t ws_bytes,
+                         mhc_stream stream, bool mailbox = false) {
   mhc_status st = check_mixes(residual, post, comb, residual_out);
   if (st != MHC_OK) return st;
   Params p{};
   for (int u = 0; u < num_partials; ++u) p.pptr[u] = pptr[u];
-  p.premote = 1;
+  p.premote = remote ? 1 : 0;
   p.P = num_partials;
+  p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
   p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
@@ -1529,9 +1482,7 @@ mhc_status post_pre_table(const __nv_bfloat16* const* pptr, int num_partials, co
     if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return MHC_ERR_WORKSPACE;
     p.ctl = static_cast<unsigned*>(workspace);
   }
-  Sources src;
-  src.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
-  return mailbox ? dispatch_n<kMailbox>(p, src, hc_mult, stream) : dispatch_n<kTable>(p, src, hc_mult, stream);
+  return mailbox ? dispatch_n<kMailbox>(p, hc_mult, stream) : dispatch_n<kPartials>(p, hc_mult, stream);
 }
 
 }  // namespace
@@ -1549,34 +1500,12 @@ mhc_status mhc_boundary_post_pre(const mhc_bf16* partials, int num_partials, int
   if (num_partials < 1 || num_partials > kMaxPartials) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!partials || !aligned(partials, 16) || partial_stride % 8 != 0) return MHC_ERR_INVALID_ARG;
   if (num_partials > 1 && partial_stride == 0) return MHC_ERR_INVALID_ARG;
-  if (num_partials > 1 && partial_stride < 0) {  // not a tensor map: the lanes load the partials
-    const __nv_bfloat16* pptr[kMaxPartials];
-    for (int u = 0; u < num_partials; ++u)
-      pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials) + static_cast<int64_t>(u) * partial_stride;
-    return post_pre_table(pptr, num_partials, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out,
-                          aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult, workspace,
-                          ws_bytes, stream, false);
-  }
-  mhc_status st = check_mixes(residual, post, comb, residual_out);
-  if (st != MHC_OK) return st;
-  Params p{};
-  p.P = num_partials;
-  p.post = post;
-  p.comb = comb;
-  p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
-  p.write_res = 1;
-  if (aux_out && !aligned(aux_out, 16)) return MHC_ERR_INVALID_ARG;
-  p.aux_out = reinterpret_cast<__nv_bfloat16*>(aux_out);
-  p.R = rows;
-  p.H = hidden;
-  st = fill_tail(p, pre, norm_weight, norm_eps, coeffs, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
-                 hidden, hc_mult, workspace, ws_bytes);
-  if (st != MHC_OK) return st;
-  Sources src;
-  src.partials = reinterpret_cast<const __nv_bfloat16*>(partials);
-  src.partial_stride = partial_stride;
-  src.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
-  return dispatch_n<kPartials>(p, src, hc_mult, stream);
+  const __nv_bfloat16* pptr[kMaxPartials];
+  for (int u = 0; u < num_partials; ++u)
+    pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials) + static_cast<int64_t>(u) * partial_stride;
+  return post_pre_impl(pptr, num_partials, false, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                       residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult,
+                       workspace, ws_bytes, stream);
 }
 
 mhc_status mhc_boundary_post_pre_ptrs(const mhc_bf16* const* partials, int num_partials, const mhc_bf16* residual,
@@ -1594,9 +1523,9 @@ mhc_status mhc_boundary_post_pre_ptrs(const mhc_bf16* const* partials, int num_p
     if (!partials[u] || !aligned(partials[u], 16)) return MHC_ERR_INVALID_ARG;
     pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials[u]);
   }
-  return post_pre_table(pptr, num_partials, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out,
-                        aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult, workspace,
-                        ws_bytes, stream, false);
+  return post_pre_impl(pptr, num_partials, true, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                       residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult,
+                       workspace, ws_bytes, stream);
 }
 
 size_t mhc_mailbox_bytes(int world, int max_rows, int hidden) {
@@ -1658,9 +1587,9 @@ mhc_status mhc_boundary_collect(void* mailbox, int world, int max_rows, uint32_t
   const __nv_bfloat16* pptr[kMaxPartials];
   for (int u = 0; u < world; ++u)
     pptr[u] = slots + (static_cast<size_t>(par) * world + u) * max_rows * static_cast<size_t>(hidden);
-  mhc_status st = post_pre_table(pptr, world, residual, post, comb, pre, norm_weight, norm_eps, coeffs, residual_out,
-                                 aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden, hc_mult,
-                                 workspace, ws_bytes, stream, true);
+  mhc_status st = post_pre_impl(pptr, world, true, residual, post, comb, pre, norm_weight, norm_eps, coeffs,
+                                residual_out, aux_out, layer_input, mxfp8, post_out, comb_out, pre_out, rows, hidden,
+                                hc_mult, workspace, ws_bytes, stream, true);
   if (st != MHC_OK) return st;
   // an ordinary launch: it runs once the boundary has read (and re-marked) every
   // slot of this round, and leaves the round unconsumed if the boundary recorded
@@ -1677,8 +1606,9 @@ mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_per
                                      const float* comb, const float* pre, const mhc_bf16* norm_weight,
                                      float norm_eps, const mhc_coeff_args* coeffs, mhc_bf16* residual_out,
                                      mhc_bf16* aux_out, mhc_bf16* layer_input, const mhc_mxfp8_out* mxfp8,
-                                     float* post_out, float* comb_out, float* pre_out, int rows, int hidden,
-                                     int hc_mult, void* workspace, size_t ws_bytes, mhc_stream stream) {
+                                     float* post_out,
+                                     float* comb_out, float* pre_out, int rows, int hidden, int hc_mult,
+                                     void* workspace, size_t ws_bytes, mhc_stream stream) {
   if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (top_k < 1 || top_k > kMaxTopK || num_permuted < 0) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!gemm2_permuted || !expert_weights || !expanded_idx_to_permuted_idx || !shared_output)
@@ -1694,6 +1624,8 @@ mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_per
   p.ew = expert_weights;
   p.e2p = expanded_idx_to_permuted_idx;
   p.topk = top_k;
+  p.shared_out = reinterpret_cast<const __nv_bfloat16*>(shared_output);
+  p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
   p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
@@ -1702,17 +1634,16 @@ mhc_status mhc_boundary_moe_finalize(const mhc_bf16* gemm2_permuted, int num_per
   p.aux_out = reinterpret_cast<__nv_bfloat16*>(aux_out);
   p.R = rows;
   p.H = hidden;
+  // the MoE routing of every row is staged in shared memory; the residual-only
+  // form still needs the workspace header for the status word
   st = fill_tail(p, pre, norm_weight, norm_eps, coeffs, layer_input, mxfp8, post_out, comb_out, pre_out, rows,
                  hidden, hc_mult, workspace, ws_bytes);
   if (st != MHC_OK) return st;
-  if (pre == nullptr) {  // the residual-only form records gather-index errors in the workspace header
+  if (pre == nullptr) {
     if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return MHC_ERR_WORKSPACE;
     p.ctl = static_cast<unsigned*>(workspace);
   }
-  Sources src;
-  src.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
-  src.rows2d = reinterpret_cast<const __nv_bfloat16*>(shared_output);
-  return dispatch_n<kMoe>(p, src, hc_mult, stream);
+  return dispatch_n<kMoe>(p, hc_mult, stream);
 }
 
 mhc_status mhc_boundary_residual_only(const mhc_bf16* partials, int num_partials, int64_t partial_stride,
@@ -1726,12 +1657,10 @@ mhc_status mhc_boundary_residual_only(const mhc_bf16* partials, int num_partials
   mhc_status st = check_mixes(residual, post, comb, residual_out);
   if (st != MHC_OK) return st;
   Params p{};
-  if (num_partials > 1 && partial_stride < 0) {  // not a tensor map: the lanes load the partials
-    for (int u = 0; u < num_partials; ++u)
-      p.pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials) + static_cast<int64_t>(u) * partial_stride;
-    p.premote = 1;
-  }
+  for (int u = 0; u < num_partials; ++u)
+    p.pptr[u] = reinterpret_cast<const __nv_bfloat16*>(partials) + static_cast<int64_t>(u) * partial_stride;
   p.P = num_partials;
+  p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.post = post;
   p.comb = comb;
   p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
@@ -1740,12 +1669,7 @@ mhc_status mhc_boundary_residual_only(const mhc_bf16* partials, int num_partials
   p.aux_out = reinterpret_cast<__nv_bfloat16*>(aux_out);
   p.R = rows;
   p.H = hidden;
-  Sources src;
-  src.partials = reinterpret_cast<const __nv_bfloat16*>(partials);
-  src.partial_stride = partial_stride;
-  src.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
-  if (p.premote) return dispatch_n<kTable>(p, src, hc_mult, stream);
-  return dispatch_n<kPartials>(p, src, hc_mult, stream);
+  return dispatch_n<kPartials>(p, hc_mult, stream);
 }
 
 mhc_status mhc_coeffs(const mhc_bf16* residual, const mhc_coeff_args* coeffs, const float* pre_mix,
@@ -1757,13 +1681,15 @@ mhc_status mhc_coeffs(const mhc_bf16* residual, const mhc_coeff_args* coeffs, co
   if (!coeffs || !post_out || !comb_out || !pre_out) return MHC_ERR_INVALID_ARG;
   mhc_status st = check_coeff(coeffs);
   if (st != MHC_OK) return st;
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < ws_layout(rows, hidden, hc_mult)) return MHC_ERR_WORKSPACE;
+  size_t sc2_off, dot_off;
+  const size_t need = ws_layout(rows, hidden, hc_mult, &sc2_off, &dot_off);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < need) return MHC_ERR_WORKSPACE;
   Params p{};
   p.R = rows;
   p.H = hidden;
   p.do_coeff = 1;
   p.fn = coeffs->fn;
-  p.fn_packed = static_cast<const unsigned char*>(coeffs->fn_packed);
+  p.fn_packed = static_cast<const __nv_bfloat16*>(coeffs->fn_packed);
   p.scale = coeffs->scale;
   p.base = coeffs->base;
   p.rms_eps = coeffs->rms_eps;
@@ -1774,7 +1700,9 @@ mhc_status mhc_coeffs(const mhc_bf16* residual, const mhc_coeff_args* coeffs, co
   p.post_out = post_out;
   p.comb_out = comb_out;
   p.pre_out = pre_out;
-  set_workspace(p, workspace, hc_mult);
+  p.ctl = static_cast<unsigned*>(workspace);
+  p.sc2_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + sc2_off);
+  p.dot_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + dot_off);
   if (layer_input) {
     if (!norm_weight || !aligned(norm_weight, 16) || !aligned(layer_input, 16) || !(norm_eps >= 0.f))
       return MHC_ERR_INVALID_ARG;
@@ -1783,20 +1711,19 @@ mhc_status mhc_coeffs(const mhc_bf16* residual, const mhc_coeff_args* coeffs, co
     p.norm_eps = norm_eps;
     p.layer_input = reinterpret_cast<__nv_bfloat16*>(layer_input);
   }
-  Sources src;
   if (x) {
     if (pre_mix || !aligned(x, 16)) return MHC_ERR_INVALID_ARG;
     if (residual_out && !aligned(residual_out, 16)) return MHC_ERR_INVALID_ARG;
+    p.x = reinterpret_cast<const __nv_bfloat16*>(x);
     p.residual_out = reinterpret_cast<__nv_bfloat16*>(residual_out);
     p.write_res = residual_out != nullptr;
-    src.rows2d = reinterpret_cast<const __nv_bfloat16*>(x);
-    return dispatch_n<kBroadcast>(p, src, hc_mult, stream);
+    return dispatch_n<kBroadcast>(p, hc_mult, stream);
   }
   if (residual_out || !aligned(residual, 16)) return MHC_ERR_INVALID_ARG;
   if (layer_input && (!pre_mix || !aligned(pre_mix, 4))) return MHC_ERR_INVALID_ARG;
+  p.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
   p.pre = pre_mix;
-  src.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
-  return dispatch_n<kStreams>(p, src, hc_mult, stream);
+  return dispatch_n<kStreams>(p, hc_mult, stream);
 }
 
 mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden, const mhc_mxfp8_out* out,
@@ -1837,7 +1764,7 @@ mhc_status mxfp8_quantize_rows(const mhc_bf16* x, int rows, int hidden, const mh
 size_t mhc_projection_pack_bytes(int hidden, int hc_mult) {
   if (!shape_ok(1, hidden, hc_mult)) return 0;
   const int G = hidden / kCols;
-  const int pb = hc_mult == 1 ? aimage_bytes(1) : (hc_mult == 2 ? aimage_bytes(2) : aimage_bytes(4));
+  const int pb = hc_mult == 1 ? packed_slice_bytes(1) : (hc_mult == 2 ? packed_slice_bytes(2) : packed_slice_bytes(4));
   return static_cast<size_t>(G) * pb;
 }
 
@@ -1845,7 +1772,7 @@ mhc_status mhc_projection_pack(const float* fn, void* packed, int hidden, int hc
   if (!shape_ok(1, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (!fn || !packed || !aligned(fn, 4) || !aligned(packed, 16)) return MHC_ERR_INVALID_ARG;
   const int G = hidden / kCols;
-  unsigned char* out = static_cast<unsigned char*>(packed);
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(packed);
   switch (hc_mult) {
     case 1: pack_projection_kernel<1><<<G, 256, 0, stream>>>(fn, hidden, out); break;
     case 2: pack_projection_kernel<2><<<G, 256, 0, stream>>>(fn, hidden, out); break;
@@ -1987,15 +1914,13 @@ namespace {
 constexpr int kNoAllocMaxRows = 128;
 constexpr int kNoAllocMaxHidden = 7168;
 constexpr int kNoAllocMaxHc = 4;
-// 3,097,600 bytes: mhc_workspace_bytes(128, 7168, 4), the header, the row
-// records [112 CTAs][128 rows][26 fields] and the totals [112 copies][128 rows]
-constexpr size_t kNoAllocBytes =
-    kWsHeader + static_cast<size_t>(fields_of(kNoAllocMaxHc) + 1) * (kNoAllocMaxHidden / kCols) * kNoAllocMaxRows * 8;
-static_assert(kNoAllocBytes == 3097600, "the no-alloc scratch size");
+// mhc_workspace_bytes(128, 7168, 4): header, c^2 sums [128][112] (rounded to
+// 256 bytes), projection sums [128][112][32] floats
+constexpr size_t kNoAllocBytes = kWsHeader + ((static_cast<size_t>(kNoAllocMaxRows) * (kNoAllocMaxHidden / kCols) * 4 + 255) & ~static_cast<size_t>(255)) +
+                                 static_cast<size_t>(kNoAllocMaxRows) * (kNoAllocMaxHidden / kCols) * red_of(kNoAllocMaxHc) * 4;
 
-// The array is zero at module load, as a workspace must be before first use
-// (mhc_workspace_init): the status word, and the launch epoch that tags the
-// row records every call rewrites.
+// The array is zero at module load. A kernel never needs its contents to start
+// at zero except the status word, which only a failed wait writes.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 // The calling thread's current CUDA context (the driver's cuCtxGetCurrent), or
@@ -2053,7 +1978,7 @@ mhc_status mhc_boundary_post_pre_noalloc(const mhc_bf16* partials, int num_parti
                                          int hc_mult, mhc_stream stream) {
   if (!shape_ok(rows, hidden, hc_mult)) return MHC_ERR_UNSUPPORTED_SHAPE;
   if (rows > kNoAllocMaxRows || hidden > kNoAllocMaxHidden || hc_mult > kNoAllocMaxHc ||
-      ws_layout(rows, hidden, hc_mult) > kNoAllocBytes)
+      ws_layout(rows, hidden, hc_mult, nullptr, nullptr) > kNoAllocBytes)
     return MHC_ERR_WORKSPACE;  // needs more scratch than the fixed array holds
   void* ws = noalloc_scratch();
   if (ws == nullptr) return MHC_ERR_CUDA;

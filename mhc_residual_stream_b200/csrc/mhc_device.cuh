@@ -1,7 +1,6 @@
 // Device helpers of the mHC boundary kernels (sm_100a): PTX wrappers for the
-// bulk-copy and tensor-map TMA engine, mbarriers, the warp-level tensor-core
-// MMA, thread-block clusters, tagged words between CTAs, bf16 packing, bounded
-// waits, and the E8M0/E4M3 encoders of the MXFP8 layer input.
+// bulk-copy engine and mbarriers, bf16 packing, bounded waits, and the
+// E8M0/E4M3 encoders of the MXFP8 layer input.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,7 +24,6 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
-// The first error of a launch wins; a null status (a call without a workspace) records nothing.
 __device__ __forceinline__ void record_error(unsigned* status, unsigned code) {
   if (status != nullptr) atomicCAS(status, 0u, code);
 }
@@ -57,23 +55,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       : "memory");
 }
 
-// Test phase `parity` of `bar`; while it is incomplete the thread is suspended
-// (up to the hint, 1 ms, and woken when the phase completes) rather than spinning,
-// so waiting warps take no issue slots from working ones.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   unsigned ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`, giving up at `deadline` (clock64 cycles; each
-// test may sleep up to 1 ms, so the wait ends by deadline + 1 ms).
+// Wait for phase `parity` of `bar`, giving up at `deadline` (clock64 cycles).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, long long deadline) {
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() > deadline) return false;
@@ -150,30 +144,6 @@ __device__ __forceinline__ unsigned clear_neg_zero2(unsigned w) { return w & __v
 __device__ __forceinline__ void st_v2(void* p, uint2 v) {
   asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
-__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {  // L2 only: data other agents write
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint4 ld_volatile_v4(const void* p) {  // re-read on every call
-  uint4 v;
-  asm volatile("ld.volatile.global.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ bool has_neg_zero4(const uint4 v) {
-  return (__vcmpeq2(v.x, kNegZero2) | __vcmpeq2(v.y, kNegZero2) | __vcmpeq2(v.z, kNegZero2) |
-          __vcmpeq2(v.w, kNegZero2)) != 0u;
-}
-// 8 bf16 as four column pairs: f[m] = (element 2m, element 2m + 1).
-__device__ __forceinline__ void unpack8x2(const uint4 v, float2 (&f)[4]) {
-  f[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
-  f[1] = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
-  f[2] = make_float2(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u));
-  f[3] = make_float2(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
-}
 // 4 bf16 as two column pairs: f[m] = (element 2m, element 2m + 1).
 __device__ __forceinline__ void unpack4x2(const uint2 v, float2 (&f)[2]) {
   f[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
@@ -191,51 +161,6 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
   asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
-
-// ---------------------------------------------------------------- tensor-map TMA loads (no multicast)
-
-// Tiled tensor-map loads into this CTA's shared memory; completion is counted in
-// bytes on `bar` (the full box, out-of-range elements filled with zeros).
-// `map` is the address of a __grid_constant__ kernel parameter.
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Four rows y0..y3 of a 2-D tensor map whose box is one row high, columns
-// [x, x + box width), landed as four consecutive box rows at dst.
-__device__ __forceinline__ void tma_gather4(void* dst, const void* map, int x, int y0, int y1, int y2, int y3,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Fetch a tensor map (a __grid_constant__ kernel parameter) ahead of its first use.
-__device__ __forceinline__ void prefetch_tensormap(const void* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Generic-proxy writes to shared memory made visible to the async proxy (the
-// tensor cores and the TMA engine) before they read them.
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------- warp-level tensor core MMA
 
@@ -262,70 +187,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const unsigned (&a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-
-// ---------------------------------------------------------------- thread-block clusters
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-// Address of the same shared-memory byte in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-// Bulk copy from this CTA's shared memory into CTA-of-the-cluster shared memory
-// (dst and bar are addresses from dsmem_addr); completion is counted in bytes on
-// the destination CTA's mbarrier. src, dst and bytes multiples of 16.
-__device__ __forceinline__ void bulk_s2dsmem(uint32_t dst, const void* src, unsigned bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "r"(smem_u32(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until every committed bulk copy of this thread has read its source.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Make this CTA's mbarrier initialisations visible to the cluster (before a
-// relaxed cluster arrive).
-__device__ __forceinline__ void fence_mbarrier_init_cluster() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// Arrive on the cluster barrier without ordering memory (the start-up barrier
-// that makes every CTA of the cluster resident before shared memory is shared).
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-
-// ---------------------------------------------------------------- tagged words between CTAs
-
-// A value and the tag of the launch that wrote it, as one 64-bit word: a
-// reader that sees the expected tag has the value written with it (a 64-bit
-// access is single-copy atomic), with no flag and no fence between them.
-__device__ __forceinline__ void st_tagged(unsigned long long* p, uint32_t tag, float v) {
-  const unsigned long long w = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
-  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
-  unsigned long long w;
-  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
-  return w;
-}
-// Two consecutive tagged words (16-byte aligned); each word is read as one
-// single-copy atomic access.
-__device__ __forceinline__ ulonglong2 ld_tagged2(const unsigned long long* p) {
-  ulonglong2 w;
-  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p) : "memory");
-  return w;
-}
-__device__ __forceinline__ uint32_t tag_of(unsigned long long w) { return static_cast<uint32_t>(w >> 32); }
-__device__ __forceinline__ float value_of(unsigned long long w) { return __uint_as_float(static_cast<uint32_t>(w)); }
 
 // ---------------------------------------------------------------- bf16 packing
 

@@ -480,32 +480,23 @@ def test_packed_projection_moe_and_coeffs_entry():
 
 @pytest.mark.parametrize("n", [1, 4])
 def test_packed_layout_holds_the_three_bf16_terms(n):
-    # block g's image is [n atom columns][arows][128 bytes]: row m = t*C + c holds
-    # term t of fn column c for K values kin = 0..63 of stream j, the 16-byte
-    # chunk kin // 8 stored at chunk (kin // 8) ^ (m % 8); the terms add back to fn
+    # element (t, c, k) of block g is term t of fn[(k/64)*H + 64g + k%64][c]; terms add back to fn
     H = 128
     C = 2 * n + n * n
-    AR = (3 * C + 7) // 8 * 8
     fn = torch.randn(n * H, C, dtype=torch.float32) * 0.02
     pk = M.mhc_projection_pack(fn.to(DEV), H, n)
     torch.cuda.synchronize()
-    raw = pk.cpu().view(torch.bfloat16).view(H // 64, n, AR, 8, 8).to(torch.float64)  # [g][j][m][chunk][8]
-    assert raw.numel() * 2 == M.mhc_projection_pack_bytes(H, n)
-
-    def term(g, t, c, k):
-        j, kin = divmod(k, 64)
-        m = t * C + c
-        return raw[g, j, m, (kin // 8) ^ (m % 8), kin % 8]
-
+    KS, CP8 = n * 64 + 8, ((C + 7) // 8) * 8
+    t = pk.cpu().view(torch.bfloat16).view(H // 64, 3, CP8, KS).to(torch.float64)
     for g in range(H // 64):
         for k in [k for k in (0, 5, 63, 64, 200, n * 64 - 1) if k < n * 64]:
             row = (k // 64) * H + 64 * g + k % 64
-            s = torch.tensor([term(g, 0, c, k) + term(g, 1, c, k) + term(g, 2, c, k) for c in range(C)])
+            s = t[g, 0, :C, k] + t[g, 1, :C, k] + t[g, 2, :C, k]
             assert torch.allclose(s, fn[row].double(), rtol=2 ** -22, atol=0), (g, k)
             hi = fn[row].to(torch.bfloat16).double()
-            assert torch.equal(torch.tensor([term(g, 0, c, k) for c in range(C)]).double(), hi), (g, k)
-    pad = raw[:, :, 3 * C:]  # rows past the three terms are zero
-    assert pad.numel() == 0 or float(pad.abs().max()) == 0.0
+            assert torch.equal(t[g, 0, :C, k], hi), (g, k)
+    for pad in (t[:, :, C:, :], t[:, :, :, n * 64:]):  # padding columns and gaps are zero
+        assert pad.numel() == 0 or float(pad.abs().max()) == 0.0
 
 
 # ---------------------------------------------------------------- bounded waits
