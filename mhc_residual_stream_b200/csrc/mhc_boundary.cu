@@ -5,9 +5,9 @@
 // The streaming kernel (boundary_kernel): block g owns columns [64g, 64g+64)
 // of H for every row, so each weight of fn is read from HBM exactly once.
 //   1. A TMA bulk copy brings the block's fn slice into shared memory (packed
-//      bf16 terms, or fp32 that the block splits into bf16 terms) and the
-//      block's activations are prefetched into L2, both before the kernel waits
-//      for its predecessor on the stream;
+//      bf16 terms, or fp32 that the block splits into bf16 terms while its row
+//      data are in flight) and the block's activations are prefetched into L2,
+//      both before the kernel waits for its predecessor on the stream;
 //   2. per (row, 4 columns) a lane sums the partials (local buffers, peers'
 //      buffers, or the slots of a publish/collect mailbox as they fill) or
 //      finalizes the MoE output, applies the mHC post-mix (vllm
@@ -49,6 +49,7 @@ constexpr int kMaxPartials = 16;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxIters = 1000;
 constexpr int kMaxBlocks = 148;  // most H/64 blocks: the tail's per-lane loads are sized for it
+constexpr int kPrefetchRows = 64;  // the streaming kernel prefetches its rows into L2 up to this many
 // Workspace header: the status word (byte 0); the partial sums follow.
 constexpr size_t kWsHeader = 1024;
 constexpr int kStatusWord = 0;
@@ -332,7 +333,10 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
   // ---- 2. bring this block's activations into L2 while the preceding kernel may
   // still run: a prefetch is only a hint and L2 is the point of coherence, so
   // it is safe before the wait; gather indices read now only steer prefetches.
-  if (vec == 0 || vec == 15) {
+  // Up to 64 rows: past that the prefetches cost more than they save (us per
+  // boundary with / without, B200: 7.65 / 8.23 at 32 rows, 9.81 / 10.20 at 48,
+  // 15.79 / 15.45 at 96, 19.52 / 18.17 at 128).
+  if ((vec == 0 || vec == 15) && R <= kPrefetchRows) {
     for (int q = warp; q < npairs; q += kW1) {
       const int r = q * 2 + rq;
       if (r >= R) break;
@@ -355,22 +359,6 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
     }
   }
 
-  if (p.do_coeff && !packed) {
-    // Split the fn slice into three bf16 terms (split3), stored column-major for
-    // the MMA's B operand (weights only: before the wait).
-    const bool ok = mbar_wait_bounded(bar, 0, deadline);
-    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-    if (__syncthreads_or(!ok)) return;  // every copy issued has landed or never will
-    for (int e = tid; e < CP8 * KC; e += kT1) {
-      const int c = e / KC, k = e - c * KC;
-      const float f = c < C ? reinterpret_cast<const float*>(fn_s + (k >> 3) * PIECE + (k & 7) * C * 4)[c] : 0.f;
-      __nv_bfloat16 hi, mid, lo;
-      split3(f, hi, mid, lo);
-      bs_s[(0 * CP8 + c) * KS + k] = hi;
-      bs_s[(1 * CP8 + c) * KS + k] = mid;
-      bs_s[(2 * CP8 + c) * KS + k] = lo;
-    }
-  }
   if (warp == 1 && lane < 3) {  // the mixes' first lines: L2 and address translation warm before the wait
     const float* mp = lane == 0 ? p.post : (lane == 1 ? p.comb : p.pre);
     if (mp != nullptr) prefetch_l2(mp);
@@ -400,6 +388,38 @@ __global__ void __maxnreg__(80) boundary_kernel(const Params p) {
     for (int k = tid; k < R * p.topk; k += kT1) {
       cp_async4(e2p_s + k, p.e2p + k);
       cp_async4(ew_s + k, p.ew + k);
+    }
+  }
+  if (p.do_coeff && !packed) {
+    // Split the fn slice into three bf16 terms (split3), stored column-major for
+    // the MMA's B operand, while the row data and the mixes are in flight: a
+    // thread takes 8 consecutive K values k = 8*oct .. 8*oct + 7 of column c (one
+    // landed piece), consecutive threads consecutive columns, and writes each
+    // term's 16 bytes at once.
+    const bool ok = mbar_wait_bounded(bar, 0, deadline);
+    if (!ok) record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+    if (__syncthreads_or(!ok)) {  // every copy issued has landed or never will
+      cp_async_wait_all();
+      return;
+    }
+    for (int e = tid; e < CP8 * (KC / 8); e += kT1) {
+      const int c = e % CP8, oct = e / CP8;
+      const float* src = reinterpret_cast<const float*>(fn_s + oct * PIECE) + c;  // k = 8*oct + i at src[i * C]
+      unsigned w[3][4];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const float f0 = c < C ? src[i * C] : 0.f, f1 = c < C ? src[(i + 1) * C] : 0.f;
+        __nv_bfloat16 t0[3], t1[3];
+        split3(f0, t0[0], t0[1], t0[2]);
+        split3(f1, t1[0], t1[1], t1[2]);
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          w[t][i / 2] = static_cast<unsigned>(__bfloat16_as_ushort(t0[t])) |
+                        (static_cast<unsigned>(__bfloat16_as_ushort(t1[t])) << 16);
+      }
+#pragma unroll
+      for (int t = 0; t < 3; ++t)
+        *reinterpret_cast<uint4*>(bs_s + (t * CP8 + c) * KS + oct * 8) = make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
     }
   }
   cp_async_wait_all();

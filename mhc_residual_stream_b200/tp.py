@@ -157,8 +157,11 @@ class PeerMailbox:
     Rounds are checked on the host before anything is launched ([all_reduce]
     mark_published / reset keep the same kind of state): this rank publishes
     rounds 0, 1, 2, ... in order, at most one round ahead of its collects, and
-    collects only a round it has published, in order. `reset` drops what an
-    aborted step left behind, on every rank of the group together."""
+    collects only a round it has published, in order, over as many rows as it
+    published in that round (slots past the rows a collect reads would keep
+    their values, and a later round of the same parity would take them for
+    fresh ones). `reset` drops what an aborted step left behind, on every rank
+    of the group together."""
 
     def __init__(self, max_rows: int, hidden: int, group: Optional[dist.ProcessGroup] = None, device=None,
                  heartbeat: Optional[Heartbeat] = None):
@@ -173,6 +176,7 @@ class PeerMailbox:
         self.ptrs, self._imported = partial_table(self.rank, self.local.data_ptr(), gathered, M.ipc_import)
         self.published = -1  # the last round this rank published
         self.collected = -1  # the last round this rank collected
+        self.rows = {}  # round -> rows this rank published in it (the rounds not yet collected)
 
     def publish(self, x: torch.Tensor, round_: int, stream=None):
         """This rank's contribution of round `round_` into every rank's mailbox.
@@ -187,6 +191,7 @@ class PeerMailbox:
             self.heartbeat.require(round_ - 1)
         M.mhc_mailbox_publish(x, self.rank, round_, self.ptrs, self.max_rows, stream)
         self.published = round_
+        self.rows[round_] = int(x.shape[0])
         if self.heartbeat is not None:
             self.heartbeat.beat(round_)
 
@@ -195,9 +200,13 @@ class PeerMailbox:
         if round_ != self.collected + 1 or round_ > self.published:
             raise RuntimeError(f"round {round_} collected out of order (last collected {self.collected}, "
                                f"last published {self.published})")
+        if int(residual.shape[0]) != self.rows[round_]:
+            raise RuntimeError(f"round {round_} collected over {int(residual.shape[0])} rows, "
+                               f"published over {self.rows[round_]}")
         M.mhc_boundary_collect(self.local, self.world, self.max_rows, round_, residual, post, comb, pre, norm_weight,
                                norm_eps, coeffs, residual_out, **kw)
         self.collected = round_
+        del self.rows[round_]
 
     def reset(self, stream=None):
         """Drop the rounds an aborted step left published but uncollected: every
@@ -210,6 +219,7 @@ class PeerMailbox:
         _sync(self.local.device)
         dist.barrier(group=self.group)
         self.published = self.collected = -1
+        self.rows = {}
         if self.heartbeat is not None:
             self.heartbeat.next_epoch()
 

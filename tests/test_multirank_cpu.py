@@ -224,7 +224,7 @@ def test_peer_mailbox_round_checks_and_reset(monkeypatch):
     try:
         hb = tp.Heartbeat(0, 1)
         box = tp.PeerMailbox(4, 64, heartbeat=hb)
-        x, args = torch.zeros(4, 64), (None,) * 8
+        x, args = torch.zeros(4, 64), (torch.zeros(4, 4, 64),) + (None,) * 7
         box.publish(x, 0)
         box.publish(x, 1)
         with pytest.raises(RuntimeError):
@@ -236,6 +236,8 @@ def test_peer_mailbox_round_checks_and_reset(monkeypatch):
         with pytest.raises(RuntimeError):
             box.publish(x, 4)          # round 3 skipped
         box.collect(1, *args)
+        with pytest.raises(RuntimeError):
+            box.collect(2, torch.zeros(3, 4, 64), *args[1:])  # 4 rows published, 3 collected
         box.collect(2, *args)
         with pytest.raises(RuntimeError):
             box.collect(3, *args)      # not published by this rank

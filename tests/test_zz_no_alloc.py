@@ -17,7 +17,8 @@ import torch
 from mhc_residual_stream_b200 import mhc as M
 from mhc_residual_stream_b200 import synthetic as S
 
-from _parity import DEV, alloc_outputs, assert_bf16_close, f64, gpu_post_pre, to_dev
+from _parity import (DEV, alloc_outputs, assert_bf16_close, assert_bf16_ulp, check_tail, f64, gpu_post_pre,
+                     oracle_post_pre, stream_terms, to_dev)
 
 
 def _noalloc(d):
@@ -50,6 +51,25 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
         assert np.array_equal(got["q_scale"].numpy(), ref["q_scale"].numpy()), what + " mxfp8 scales"
         for k in ("post", "comb", "pre"):
             assert np.max(np.abs(f64(got[k]) - f64(ref[k]))) <= 1e-5, what + " " + k
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("R", [32, 128])
+def test_noalloc_matches_the_oracle_at_full_size(R):
+    # rows 32 and 128 (the largest the scratch holds), H 7168, n 4, P 8: the streams
+    # and the layer input within the bf16 bounds, MXFP8 data and E8M0 scales
+    # bit-exact, the coefficients within 1e-5 of the oracle fed the GPU's streams
+    from mhc_residual_stream_b200 import build
+    build.build()
+    M.lib()
+    d = S.draw_boundary(R, 7168, n=4, partials=8, seed=7100 + R)
+    got = _noalloc(d)
+    orc = oracle_post_pre(d)
+    what = f"no-alloc rows {R}"
+    assert_bf16_close(f64(got["residual_out"]), orc["residual"], what + " streams")
+    assert_bf16_ulp(f64(got["residual_out"]), orc["residual"], what + " streams (ulp)",
+                    terms=stream_terms(f64(d["partials"]), f64(d["residual"]), f64(d["post"]), f64(d["comb"])))
+    check_tail(d, got, orc, what=what)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
