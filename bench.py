@@ -519,6 +519,35 @@ def reference(args):
     }), flush=True)
 
 
+def phases(args):
+    """Per-phase clock stamps of chained boundaries (a stamped copy of the library,
+    built into a temporary directory): one markdown table row per row count."""
+    from mhc_residual_stream_b200 import mhc as M
+    from mhc_residual_stream_b200 import phase_stamps as PS
+    M.LIB_PATH = PS.build_stamped()
+    L = M.lib()
+    device = torch.device("cuda", 0)
+    G = HIDDEN // 64
+    keys = [k for k, _ in PS.PHASES]
+    print("| rows | µs / boundary (stamped copy) | " + " | ".join(keys) + " |")
+    print("|---" * (len(keys) + 2) + "|")
+    for R in args.phases:
+        sets = [BoundarySet(R, 500 + i, device) for i in range(sets_for(R))]
+        ws = M.new_workspace(R, HIDDEN, HC, device)
+        graph = step_graph(sets, ws)
+        run_timed(graph, 3, args.warmup)
+        PS.reset(L)  # every block's ring starts with the timed replays
+        ms = run_timed(graph, args.steps, 0)
+        if M.mhc_get_device_status(ws) != M.OK:
+            raise RuntimeError(f"rows {R}: device status")
+        S, T = PS.read(L)
+        ph = PS.summary(S, T, G)
+        us = ms * 1000.0 / (args.steps * GRAPH_LEN)
+        print(f"| {R} | {us:.2f} | " + " | ".join("-" if ph[k] is None else f"{ph[k] / 1000:.2f}" for k in keys) + " |",
+              flush=True)
+        del sets, graph
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,12 +558,17 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--unpacked-fn", action="store_true",
                     help="pass fp32 fn (split into bf16 terms in every call) instead of the packed form")
+    ap.add_argument("--phases", type=int, nargs="+", metavar="ROWS",
+                    help="instead of the benchmark: per-phase clock stamps (µs after the streaming kernel's "
+                         "wait) of chained boundaries at these row counts, from a stamped copy of the library")
     args = ap.parse_args()
     global PACK_FN
     PACK_FN = not args.unpacked_fn
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.phases:
+        phases(args)
+    elif args.impl == "reference":
         reference(args)
     else:
         ours(args)

@@ -116,7 +116,7 @@ struct Params {
   // embedding of the first layer (whose identity pre-mix selects it)
   const __nv_bfloat16* tail_streams;
   int tail_broadcast;
-  int tail_layer_blocks;  // tail blocks that write the layer input (at most G, or 0)
+  int tail_layer_blocks;  // tail blocks that write the layer input (or 0)
   int tail_coeff_blocks;  // tail blocks that finish the coefficients of rows j, j + this, ...
   int tail_coeff_first;   // coefficient blocks take the tail's first block indices
   int extra_tx;  // test hook: 16-byte units the fn wait expects beyond what arrives
@@ -1364,13 +1364,18 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
     p.tail_streams = FRONT == kStreams ? p.residual : p.residual_out;
     p.tail_broadcast = 0;
   }
-  // layer-input blocks: one 256-column task per warp, at most G blocks; coefficient
-  // blocks run beside them, on the SMs those leave
+  // Coefficient blocks: as many as the SMs that G layer-input blocks leave (at
+  // most one per row). Layer-input blocks: one 256-column task per warp, as many
+  // blocks as fill the SMs twice (the tail runs two blocks an SM) beside the
+  // coefficient blocks; up to G of them start beside the streaming kernel, the
+  // rest as its blocks retire. Against at most G layer-input blocks (B200, us per
+  // boundary): 10.92 / 11.12 at 64 rows, 14.34 / 15.53 at 96, 16.93 / 18.20 at 128.
   const int tasks = p.R * ((G + 3) / 4);
   const int lb = (tasks + kWarps - 1) / kWarps;
-  p.tail_layer_blocks = p.do_layer ? (lb < G ? lb : G) : 0;
-  const int spare = sm_count() - p.tail_layer_blocks;
+  const int spare = sm_count() - (p.do_layer ? (lb < G ? lb : G) : 0);
   p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
+  const int lcap = 2 * sm_count() - p.tail_coeff_blocks;
+  p.tail_layer_blocks = p.do_layer ? (lb < lcap ? lb : lcap) : 0;
   p.tail_coeff_first = few_rows && p.R >= kCoeffFirstRows;
   return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>().total,
                     stream, p);
