@@ -9,7 +9,8 @@ the streaming kernel's first wait return of the same boundary, latest block
 unless marked median), averaged as medians over the boundaries in the ring.
 
 Streaming kernel events: 0 start, 1 before the wait, 2 after the wait, 3 mixes
-staged, 6 first row data in (block's warp 0), 4 all row pairs done, 5 end.
+staged, 7 tensor-map copies of the rows landed (staged form), 6 first row data
+in (block's warp 0), 4 all row pairs done, 5 end.
 Tail events: 0 start, 4 at the wait (layer blocks), 1 after the wait, 3 first
 layer task's data in (layer blocks) or records added up (coefficient blocks),
 4/5 Sinkhorn start / end (coefficient blocks), 6 end; word 7 holds the block
@@ -61,9 +62,9 @@ _STAMPS = [
      "  unsigned tslot = 0;\n  const unsigned long long t0s = mhc::gtimer();\n"
      "  if (tid == 0) {\n    tslot = atomicAdd(&mhc::g_seq_s[blockIdx.x], 1u) & 7u;\n"
      "    mhc::g_ts[tslot][blockIdx.x][0] = t0s;\n  }\n", True),
-    ("  // ---- 3. wait for the preceding kernel, let the next one launch, and read\n",
+    ("  griddep_wait();\n  griddep_launch_dependents();\n  PairLoads<N> cur;",
      "  if (tid == 0) mhc::g_ts[tslot][blockIdx.x][1] = mhc::gtimer();\n", False),
-    ("  // ---- 3. wait for the preceding kernel, let the next one launch, and read\n  griddep_wait();\n",
+    ("  griddep_wait();\n  griddep_launch_dependents();\n  PairLoads<N> cur;",
      "  if (tid == 0) mhc::g_ts[tslot][blockIdx.x][2] = mhc::gtimer();\n", True),
     ("  if (FRONT == kMoe && warp < npairs) load_pair<N, FRONT>(p, warp * 2 + rq, h0, e2p_s, cur);\n",
      "  if (tid == 0) mhc::g_ts[tslot][blockIdx.x][3] = mhc::gtimer();\n", True),
@@ -97,12 +98,23 @@ _STAMPS = [
 ]
 
 
+# stamps of code that only some forms of the kernel have: inserted where found
+_OPTIONAL = [
+    ("    if (!mbar_wait_bounded(sbar, 0, deadline)) record_error(status, MHC_ERR_DEVICE_TIMEOUT);\n",
+     "    if (tid == 0) mhc::g_ts[tslot][blockIdx.x][7] = mhc::gtimer();\n", True),
+]
+
+
 def instrument(src: str) -> str:
     """The kernel source with the stamps inserted (each anchor must occur once)."""
     head = "namespace mhc {\n\nconstexpr int kCols"
     if src.count(head) != 1:
         raise RuntimeError("kernel source layout changed: namespace anchor")
     src = src.replace(head, _PRE + "\n" + head, 1)
+    for anchor, code, after in _OPTIONAL:
+        if src.count(anchor) == 1:
+            i = src.index(anchor) + (len(anchor) if after else 0)
+            src = src[:i] + code + src[i:]
     for anchor, code, after in _STAMPS:
         if src.count(anchor) != 1:
             raise RuntimeError(f"kernel source layout changed: {anchor[:60]!r}")
@@ -149,6 +161,7 @@ def read(L: ctypes.CDLL):
 
 PHASES = [  # key, what
     ("prewait", "streaming: last block reaches its wait"),
+    ("staged_med", "streaming: tensor-map copies of the rows landed (median block; staged form only)"),
     ("mixes_med", "streaming: mixes staged (median block)"),
     ("data_med", "streaming: first rows' data in (median block)"),
     ("rows", "streaming: all row pairs post-mixed"),
@@ -177,6 +190,8 @@ def summary(S: np.ndarray, T: np.ndarray, G: int) -> dict:
         base = st[:, 2].min()
         out["prewait"].append(st[:, 1].max() - base)
         out["mixes_med"].append(int(np.median(st[:, 3])) - base)
+        if (st[:, 7] != 0).all():
+            out["staged_med"].append(int(np.median(st[:, 7])) - base)
         out["data_med"].append(int(np.median(st[:, 6])) - base)
         out["rows"].append(st[:, 4].max() - base)
         out["stream_end"].append(st[:, 5].max() - base)
