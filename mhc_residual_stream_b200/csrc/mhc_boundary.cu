@@ -1462,15 +1462,19 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
     p.tail_broadcast = 0;
   }
   // Coefficient blocks: as many as the SMs that G layer-input blocks leave (at
-  // most one per row). Layer-input blocks: one 256-column task per warp, as many
-  // blocks as fill the SMs twice (the tail runs two blocks an SM) beside the
-  // coefficient blocks; up to G of them start beside the streaming kernel, the
-  // rest as its blocks retire. Against at most G layer-input blocks (B200, us per
-  // boundary): 10.92 / 11.12 at 64 rows, 14.34 / 15.53 at 96, 16.93 / 18.20 at 128.
+  // most one per row), and at least one for every two rows (a block takes its
+  // rows' records one after the other: 14.02 / 14.53 us per boundary at 96 rows,
+  // 16.19 / 16.81 at 128 against the free SMs alone; one block per row, 17.31 at
+  // 128). Layer-input blocks: one 256-column task per warp, as many blocks as fill
+  // the SMs twice (the tail runs two blocks an SM) beside the coefficient
+  // blocks; up to G of them start beside the streaming kernel, the rest as its
+  // blocks retire. Against at most G layer-input blocks (B200, us per boundary):
+  // 10.92 / 11.12 at 64 rows, 14.34 / 15.53 at 96, 16.93 / 18.20 at 128.
   const int tasks = p.R * ((G + 3) / 4);
   const int lb = (tasks + kWarps - 1) / kWarps;
   const int spare = sm_count() - (p.do_layer ? (lb < G ? lb : G) : 0);
   p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
+  if (p.do_coeff && p.tail_coeff_blocks < (p.R + 1) / 2) p.tail_coeff_blocks = (p.R + 1) / 2;
   const int lcap = 2 * sm_count() - p.tail_coeff_blocks;
   p.tail_layer_blocks = p.do_layer ? (lb < lcap ? lb : lcap) : 0;
   p.tail_coeff_first = few_rows && p.R >= kCoeffFirstRows;
