@@ -1477,6 +1477,12 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   if (p.do_coeff && p.tail_coeff_blocks < (p.R + 1) / 2) p.tail_coeff_blocks = (p.R + 1) / 2;
   const int lcap = 2 * sm_count() - p.tail_coeff_blocks;
   p.tail_layer_blocks = p.do_layer ? (lb < lcap ? lb : lcap) : 0;
+  // Up to 4 rows the layer-input blocks are few (7 at 2 rows) and the swizzled
+  // scale buffer's padding (127 rows of zeros at 1 row) falls on them: 32 blocks
+  // share it (us per boundary, 32 / as many as the tasks need: 5.81 / 6.33 at 1
+  // row, 5.73 / 5.91 at 2, 5.81 / 5.89 at 4; at 8 rows it was slower, 6.19 / 5.94).
+  if (p.do_layer && p.q_data != nullptr && p.q_swizzled && p.R <= 4 && p.tail_layer_blocks < 32)
+    p.tail_layer_blocks = 32 < lcap ? 32 : lcap;
   p.tail_coeff_first = few_rows && p.R >= kCoeffFirstRows;
   return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>().total,
                     stream, p);
