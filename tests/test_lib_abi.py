@@ -187,3 +187,14 @@ def test_other_entry_points_host_checks(L):
     assert L.mhc_mailbox_init(a, 4100, None) == M.INVALID_ARG  # not whole 16-byte units
     assert L.mhc_workspace_init(None, 4096, None) == M.WORKSPACE
     assert L.mhc_get_device_status(None, None) == M.WORKSPACE
+
+
+def test_phase_stamps_apply_to_the_current_kernels():
+    # bench.py --phases instruments a copy of the kernel source at fixed anchors;
+    # every anchor must still be found once (the stamped copy is built on the GPU machine)
+    from mhc_residual_stream_b200 import build, phase_stamps
+    with open(build.SOURCES[0]) as f:
+        src = f.read()
+    out = phase_stamps.instrument(src)
+    assert out.count("mhc::g_ts[tslot]") >= 7 and out.count("mhc::g_tt[tslot]") >= 7
+    assert "mhc_phase_read" in out and "mhc_phase_reset" in out
