@@ -1421,9 +1421,14 @@ constexpr int kSmemLimit = 200 * 1024;
 // us per boundary): 7.84 against 8.26 at 32 rows, 6.84 against 7.05 at 16, 5.85
 // against 5.94 at 4; the largest split is slower from 48 rows on (10.23 against
 // 9.95 at 48, 11.6 against 10.9 at 64, 22.2 against 19.9 at 128), and at 2 rows
-// the coefficient blocks first are (6.20 against 6.07).
+// the coefficient blocks first are (6.20 against 6.07). The coefficient blocks
+// stay first up to kCoeffFirstMaxRows rows, without the largest split: 9.31 /
+// 9.64 / 10.09 / 10.73 / 12.95 against 9.53 / 9.82 / 10.59 / 11.04 / 13.15 at
+// 40 / 48 / 56 / 64 / 80 rows; from 96 rows on they are better last (14.07 /
+// 16.16 against 14.26 / 16.30 at 96 / 128).
 constexpr int kCoexistRows = 32;
 constexpr int kCoeffFirstRows = 4;
+constexpr int kCoeffFirstMaxRows = 80;
 template <typename Kern>
 bool allow_smem(Kern kern, int bytes, std::atomic<int>* configured) {
   int dev = 0;
@@ -1483,7 +1488,7 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   // row, 5.73 / 5.91 at 2, 5.81 / 5.89 at 4; at 8 rows it was slower, 6.19 / 5.94).
   if (p.do_layer && p.q_data != nullptr && p.q_swizzled && p.R <= 4 && p.tail_layer_blocks < 32)
     p.tail_layer_blocks = 32 < lcap ? 32 : lcap;
-  p.tail_coeff_first = few_rows && p.R >= kCoeffFirstRows;
+  p.tail_coeff_first = p.R >= kCoeffFirstRows && p.R <= kCoeffFirstMaxRows;
   return launch_pdl(boundary_tail_kernel<N>, p.tail_layer_blocks + p.tail_coeff_blocks, tail_layout<N>().total,
                     stream, p);
 }
