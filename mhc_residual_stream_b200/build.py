@@ -40,9 +40,9 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found: set CUDA_HOME or put nvcc on PATH")
 
 
-def source_digest() -> str:
+def source_digest(sources=None, headers=None) -> str:
     h = hashlib.sha256()
-    for f in SOURCES + HEADERS:
+    for f in (SOURCES if sources is None else sources) + (HEADERS if headers is None else headers):
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())
@@ -50,19 +50,21 @@ def source_digest() -> str:
     return h.hexdigest()
 
 
-def up_to_date() -> bool:
-    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
+def up_to_date(lib=LIB, sources=None, headers=None) -> bool:
+    stamp = lib + ".src-sha256"
+    if not (os.path.exists(lib) and os.path.exists(stamp)):
         return False
-    with open(STAMP) as f:
-        return f.read().strip() == source_digest()
+    with open(stamp) as f:
+        return f.read().strip() == source_digest(sources, headers)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libmhc.so unless it is up to date with the sources; return its path."""
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *SOURCES]
+def compile_shared(lib, sources, headers, force=False, verbose=False) -> str:
+    """Compile `sources` into the shared library `lib` unless its stamp matches
+    the sources and headers; return its path."""
+    if not force and up_to_date(lib, sources, headers):
+        return lib
+    tmp = lib + ".tmp"
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
@@ -71,11 +73,27 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr}")
     if verbose and res.stderr:
         print(res.stderr)
-    os.replace(tmp, LIB)
-    with open(STAMP, "w") as f:
-        f.write(source_digest())
-    return LIB
+    os.replace(tmp, lib)
+    with open(lib + ".src-sha256", "w") as f:
+        f.write(source_digest(sources, headers))
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libmhc.so unless it is up to date with the sources; return its path."""
+    return compile_shared(LIB, SOURCES, HEADERS, force, verbose)
+
+
+# The mailbox slot protocol's concurrency check (test infrastructure): one
+# cooperative kernel whose blocks play producers and a consumer at the same time.
+RACE_LIB = os.path.join(ROOT, "tests", "csrc", "libmhc_mailbox_race.so")
+RACE_SOURCES = [os.path.join(ROOT, "tests", "csrc", "mailbox_race.cu")]
+
+
+def build_race_check(force: bool = False, verbose: bool = False) -> str:
+    return compile_shared(RACE_LIB, RACE_SOURCES, HEADERS, force, verbose)
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build_race_check(force="--force" in sys.argv, verbose="-v" in sys.argv))

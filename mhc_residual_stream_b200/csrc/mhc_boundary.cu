@@ -253,20 +253,6 @@ __device__ __forceinline__ void load_pair(const Params& p, int r, int h0, const 
   }
 }
 
-// A mailbox slot's 4 elements as loaded, re-read until none is negative zero
-// (bounded: on timeout the status records it and the values are used as they are).
-__device__ __forceinline__ uint2 settle_slot(const __nv_bfloat16* src, uint2 v, long long deadline,
-                                             unsigned* status) {
-  while (has_neg_zero(v)) {
-    if (clock64() > deadline) {
-      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
-      break;
-    }
-    v = ld_volatile_v2(src);
-  }
-  return v;
-}
-
 // fn as three bf16 terms, f = hi + mid + lo to 2^-24: each bf16 x bf16 product is
 // exact in fp32, so three tensor-core products return the fp32 projection up to
 // the order of the fp32 additions.
@@ -1143,14 +1129,7 @@ __global__ void __launch_bounds__(256) mailbox_publish_kernel(const PublishParam
   __nv_bfloat16* slot = reinterpret_cast<__nv_bfloat16*>(mb + kMailboxHeader) +
                         ((static_cast<size_t>(par) * q.W + q.rank) * q.M + r) * q.H;
   const __nv_bfloat16* src = q.x + static_cast<size_t>(r) * q.H;
-  for (int k = threadIdx.x * 8; k < q.H; k += blockDim.x * 8) {
-    uint4 v = ld_nc_v4(src + k);
-    v.x = clear_neg_zero2(v.x);
-    v.y = clear_neg_zero2(v.y);
-    v.z = clear_neg_zero2(v.z);
-    v.w = clear_neg_zero2(v.w);
-    st_v4(slot + k, v);
-  }
+  mailbox_store_row(slot, src, q.H, threadIdx.x, blockDim.x);
 }
 
 // After a collect: the round is consumed, its parity's slots may be reused. If

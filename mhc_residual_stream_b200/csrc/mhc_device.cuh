@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/mhc.h"
+
 namespace mhc {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -174,6 +176,39 @@ __device__ __forceinline__ uint4 ld_v4(const void* p) {  // coherent (may alias 
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
   asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
+}
+
+// ---------------------------------------------------------------- mailbox slots
+
+// Producer side: one row of H bf16 (H a multiple of 8) into its slot with
+// 16-byte stores, negative zeros made positive; thread t of nt takes every
+// nt-th 8-element chunk. No fence and no flag follow: each element is its own
+// "written" mark.
+__device__ __forceinline__ void mailbox_store_row(__nv_bfloat16* slot, const __nv_bfloat16* src, int H, int t,
+                                                  int nt) {
+  for (int k = t * 8; k < H; k += nt * 8) {
+    uint4 v = ld_nc_v4(src + k);
+    v.x = clear_neg_zero2(v.x);
+    v.y = clear_neg_zero2(v.y);
+    v.z = clear_neg_zero2(v.z);
+    v.w = clear_neg_zero2(v.w);
+    st_v4(slot + k, v);
+  }
+}
+
+// Consumer side: a slot's 4 elements as loaded, re-read until none is negative
+// zero (bounded: on timeout the status records it and the values are used as
+// they are).
+__device__ __forceinline__ uint2 settle_slot(const __nv_bfloat16* src, uint2 v, long long deadline,
+                                             unsigned* status) {
+  while (has_neg_zero(v)) {
+    if (clock64() > deadline) {
+      record_error(status, MHC_ERR_DEVICE_TIMEOUT);
+      break;
+    }
+    v = ld_volatile_v2(src);
+  }
+  return v;
 }
 
 // ---------------------------------------------------------------- warp-level tensor core MMA
