@@ -533,6 +533,10 @@ def phases(args):
     print("|---" * (len(keys) + 2) + "|")
     for R in args.phases:
         sets = [BoundarySet(R, 500 + i, device) for i in range(sets_for(R))]
+        if args.shared_inputs:  # every boundary reads set 0's inputs and weights, which stay in L2
+            for s in sets[1:]:
+                s.partials, s.residual, s.coeffs = sets[0].partials, sets[0].residual, sets[0].coeffs
+                s.post, s.comb, s.pre, s.norm_weight = sets[0].post, sets[0].comb, sets[0].pre, sets[0].norm_weight
         ws = M.new_workspace(R, HIDDEN, HC, device)
         graph = step_graph(sets, ws)
         run_timed(graph, 3, args.warmup)
@@ -561,6 +565,9 @@ def main():
     ap.add_argument("--phases", type=int, nargs="+", metavar="ROWS",
                     help="instead of the benchmark: per-phase clock stamps (µs after the streaming kernel's "
                          "wait) of chained boundaries at these row counts, from a stamped copy of the library")
+    ap.add_argument("--shared-inputs", action="store_true",
+                    help="with --phases: every boundary reads the same inputs and weights, so that they stay in L2 "
+                         "(a bound on what the HBM traffic costs; not a benchmark of the workload)")
     args = ap.parse_args()
     global PACK_FN
     PACK_FN = not args.unpacked_fn
