@@ -255,32 +255,90 @@ def launch_floor_us(reps=20, graph_len=240):
     return statistics.median(times)
 
 
+E2E_INPUTS = ("partials", "residual", "post", "comb", "pre")
+E2E_OUTPUTS = ("residual_out", "layer_input", "q_data", "q_scale", "post_out", "comb_out", "pre_out")
+
+
+def _arena_views(like, keys, buf):
+    """Views of the uint8 buffer `buf` shaped like `like`'s tensors `keys`, each 256-byte aligned."""
+    views, off = {}, 0
+    for k in keys:
+        t = getattr(like, k)
+        nb = t.numel() * t.element_size()
+        views[k] = buf[off:off + nb].view(t.dtype).view(t.shape)
+        off += (nb + 255) // 256 * 256
+    return views
+
+
+def _arena_bytes(like, keys):
+    return sum((getattr(like, k).numel() * getattr(like, k).element_size() + 255) // 256 * 256 for k in keys)
+
+
 def e2e_time(bset, ws, steps, device):
-    """Per boundary through the C ABI with host buffers: pinned H2D copies of the step's inputs,
-    the launch, and the D2H read of every output, all inside the timed region."""
-    h_in = {k: getattr(bset, k).cpu().pin_memory() for k in ("partials", "residual", "post", "comb", "pre")}
-    outs = ("residual_out", "layer_input", "q_data", "q_scale", "post_out", "comb_out", "pre_out")
-    h_out = {k: torch.empty(getattr(bset, k).shape, dtype=getattr(bset, k).dtype).pin_memory() for k in outs}
-    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    """Per boundary through the C ABI with host buffers. Every step copies its inputs
+    (partials, streams, mixes) from one pinned host staging buffer to the device,
+    runs the boundary, and copies every output back into a pinned host buffer, all
+    inside the timed region. The inputs and outputs of a step live in one device
+    buffer each (two slots, used by alternate steps), so a step is one host-to-device
+    copy, the two kernels and one device-to-host copy; the copies run on their own
+    streams, so the next step's upload overlaps this step's boundary and download.
+    The weights stay resident, as they would in a model."""
+    import copy
+    nin, nout = _arena_bytes(bset, E2E_INPUTS), _arena_bytes(bset, E2E_OUTPUTS)
+    h_in = torch.empty(nin, dtype=torch.uint8).pin_memory()
+    for k, v in _arena_views(bset, E2E_INPUTS, h_in).items():
+        v.copy_(getattr(bset, k).cpu())
+    h_out = torch.empty(nout, dtype=torch.uint8).pin_memory()
+    slots = []
+    for _ in range(2):
+        b = copy.copy(bset)
+        d_in = torch.empty(nin, dtype=torch.uint8, device=device)
+        d_out = torch.empty(nout, dtype=torch.uint8, device=device)
+        for keys, buf in ((E2E_INPUTS, d_in), (E2E_OUTPUTS, d_out)):
+            for k, v in _arena_views(bset, keys, buf).items():
+                setattr(b, k, v)
+        slots.append((b, d_in, d_out))
+    main = torch.cuda.current_stream()
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    run_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    for ev in run_done + out_done:
+        ev.record(main)
+    for st in (s_in, s_run, s_out):
+        st.wait_stream(main)
 
-    def one():
-        for k, t in h_in.items():
-            getattr(bset, k).copy_(t, non_blocking=True)
-        bset.launch(ws)
-        for k, t in h_out.items():
-            t.copy_(getattr(bset, k), non_blocking=True)
+    def step(i):
+        j = i & 1
+        b, d_in, d_out = slots[j]
+        s_in.wait_event(run_done[j])  # the slot's inputs are free again
+        with torch.cuda.stream(s_in):
+            d_in.copy_(h_in, non_blocking=True)
+        in_done[j].record(s_in)
+        s_run.wait_event(in_done[j])
+        s_run.wait_event(out_done[j])  # the slot's outputs have been read out
+        with torch.cuda.stream(s_run):
+            b.launch(ws)
+        run_done[j].record(s_run)
+        s_out.wait_event(run_done[j])
+        with torch.cuda.stream(s_out):
+            h_out.copy_(d_out, non_blocking=True)
+        out_done[j].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(100):  # warm-up: the first copies from freshly pinned pages are slower
+        step(i)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(steps):
-        one()
-    end.record()
+    start.record(main)
+    for st in (s_in, s_run, s_out):
+        st.wait_stream(main)
+    for i in range(steps):
+        step(i)
+    for st in (s_in, s_run, s_out):
+        main.wait_stream(st)
+    end.record(main)
     torch.cuda.synchronize()
-    return start.elapsed_time(end) * 1000.0 / steps, h2d, d2h
+    return start.elapsed_time(end) * 1000.0 / steps, nin, nout
 
 
 def cpu_baseline(budget_s=12.0):
@@ -459,7 +517,7 @@ def ours(args):
         if M.mhc_get_device_status(loop.workspace) != M.OK:
             raise RuntimeError("decode loop device status")
 
-    e2e_us, h2d, d2h = e2e_time(sets[0], ws, min(200, max(10, args.steps)), device)
+    e2e_us, h2d, d2h = e2e_time(sets[0], ws, 200, device)
     e2e_us = max_over_ranks(e2e_us, world) / world
     result["e2e"] = {"value": round(e2e_us, 2), "unit": "µs/boundary", "h2d_bytes_per_step": h2d,
                      "d2h_bytes_per_step": d2h}
