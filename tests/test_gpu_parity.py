@@ -31,9 +31,10 @@ def _lib():
 
 # ---------------------------------------------------------------- partial-sum boundary
 
-def _case(R, H, n, P, seed, swizzled=True, mxfp8=True, coeff=True, affine=True, fn_std=0.01, part_std=0.05):
+def _case(R, H, n, P, seed, swizzled=True, mxfp8=True, coeff=True, affine=True, fn_std=0.01, part_std=0.05,
+          packed=False):
     d = S.draw_boundary(R, H, n=n, partials=P, seed=seed, fn_std=fn_std, affine=affine, part_std=part_std)
-    gpu = gpu_post_pre(d, mxfp8=mxfp8, swizzled=swizzled, coeff=coeff)
+    gpu = gpu_post_pre(d, mxfp8=mxfp8, swizzled=swizzled, coeff=coeff, packed=packed)
     orc = oracle_post_pre(d, mxfp8=mxfp8, swizzled=swizzled, coeff=coeff)
     what = f"R={R} H={H} n={n} P={P}"
     assert_bf16_close(f64(gpu["residual_out"]), orc["residual"], what + " residual")
@@ -63,6 +64,27 @@ def test_decode_attention_boundary_rows32_full_size():
 ])
 def test_boundary_shapes(R, H, n, P, swz):
     _case(R, H, n, P, seed=7000 + R * 7 + n, swizzled=swz)
+
+
+def _random_cases(count=40, seed=20261203):
+    """Seeded draws over the supported shape space: rows 1-128, H = 64 x 1-148
+    column blocks, n in {1, 2, 4}, 1-16 partials, both scale layouts, with and
+    without MXFP8 and coefficients, fp32 or packed fn, small or unit partials."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(count):
+        R = int(rng.choice([1, 2, 3, 4, 5, 8, 15, 16, 17, 31, 32, 33, 47, 48, 63, 64, 65, 96, 127, 128]))
+        G = int(rng.integers(1, 149))
+        cases.append((R, 64 * G, int(rng.choice([1, 2, 4])), int(rng.integers(1, 17)), bool(rng.integers(2)),
+                      bool(rng.integers(4) > 0), bool(rng.integers(4) > 0), bool(rng.integers(2)),
+                      float(rng.choice([0.05, 1.0])), 9000 + i))
+    return cases
+
+
+@pytest.mark.parametrize("R,H,n,P,swz,mxfp8,coeff,packed,part_std,seed", _random_cases())
+def test_boundary_random_shapes(R, H, n, P, swz, mxfp8, coeff, packed, part_std, seed):
+    _case(R, H, n, P, seed=seed, swizzled=swz, mxfp8=mxfp8, coeff=coeff, packed=packed and coeff,
+          part_std=part_std)
 
 
 def test_boundary_without_mxfp8_and_without_coefficients():
@@ -245,6 +267,30 @@ def test_moe_shapes_with_mxfp8(R, H, k, extra):
     assert_bf16_ulp(f64(gpu["residual_out"]), orc["residual"], f"moe R={R} H={H} k={k} residual (ulp)",
                     terms=_moe_terms(d))
     check_tail(d, gpu, orc, mxfp8=True, what="moe")
+
+
+def _random_moe_cases(count=16, seed=20261204):
+    """Seeded draws of MoE-finalize boundaries: rows 1-128, H = 64 x 1-148, n in
+    {1, 2, 4}, top_k 1-16, 0-64 permuted rows beyond rows x top_k, with and
+    without MXFP8, fp32 or packed fn."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(count):
+        R = int(rng.choice([1, 2, 3, 7, 8, 16, 31, 32, 33, 64, 65, 100, 128]))
+        cases.append((R, 64 * int(rng.integers(1, 149)), int(rng.choice([1, 2, 4])), int(rng.integers(1, 17)),
+                      int(rng.integers(0, 65)), bool(rng.integers(2)), bool(rng.integers(2)), 9500 + i))
+    return cases
+
+
+@pytest.mark.parametrize("R,H,n,k,extra,mxfp8,packed,seed", _random_moe_cases())
+def test_moe_random_shapes(R, H, n, k, extra, mxfp8, packed, seed):
+    d = S.draw_moe(R, H, n=n, top_k=k, seed=seed, extra_permuted=extra)
+    gpu, _ = _moe_gpu(d, mxfp8=mxfp8, packed=packed)
+    orc = _moe_oracle(d, mxfp8=mxfp8)
+    what = f"moe R={R} H={H} n={n} k={k}"
+    assert_bf16_close(f64(gpu["residual_out"]), orc["residual"], what + " residual")
+    assert_bf16_ulp(f64(gpu["residual_out"]), orc["residual"], what + " residual (ulp)", terms=_moe_terms(d))
+    check_tail(d, gpu, orc, mxfp8=mxfp8, what=what)
 
 
 def test_moe_gather_indexing_bit_exact():
