@@ -27,7 +27,13 @@ def pytest_collection_modifyitems(config, items):
 
 
 def pytest_terminal_summary(terminalreporter):
-    """The 1-ulp bf16 flips the parity checks counted (GPU runs only)."""
+    """The 1-ulp bf16 flips the parity checks counted, and how often the mailbox
+    consumer met unwritten slots in the concurrent rounds (GPU runs only)."""
+    race = sys.modules.get("test_gpu_mailbox_race")
+    waits = getattr(race, "WAITS", None) if race else None
+    if waits:
+        terminalreporter.write_line("mailbox rounds with producers running: " + "; ".join(
+            f"{c}: {w} of {n} slot groups first read unwritten" for c, w, n in waits))
     mod = sys.modules.get("_parity")
     flips = getattr(mod, "FLIPS", None) if mod else None
     if not flips:

@@ -31,6 +31,7 @@ from mhc_residual_stream_b200 import build
 
 NEG_ZERO = 0x8000
 DEVICE_TIMEOUT = 5  # MHC_ERR_DEVICE_TIMEOUT
+WAITS = []  # (case, 8-byte groups the consumer first loaded unwritten, groups read); printed after a GPU run
 
 
 def _lib():
@@ -104,6 +105,7 @@ def test_concurrent_round_is_exact(W, R, H, max_delay, seed):
     rng = np.random.default_rng(seed)
     delays = rng.integers(0, max_delay, size=(W, R)).astype(np.int32)
     got, status, slots = _run(L, x, delays, consumers=8, budget_ns=500_000_000)
+    WAITS.append((f"W={W} R={R} H={H}", int(status[1]), W * R * H // 4))
     assert status[0] == 0
     assert status[1] > 0, "the consumer never met an unwritten element: nothing ran concurrently"
     want = _expected(x)
