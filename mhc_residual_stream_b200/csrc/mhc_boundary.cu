@@ -52,6 +52,7 @@ constexpr int kMaxTopK = 16;
 constexpr int kMaxIters = 1000;
 constexpr int kMaxBlocks = 148;  // most H/64 blocks: the tail's per-lane loads are sized for it
 constexpr int kPrefetchRows = 64;  // the streaming kernel prefetches its rows into L2 up to this many
+constexpr int kPrefetchPartRows = 96;  // and its first kPrefetchRows rows up to this many
 // Workspace header: the status word (byte 0); the partial sums follow.
 constexpr size_t kWsHeader = 1024;
 constexpr int kStatusWord = 0;
@@ -339,13 +340,16 @@ __global__ void __maxnreg__(80) boundary_kernel(const __grid_constant__ Params p
   // ---- 2. bring this block's activations into L2 while the preceding kernel may
   // still run: a prefetch is only a hint and L2 is the point of coherence, so
   // it is safe before the wait; gather indices read now only steer prefetches.
-  // Up to 64 rows: past that the prefetches cost more than they save (us per
-  // boundary with / without, B200: 7.65 / 8.23 at 32 rows, 9.81 / 10.20 at 48,
-  // 15.79 / 15.45 at 96, 19.52 / 18.17 at 128).
-  if ((vec == 0 || vec == 15) && R <= kPrefetchRows) {
+  // Every row up to 64 rows; the first 64 rows up to 96 (the paired
+  // instantiation, which serves 49 rows and more); past that the prefetches
+  // cost more than they save (us per boundary with / without, B200: 7.65 / 8.23
+  // at 32 rows, 9.81 / 10.20 at 48; all 96 rows 15.79 / 15.45, the first 64 of
+  // 96 13.84 / 14.09; the first 64 of 128 16.27 / 16.02).
+  const int pf_rows = PAIRED ? (R <= kPrefetchRows ? R : (R <= kPrefetchPartRows ? kPrefetchRows : 0)) : R;
+  if ((vec == 0 || vec == 15) && (PAIRED ? pf_rows > 0 : R <= kPrefetchRows)) {
     for (int q = warp; q < npairs; q += kW1) {
       const int r = q * 2 + rq;
-      if (r >= R) break;
+      if (r >= pf_rows) break;
       if constexpr (FRONT == kBroadcast) {
         prefetch_l2(p.x + static_cast<size_t>(r) * H + h0);
       } else {
