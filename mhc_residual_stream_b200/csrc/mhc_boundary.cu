@@ -1463,9 +1463,10 @@ mhc_status launch_boundary(Params& p, cudaStream_t stream) {
   const int spare = sm_count() - (p.do_layer ? (lb < G ? lb : G) : 0);
   p.tail_coeff_blocks = p.do_coeff ? (p.R < spare ? p.R : (spare > 1 ? spare : 1)) : 0;
   if (p.do_coeff && p.tail_coeff_blocks < (p.R + 1) / 2) p.tail_coeff_blocks = (p.R + 1) / 2;
-  // up to 48 rows one coefficient block per row (9.08 / 9.46 against 9.29 / 9.53
-  // us at 40 / 48 rows; at 64 rows it was slower, 11.17 against 10.73)
-  if (p.do_coeff && p.R <= 48) p.tail_coeff_blocks = p.R;
+  // up to 56 rows one coefficient block per row (9.08 / 9.46 against 9.29 / 9.53
+  // us at 40 / 48 rows, 9.78 / 9.85 against 10.03 / 9.99 at 49 / 52; at 64 rows
+  // it was slower, 11.11 against 10.84)
+  if (p.do_coeff && p.R <= 56) p.tail_coeff_blocks = p.R;
   const int lcap = 2 * sm_count() - p.tail_coeff_blocks;
   p.tail_layer_blocks = p.do_layer ? (lb < lcap ? lb : lcap) : 0;
   // Up to 4 rows the layer-input blocks are few (7 at 2 rows) and the swizzled
