@@ -386,6 +386,53 @@ def test_first_layer_broadcast(R):
                         "first-layer coefficients")
 
 
+def _random_entry_cases(count, seed):
+    rng = np.random.default_rng(seed)
+    return [(int(rng.choice([1, 2, 3, 5, 8, 16, 17, 32, 33, 48, 64, 97, 128])), 64 * int(rng.integers(1, 149)),
+             int(rng.choice([1, 2, 4])), bool(rng.integers(2)), 9700 + i) for i in range(count)]
+
+
+@pytest.mark.parametrize("R,H,n,with_layer,seed", _random_entry_cases(10, 20261205))
+def test_first_layer_broadcast_random_shapes(R, H, n, with_layer, seed):
+    """Seeded draws of the first-layer entry: streams bitwise x, identity pre-mix."""
+    d = S.draw_first_layer(R, H, n=n, seed=seed)
+    out = alloc_outputs(R, n, H, False, True, True)
+    ws = M.new_workspace(R, H, n, DEV)
+    M.mhc_coeffs(M.Coeffs.from_weights(d["coeff"], DEV), out["post"], out["comb"], out["pre"], x=d["x"].to(DEV),
+                 residual_out=out["residual_out"], norm_weight=d["norm_weight"].to(DEV) if with_layer else None,
+                 norm_eps=d["norm_eps"], layer_input=out["layer_input"] if with_layer else None, workspace=ws)
+    torch.cuda.synchronize()
+    assert M.mhc_get_device_status(ws) == M.OK
+    assert torch.equal(out["residual_out"].cpu(), d["x"][:, None, :].expand(R, n, H))
+    o = O.coeffs_entry(x=f64(d["x"]), hc_mult=n, norm_weight=f64(d["norm_weight"]), norm_eps=d["norm_eps"],
+                       coeff=coeff_np(d["coeff"]))
+    if with_layer:
+        assert_bf16_close(f64(out["layer_input"]), o["layer_input"], f"broadcast R={R} H={H} n={n} layer input")
+    assert_coeffs_close({k: out[k].cpu() for k in ("post", "comb", "pre")}, o["post"], o["comb"], o["pre"],
+                        f"broadcast R={R} H={H} n={n} coefficients")
+
+
+@pytest.mark.parametrize("R,H,n,with_layer,seed", _random_entry_cases(10, 20261206))
+def test_coeffs_on_given_streams_random_shapes(R, H, n, with_layer, seed):
+    """Seeded draws of the coefficients entry on given streams (Engram-entry form)."""
+    d = S.draw_boundary(R, H, n=n, partials=1, seed=seed)
+    g = to_dev(d)
+    out = alloc_outputs(R, n, H, False, True, True)
+    ws = M.new_workspace(R, H, n, DEV)
+    M.mhc_coeffs(M.Coeffs.from_weights(d["coeff"], DEV), out["post"], out["comb"], out["pre"],
+                 residual=g["residual"], pre_mix=g["pre"] if with_layer else None,
+                 norm_weight=g["norm_weight"] if with_layer else None, norm_eps=d["norm_eps"],
+                 layer_input=out["layer_input"] if with_layer else None, workspace=ws)
+    torch.cuda.synchronize()
+    assert M.mhc_get_device_status(ws) == M.OK
+    o = O.coeffs_entry(residual=f64(d["residual"]), pre_mix=f64(d["pre"]), norm_weight=f64(d["norm_weight"]),
+                       norm_eps=d["norm_eps"], coeff=coeff_np(d["coeff"]))
+    what = f"coeffs R={R} H={H} n={n}"
+    assert_coeffs_close({k: out[k].cpu() for k in ("post", "comb", "pre")}, o["post"], o["comb"], o["pre"], what)
+    if with_layer:
+        assert_bf16_close(f64(out["layer_input"]), o["layer_input"], what + " layer input")
+
+
 # ---------------------------------------------------------------- standalone MXFP8
 
 def _mxfp8_inputs(R, H, seed):

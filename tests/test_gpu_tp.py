@@ -51,6 +51,18 @@ def test_partial_table_matches_strided_bitwise(R, H, n, P):
         assert torch.equal(v.cpu(), ref[k]), k
 
 
+def _random_table_cases(count=8, seed=20261207):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    return [(int(rng.choice([1, 2, 4, 9, 16, 17, 32, 64, 100, 128])), 64 * int(rng.integers(1, 149)),
+             int(rng.choice([1, 2, 4])), int(rng.integers(1, 17))) for _ in range(count)]
+
+
+@pytest.mark.parametrize("R,H,n,P", _random_table_cases())
+def test_partial_table_random_shapes(R, H, n, P):
+    test_partial_table_matches_strided_bitwise(R, H, n, P)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
