@@ -341,12 +341,13 @@ __global__ void __maxnreg__(80) boundary_kernel(const __grid_constant__ Params p
   // still run: a prefetch is only a hint and L2 is the point of coherence, so
   // it is safe before the wait; gather indices read now only steer prefetches.
   // Every row up to 64 rows; the first 64 rows up to 96 (the paired
-  // instantiation, which serves 49 rows and more); past that the prefetches
+  // instantiation, which serves 49 rows and more, except the MoE gathers); past that the prefetches
   // cost more than they save (us per boundary with / without, B200: 7.65 / 8.23
   // at 32 rows, 9.81 / 10.20 at 48; all 96 rows 15.79 / 15.45, the first 64 of
   // 96 13.84 / 14.09; the first 64 of 128 16.27 / 16.02).
-  const int pf_rows = PAIRED ? (R <= kPrefetchRows ? R : (R <= kPrefetchPartRows ? kPrefetchRows : 0)) : R;
-  if ((vec == 0 || vec == 15) && (PAIRED ? pf_rows > 0 : R <= kPrefetchRows)) {
+  constexpr bool kPart = PAIRED && FRONT != kMoe;  // (the gathers keep the 64-row limit)
+  const int pf_rows = kPart ? (R <= kPrefetchRows ? R : (R <= kPrefetchPartRows ? kPrefetchRows : 0)) : R;
+  if ((vec == 0 || vec == 15) && (kPart ? pf_rows > 0 : R <= kPrefetchRows)) {
     for (int q = warp; q < npairs; q += kW1) {
       const int r = q * 2 + rq;
       if (r >= pf_rows) break;
