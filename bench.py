@@ -282,7 +282,8 @@ def e2e_time(bset, ws, steps, device):
     buffer each (two slots, used by alternate steps), so a step is one host-to-device
     copy, the two kernels and one device-to-host copy; the copies run on their own
     streams, so the next step's upload overlaps this step's boundary and download.
-    The weights stay resident, as they would in a model. Median of three timed runs."""
+    The weights stay resident, as they would in a model. Median of three timed runs;
+    also returns the last step's downloaded outputs (views of the host buffer)."""
     import copy
     nin, nout = _arena_bytes(bset, E2E_INPUTS), _arena_bytes(bset, E2E_OUTPUTS)
     h_in = torch.empty(nin, dtype=torch.uint8).pin_memory()
@@ -341,7 +342,7 @@ def e2e_time(bset, ws, steps, device):
         end.record(main)
         torch.cuda.synchronize()
         runs.append(start.elapsed_time(end) * 1000.0 / steps)
-    return statistics.median(runs), nin, nout
+    return statistics.median(runs), nin, nout, _arena_views(bset, E2E_OUTPUTS, h_out)
 
 
 def cpu_baseline(budget_s=12.0):
@@ -520,7 +521,7 @@ def ours(args):
         if M.mhc_get_device_status(loop.workspace) != M.OK:
             raise RuntimeError("decode loop device status")
 
-    e2e_us, h2d, d2h = e2e_time(sets[0], ws, 200, device)
+    e2e_us, h2d, d2h, _ = e2e_time(sets[0], ws, 200, device)
     e2e_us = max_over_ranks(e2e_us, world) / world
     result["e2e"] = {"value": round(e2e_us, 2), "unit": "µs/boundary", "h2d_bytes_per_step": h2d,
                      "d2h_bytes_per_step": d2h}

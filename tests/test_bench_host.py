@@ -1,9 +1,11 @@
 """Host-side arithmetic of the benchmark (no GPU): the algorithmic byte count the
 roofline divides by, the rotation that keeps inputs out of L2, and the staging
-buffers of the end-to-end measurement."""
+buffers of the end-to-end measurement; on a GPU, that the end-to-end loop
+downloads what the boundary computes."""
 
 import types
 
+import pytest
 import torch
 
 import bench
@@ -62,3 +64,20 @@ def test_end_to_end_staging_views_are_aligned_and_disjoint():
         views[k].fill_(i + 1)
     for i, k in enumerate(keys):
         assert torch.all(views[k] == i + 1)
+
+
+@pytest.mark.gpu
+def test_end_to_end_steps_download_the_boundary_outputs():
+    """The end-to-end loop (uploads, boundaries and downloads on three streams,
+    two device slots) hands back bitwise the outputs of a direct call."""
+    from mhc_residual_stream_b200 import mhc as M
+    dev = torch.device("cuda", 0)
+    b = bench.BoundarySet(4, 4242, dev)
+    ws = M.new_workspace(4, bench.HIDDEN, bench.HC, dev)
+    _, nin, nout, got = bench.e2e_time(b, ws, 5, dev)
+    assert nin == bench._arena_bytes(b, bench.E2E_INPUTS) and nout == bench._arena_bytes(b, bench.E2E_OUTPUTS)
+    b.launch(ws)
+    torch.cuda.synchronize()
+    assert M.mhc_get_device_status(ws) == M.OK
+    for k in bench.E2E_OUTPUTS:
+        assert torch.equal(got[k], getattr(b, k).cpu()), k
